@@ -1,0 +1,416 @@
+"""Decode-step benchmark: tok/s and fraction of the B200 HBM roofline.
+
+Default workload: the 30B-MoE shape at batch 1 with an 8192-token paged KV
+cache and near-uniform routing (one decode step = one launch of the
+persistent interpreter).  ``--workload`` selects another preset.  Under
+torchrun every rank runs an independent replica on its own GPU (the decode
+step does not shard: replicas only); rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the reference arm) on a bounded
+sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s at batch 1 and 8 (30B-MoE shape); % of B200 HBM roofline"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_PATH) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(name, wl, lens):
+    s = wl["shape"]
+    return (f"{name}: {s['n_layers']}L d{s['d_model']} {s['n_q_heads']}q/{s['n_kv_heads']}kv "
+            f"hd{s['head_dim']} E{s['n_experts']} top{s['top_k']} F{s['d_ff']} V{s['vocab']}, "
+            f"batch {wl['batch']}, paged KV 64-token pages, cached lengths "
+            f"{lens if len(lens) <= 8 else str(lens[:8]) + '...'}, {wl.get('routing')} routing")
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mk_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        except Exception:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+class OracleSample:
+    """The oracle on a bounded sample of one step: the first n_layers layers
+    (every expert of those layers and their KV pages copied to host memory
+    beforehand, untimed) plus lm_rows rows of the LM head."""
+
+    def __init__(self, shape, W, k, v, table, n_layers, lm_rows):
+        import numpy as np
+        from tests.oracle_io import u16
+        self.shape, self.table, self.n_layers, self.lm_rows = shape, table, n_layers, lm_rows
+        L = n_layers
+        self.c = {key: [u16(W[key][l]) for l in range(L)]
+                  for key in ("attn_norm", "w_qkv", "w_o", "w_router")}
+        self.exp = {(l, e): tuple(u16(W[kk][l][e]) for kk in ("w_gate", "w_up", "w_down"))
+                    for l in range(L) for e in range(shape["n_experts"])}
+        self.rb = W.get("router_bias")
+        self.emb = W["embed"]
+        self.fn = u16(W["final_norm"])
+        self.lm = u16(W["lm_head"][:lm_rows])
+        self.kp = {(l, "k"): u16(k[l]) for l in range(L)}
+        self.kp.update({(l, "v"): u16(v[l]) for l in range(L)})
+        self.np = np
+
+    # weight accessor protocol
+    def embed_row(self, t):
+        from tests.oracle_io import u16
+        return u16(self.emb[t])
+
+    def lm_head_rows(self, r0, r1):
+        return self.lm[r0:r1]
+
+    def final_norm(self):
+        return self.fn
+
+    def attn_norm(self, l):
+        return self.c["attn_norm"][l]
+
+    def w_qkv(self, l):
+        return self.c["w_qkv"][l]
+
+    def w_o(self, l):
+        return self.c["w_o"][l]
+
+    def w_router(self, l):
+        return self.c["w_router"][l]
+
+    def router_bias(self, l):
+        return None if self.rb is None else self.rb[l].float().cpu().numpy()
+
+    def expert(self, l, e):
+        return self.exp[(l, e)]
+
+    # KV accessor protocol
+    def pages(self, l, kind, ids):
+        return self.kp[(l, kind)][self.np.asarray(ids, dtype=self.np.int64)]
+
+    def run(self, tokens, lens):
+        """Returns (extrapolated seconds for a full step, measured seconds)."""
+        import oracle
+        from tests.oracle_io import oracle_shape
+        np = self.np
+        S = oracle_shape(self.shape)
+        t0 = time.perf_counter()
+        oracle.decode_step(S, self, self, tokens, lens, self.table, layers=self.n_layers)
+        t1 = time.perf_counter()
+        xf = np.ones(self.shape["d_model"])
+        for _ in range(len(tokens)):
+            oracle.bf16_bits_to_f64(self.lm_head_rows(0, self.lm_rows)) @ xf
+        t2 = time.perf_counter()
+        full = ((t1 - t0) / self.n_layers * self.shape["n_layers"]
+                + (t2 - t1) * self.shape["vocab"] / self.lm_rows)
+        return full, t2 - t0
+
+    def describe(self):
+        return (f"oracle (float64 numpy) on {self.n_layers} of {self.shape['n_layers']} layers "
+                f"and {self.lm_rows} of {self.shape['vocab']} LM-head rows of one step, "
+                f"scaled to a full step (weights and KV copied to host memory untimed)")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference", "unfused"])
+    ap.add_argument("--workload", default="moe30b_b1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-layers", type=int, default=2)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import torch
+    from moe_persistent_cta_b200 import configs, synth
+
+    wl = configs.WORKLOADS[args.workload]
+    shape = wl["shape"]
+    B = wl["batch"]
+    lens = synth.seq_lengths(wl["seq_lens"], B)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        run_reference(args, wl, shape, lens)
+        return 0
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        import datetime
+        dist = dist_mod
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from moe_persistent_cta_b200 import engine, mk, roofline
+
+    steps_total = args.warmup + args.steps
+    growth = max(64, steps_total + 1)
+    table, n_pages = synth.make_page_tables(lens, wl.get("contiguous", False), wl["page_seed"],
+                                            growth=growth)
+    W = synth.make_weights(shape, wl["weight_seed"], str(dev), wl.get("routing", "uniform"),
+                           wl.get("zipf_s", 1.1))
+    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], str(dev))
+    dec = engine.Decoder(shape, W, k, v, max_batch=B, device=dev.index)
+    plan_len = [s + steps_total + 1 for s in lens]
+    dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
+
+    # all steps' inputs staged in HBM before timing: step s feeds a seeded
+    # token at position len + s
+    gen = torch.Generator(device="cpu").manual_seed(wl["token_seed"])
+    toks = torch.randint(0, shape["vocab"], (steps_total, B), generator=gen, dtype=torch.int32)
+    pos = torch.tensor([[s + i for s in lens] for i in range(steps_total)], dtype=torch.int32)
+    toks_d, pos_d = toks.to(dev), pos.to(dev)
+    table_d = table.to(dev)
+    logits = torch.empty((B, shape["vocab"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    unfused = args.impl == "unfused"
+
+    def run(i):
+        dec.step(toks_d[i], pos_d[i], table_d, pos_d[i], logits, stream=stream, unfused=unfused)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            run(i)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    nslots = dec.debug(mk.MK_BUF_NSLOTS)
+
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.warmup, steps_total):
+        run(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    dec.check_ok()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    tok_s = world * B * args.steps / (ms / 1e3)
+
+    # roofline of the step (the one kernel): algorithmic bytes per launch
+    mid_lens = [s + args.warmup + args.steps // 2 for s in lens]
+    sb = roofline.step_bytes(shape, mid_lens, [int(u) for u in nslots])
+    peak, peak_kind = hbm_peak()
+    achieved = sb["total"] / (ms_per_step / 1e3) / 1e9
+
+    # end to end through the public API with host buffers: per step the
+    # inputs go host->device from pinned memory and the logits come back
+    h_toks = toks.pin_memory()
+    h_pos = pos.pin_memory()
+    h_table = table.pin_memory()
+    h_logits = torch.empty((B, shape["vocab"]), dtype=torch.float32).pin_memory()
+    d_tok = torch.empty(B, dtype=torch.int32, device=dev)
+    d_pos = torch.empty(B, dtype=torch.int32, device=dev)
+    e2e_steps = args.steps
+    dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            d_tok.copy_(h_toks[i], non_blocking=True)
+            d_pos.copy_(h_pos[i], non_blocking=True)
+            table_d.copy_(h_table, non_blocking=True)
+            dec.step(d_tok, d_pos, table_d, d_pos, logits, stream=stream, unfused=unfused)
+            h_logits.copy_(logits, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_tok_s = world * B * e2e_steps / (e2e_ms / 1e3)
+    h2d = (B * 4) * 2 + table.numel() * 4
+    d2h = B * shape["vocab"] * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(shape, W, k, v, table.numpy(), args.oracle_layers, 4096)
+        full_s, measured_s = smp.run([int(t) for t in toks[0]], lens)
+        cpu = {"value": B / full_s, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": smp.describe(), "sample_seconds": round(measured_s, 2)}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC,
+            "value": tok_s,
+            "unit": "tok/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded bf16 weights ~N(0,0.02), KV ~N(0,1), random tokens)",
+            "config": {"workload": workload_desc(args.workload, wl, lens), "batch": B,
+                       "global_batch": B * world,
+                       "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (weights+KV streamed per step >> 126 MB)",
+                       "impl": "unfused per-op launches" if unfused else "fused megakernel",
+                       "experts_per_layer_mean": float(sum(nslots) / len(nslots))},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind,
+                         "bytes_per_step": sb["total"], "weight_bytes": sb["weights"],
+                         "kv_bytes": sb["kv"],
+                         "frac_of_8tbs_spec": achieved / 8000.0},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_tok_s, "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (1 if not unfused else
+                                          sum(1 for n in dec_phase_counts(dec) if n)),
+            "clocks": clk,
+        }
+        print(json.dumps(out))
+    dec.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def dec_phase_counts(dec):
+    # phases with tasks (one launch each in the unfused path)
+    L = dec.L
+    return [1] * (8 * L + 2)
+
+
+def run_reference(args, wl, shape, lens):
+    """Reference arm: the CPU oracle as it stands, timed on the host cores on
+    a bounded sample of the workload per step."""
+    import torch
+    from moe_persistent_cta_b200 import synth
+    B = wl["batch"]
+    table, n_pages = synth.make_page_tables(lens, wl.get("contiguous", False), wl["page_seed"])
+    W = synth.make_weights(shape, wl["weight_seed"], "cuda" if torch.cuda.is_available() else
+                           "cpu", wl.get("routing", "uniform"), wl.get("zipf_s", 1.1))
+    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], "cuda" if torch.cuda.is_available()
+                         else "cpu")
+    toks = synth.make_tokens(B, shape["vocab"], wl["token_seed"])
+    times = []
+    smp = OracleSample(shape, W, k, v, table.numpy(), 1, 2048)
+    desc = smp.describe()
+    for i in range(args.warmup + args.steps):
+        full_s, _ = smp.run(toks, lens)
+        if i >= args.warmup:
+            times.append(full_s)
+    mean_s = sum(times) / len(times)
+    value = B / mean_s
+    out = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": workload_desc(args.workload, wl, lens), "batch": B},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    sys.exit(main())

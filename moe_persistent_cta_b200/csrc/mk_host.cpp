@@ -1,0 +1,574 @@
+// mk_host.cpp -- the C ABI: context creation (validation, TMA tensor maps,
+// context-owned device memory), schedule upload, step launches, status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream);
+cudaError_t max_coresident(int smem_bytes, int* blocks_per_sm);
+}  // namespace mk
+
+using mk::Params;
+using mk::Plan;
+using mk::Shape;
+using mk::SmemLayout;
+
+struct DevBuf {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+struct mk_ctx {
+  int device = 0;
+  int n_sms = 0;
+  mk_config cfg{};
+  Shape shape{};
+  int r_qkv = 16, r_ff = 16;
+  // model pointers (device) kept from mk_create
+  const void* embed = nullptr;
+  const void* lm_head = nullptr;
+  const void* final_norm = nullptr;
+  // context-owned device memory
+  void* d_tmaps = nullptr;
+  void** d_attn_norm = nullptr;
+  void** d_router_bias = nullptr;
+  void** d_kpool = nullptr;
+  void** d_vpool = nullptr;
+  double* d_inv_freq = nullptr;
+  int32_t* d_status = nullptr;
+  uint32_t* d_counters = nullptr;
+  int counters_cap = 0;
+  DevBuf desc, ntasks, phase_desc, phase_counts;
+  DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, route, expert_a, afrag,
+      moe_part;
+  // schedule
+  bool have_schedule = false;
+  Plan plan;
+  SmemLayout sl{};
+  int B = 0, S = 0, max_chunks = 1, max_pages = 0;
+  std::vector<int> phase_tasks;  // tasks per phase (0: skip the launch)
+  uint32_t epoch = 0;
+  unsigned long long timeout_ns = 2000ull * 1000ull * 1000ull;
+  cudaStream_t last_stream = nullptr;
+  Params base{};
+};
+
+namespace {
+
+mk_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MK_OK;
+  if (e == cudaErrorMemoryAllocation) return MK_ERR_OOM;
+  return MK_ERR_CUDA;
+}
+
+#define MK_TRY(expr)                        \
+  do {                                      \
+    mk_status _s = (expr);                  \
+    if (_s != MK_OK) return _s;             \
+  } while (0)
+#define MK_CUDA(expr) MK_TRY(from_cuda(expr))
+
+mk_status ensure(DevBuf& b, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  if (b.bytes >= bytes) return MK_OK;
+  if (b.ptr) cudaFree(b.ptr);
+  b.ptr = nullptr;
+  b.bytes = 0;
+  MK_CUDA(cudaMalloc(&b.ptr, bytes));
+  b.bytes = bytes;
+  return MK_OK;
+}
+
+void release(DevBuf& b) {
+  if (b.ptr) cudaFree(b.ptr);
+  b.ptr = nullptr;
+  b.bytes = 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2D bf16 view [outer][inner], box {64, box_rows}, 128-byte swizzle: each
+// box row is one 128-byte line, matching the ldmatrix addressing of the
+// tile routines.
+mk_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                    uint32_t box_rows) {
+  auto fn = get_encoder();
+  if (!fn) return MK_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MK_OK : MK_ERR_INVALID;
+}
+
+int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mk_strerror(mk_status s) {
+  switch (s) {
+    case MK_OK: return "ok";
+    case MK_ERR_INVALID: return "invalid argument";
+    case MK_ERR_CUDA: return "CUDA error";
+    case MK_ERR_OOM: return "out of device memory";
+    case MK_ERR_TIMEOUT: return "device wait exceeded its deadline";
+    case MK_ERR_CAPACITY: return "request exceeds capacity";
+    case MK_ERR_STATE: return "call out of order or schedule outgrown";
+    case MK_ERR_DEVICE: return "device-side validation failed";
+  }
+  return "unknown status";
+}
+
+void mk_destroy(mk_ctx* c) {
+  if (!c) return;
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  cudaFree(c->d_tmaps);
+  cudaFree(c->d_attn_norm);
+  cudaFree(c->d_router_bias);
+  cudaFree(c->d_kpool);
+  cudaFree(c->d_vpool);
+  cudaFree(c->d_inv_freq);
+  cudaFree(c->d_status);
+  cudaFree(c->d_counters);
+  for (DevBuf* b : {&c->desc, &c->ntasks, &c->phase_desc, &c->phase_counts, &c->x, &c->actA,
+                    &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
+                    &c->rlogits, &c->route, &c->expert_a, &c->afrag, &c->moe_part})
+    release(*b);
+  c->plan.release();
+  delete c;
+}
+
+mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ctx** out) {
+  if (!out) return MK_ERR_INVALID;
+  *out = nullptr;
+  if (!cfg || !t) return MK_ERR_INVALID;
+  Shape s{cfg->n_layers, cfg->d_model, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+          cfg->n_experts, cfg->top_k, cfg->d_ff, cfg->vocab, cfg->page_size,
+          cfg->max_batch, cfg->n_pages, cfg->rope_theta, cfg->rms_eps};
+  MK_TRY((mk_status)mk::validate_shape(s));
+  const int L = s.L;
+  if (!t->embed || !t->lm_head || !t->final_norm || !t->attn_norm || !t->w_qkv || !t->w_o ||
+      !t->w_router || !t->w_gate || !t->w_up || !t->w_down || !t->k_pool || !t->v_pool)
+    return MK_ERR_INVALID;
+  for (int l = 0; l < L; ++l) {
+    const void* ps[] = {t->attn_norm[l], t->w_qkv[l], t->w_o[l], t->w_router[l], t->w_gate[l],
+                        t->w_up[l], t->w_down[l], t->k_pool[l], t->v_pool[l]};
+    for (const void* p : ps)
+      if (!p || !aligned16(p)) return MK_ERR_INVALID;
+    if (t->router_bias && t->router_bias[l] && !aligned16(t->router_bias[l])) return MK_ERR_INVALID;
+  }
+  if (!aligned16(t->embed) || !aligned16(t->lm_head) || !aligned16(t->final_norm))
+    return MK_ERR_INVALID;
+  int ndev = 0;
+  MK_CUDA(cudaGetDeviceCount(&ndev));
+  if (device < 0 || device >= ndev) return MK_ERR_INVALID;
+  MK_CUDA(cudaSetDevice(device));
+
+  mk_ctx* c = new mk_ctx();
+  c->device = device;
+  c->cfg = *cfg;
+  c->shape = s;
+  c->r_qkv = mk::gemv_rows_for(s.d, 1);
+  c->r_ff = mk::gemv_rows_for(s.d, 2);
+  c->embed = t->embed;
+  c->lm_head = t->lm_head;
+  c->final_norm = t->final_norm;
+  auto fail = [&](mk_status st) {
+    mk_destroy(c);
+    return st;
+  };
+  if (cudaDeviceGetAttribute(&c->n_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return fail(MK_ERR_CUDA);
+
+  // tensor maps
+  const int nmaps = L * mk::kMapsPerLayer + 1;
+  std::vector<CUtensorMap> maps(nmaps);
+  std::memset(maps.data(), 0, sizeof(CUtensorMap) * nmaps);
+  const int G = s.Hq / s.Hkv;
+  const uint64_t qkvR = (uint64_t)(s.Hq + 2 * s.Hkv) * s.hd;
+  for (int l = 0; l < L; ++l) {
+    CUtensorMap* m = &maps[l * mk::kMapsPerLayer];
+    mk_status st;
+    if ((st = encode_2d(m + 0, t->w_qkv[l], s.d, qkvR, c->r_qkv)) != MK_OK) return fail(st);
+    if ((st = encode_2d(m + 1, t->w_o[l], (uint64_t)s.Hq * s.hd, s.d, 64)) != MK_OK) return fail(st);
+    if ((st = encode_2d(m + 2, t->w_router[l], s.d, s.E, c->r_qkv)) != MK_OK) return fail(st);
+    if ((st = encode_2d(m + 3, t->w_gate[l], s.d, (uint64_t)s.E * s.F, c->r_ff)) != MK_OK)
+      return fail(st);
+    if ((st = encode_2d(m + 4, t->w_up[l], s.d, (uint64_t)s.E * s.F, c->r_ff)) != MK_OK)
+      return fail(st);
+    if ((st = encode_2d(m + 5, t->w_down[l], s.F, (uint64_t)s.E * s.d, 64)) != MK_OK)
+      return fail(st);
+    const uint64_t kvrows = (uint64_t)s.n_pages * s.Hkv * mk::kPage;
+    if ((st = encode_2d(m + 6, t->k_pool[l], s.hd, kvrows, 64)) != MK_OK) return fail(st);
+    if ((st = encode_2d(m + 7, t->v_pool[l], s.hd, kvrows, 64)) != MK_OK) return fail(st);
+  }
+  {
+    mk_status st = encode_2d(&maps[L * mk::kMapsPerLayer], t->lm_head, s.d, s.V, 128);
+    if (st != MK_OK) return fail(st);
+  }
+  (void)G;
+  if (cudaMalloc(&c->d_tmaps, sizeof(CUtensorMap) * nmaps) != cudaSuccess) return fail(MK_ERR_OOM);
+  if (cudaMemcpy(c->d_tmaps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return fail(MK_ERR_CUDA);
+
+  // per-layer pointer arrays
+  std::vector<void*> an(L), rb(L, nullptr), kp(L), vp(L);
+  for (int l = 0; l < L; ++l) {
+    an[l] = const_cast<void*>(t->attn_norm[l]);
+    if (t->router_bias) rb[l] = const_cast<float*>(t->router_bias[l]);
+    kp[l] = t->k_pool[l];
+    vp[l] = t->v_pool[l];
+  }
+  auto upload_ptrs = [&](void*** dst, std::vector<void*>& src) -> mk_status {
+    MK_CUDA(cudaMalloc(reinterpret_cast<void**>(dst), sizeof(void*) * L));
+    MK_CUDA(cudaMemcpy(*dst, src.data(), sizeof(void*) * L, cudaMemcpyHostToDevice));
+    return MK_OK;
+  };
+  {
+    mk_status st;
+    if ((st = upload_ptrs(&c->d_attn_norm, an)) != MK_OK) return fail(st);
+    if ((st = upload_ptrs(&c->d_router_bias, rb)) != MK_OK) return fail(st);
+    if ((st = upload_ptrs(&c->d_kpool, kp)) != MK_OK) return fail(st);
+    if ((st = upload_ptrs(&c->d_vpool, vp)) != MK_OK) return fail(st);
+  }
+  // RoPE inverse frequencies theta^(-2i/hd), computed in double
+  std::vector<double> inv(s.hd / 2);
+  for (int i = 0; i < s.hd / 2; ++i)
+    inv[i] = std::pow((double)s.theta, -2.0 * (double)i / (double)s.hd);
+  if (cudaMalloc(&c->d_inv_freq, sizeof(double) * inv.size()) != cudaSuccess)
+    return fail(MK_ERR_OOM);
+  if (cudaMemcpy(c->d_inv_freq, inv.data(), sizeof(double) * inv.size(), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return fail(MK_ERR_CUDA);
+  if (cudaMalloc(&c->d_status, sizeof(int32_t) * 16) != cudaSuccess) return fail(MK_ERR_OOM);
+  if (cudaMemset(c->d_status, 0, sizeof(int32_t) * 16) != cudaSuccess) return fail(MK_ERR_CUDA);
+  const char* env = std::getenv("MK_TIMEOUT_MS");
+  if (env) {
+    long ms = std::atol(env);
+    if (ms > 0) c->timeout_ns = (unsigned long long)ms * 1000000ull;
+  }
+  *out = c;
+  return MK_OK;
+}
+
+mk_status mk_set_timeout_ms(mk_ctx* c, int32_t ms) {
+  if (!c || ms <= 0) return MK_ERR_INVALID;
+  c->timeout_ns = (unsigned long long)ms * 1000000ull;
+  return MK_OK;
+}
+
+mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
+                            const int32_t* plan_len, int32_t max_pages_per_seq) {
+  if (!c || !seq_lens) return MK_ERR_INVALID;
+  const Shape& s = c->shape;
+  if (batch < 1 || batch > s.max_batch) return MK_ERR_INVALID;
+  if (max_pages_per_seq < 1) return MK_ERR_INVALID;
+  for (int b = 0; b < batch; ++b) {
+    if (seq_lens[b] < 0) return MK_ERR_INVALID;
+    const long need = (long)seq_lens[b] / mk::kPage + 1;   // page of the new token
+    if (need > max_pages_per_seq) return MK_ERR_INVALID;
+    if (plan_len && plan_len[b] < seq_lens[b]) return MK_ERR_INVALID;
+  }
+  MK_CUDA(cudaSetDevice(c->device));
+  MK_CUDA(cudaDeviceSynchronize());
+  c->have_schedule = false;
+  Plan plan;
+  MK_TRY((mk_status)mk::plan_schedule(s, c->n_sms, batch, seq_lens, plan_len, true, &plan));
+  SmemLayout sl;
+  {
+    int rc = mk::smem_layout(s, batch, plan.max_chunks, &sl);
+    if (rc != MK_OK) {
+      plan.release();
+      return (mk_status)rc;
+    }
+  }
+  int per_sm = 0;
+  if (mk::max_coresident(sl.dyn_bytes, &per_sm) != cudaSuccess || per_sm < 1) {
+    plan.release();
+    return MK_ERR_CAPACITY;
+  }
+  const int B = batch, L = s.L, d = s.d, G = s.Hq / s.Hkv, NR = d / 64, S = plan.S;
+  const int qkvR = (s.Hq + 2 * s.Hkv) * s.hd;
+  const int part_stride = round_up(2 * G + G * s.hd, 4);
+  const int actA_frag = 4 * d * B;
+  const int actA_bytes = actA_frag + round_up(NR * B * 4, 16);
+  const int ofrag_bytes = 4 * G * s.hd * B;
+  const int afrag_bytes = 4 * s.F * B;
+  const int rwords = mk::route_words(B, s.k, S);
+  auto fail = [&](mk_status st) {
+    plan.release();
+    return st;
+  };
+  mk_status st;
+#define ENSURE(buf, bytes) \
+  if ((st = ensure(c->buf, (size_t)(bytes))) != MK_OK) return fail(st)
+  ENSURE(x, (size_t)(L + 1) * B * d * 4);
+  ENSURE(actA, (size_t)(L + 1) * actA_bytes);
+  ENSURE(qkv, (size_t)L * B * qkvR * 4);
+  ENSURE(cs, (size_t)B * s.hd * 4);
+  ENSURE(attn_part, (size_t)L * B * s.Hkv * plan.max_chunks * part_stride * 4);
+  ENSURE(attn_o, (size_t)L * B * s.Hq * s.hd * 4);
+  ENSURE(ofrag, (size_t)L * s.Hkv * ofrag_bytes);
+  ENSURE(o_part, (size_t)L * s.Hkv * B * d * 4);
+  ENSURE(rlogits, (size_t)L * B * s.E * 4);
+  ENSURE(route, (size_t)L * rwords * 4);
+  ENSURE(expert_a, (size_t)L * S * B * s.F * 4);
+  ENSURE(afrag, (size_t)L * S * afrag_bytes);
+  ENSURE(moe_part, (size_t)L * s.k * B * d * 4);
+  ENSURE(desc, (size_t)plan.n_ctas * plan.max_tasks * mk::kDescWords * 4);
+  ENSURE(ntasks, (size_t)plan.n_ctas * 4);
+  ENSURE(phase_desc, (size_t)plan.n_phases * plan.n_ctas * plan.phase_max_tasks * mk::kDescWords * 4);
+  ENSURE(phase_counts, (size_t)plan.n_phases * plan.n_ctas * 4);
+#undef ENSURE
+  if (plan.n_counters > c->counters_cap) {
+    cudaFree(c->d_counters);
+    c->d_counters = nullptr;
+    c->counters_cap = 0;
+    if (cudaMalloc(&c->d_counters, sizeof(uint32_t) * plan.n_counters) != cudaSuccess)
+      return fail(MK_ERR_OOM);
+    c->counters_cap = plan.n_counters;
+  }
+  if (cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap) != cudaSuccess)
+    return fail(MK_ERR_CUDA);
+  if (cudaMemset(c->route.ptr, 0, c->route.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
+  if (cudaMemcpy(c->desc.ptr, plan.desc,
+                 (size_t)plan.n_ctas * plan.max_tasks * mk::kDescWords * 4,
+                 cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->ntasks.ptr, plan.counts, (size_t)plan.n_ctas * 4, cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
+      cudaMemcpy(c->phase_desc.ptr, plan.phase_desc,
+                 (size_t)plan.n_phases * plan.n_ctas * plan.phase_max_tasks * mk::kDescWords * 4,
+                 cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->phase_counts.ptr, plan.phase_counts, (size_t)plan.n_phases * plan.n_ctas * 4,
+                 cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(MK_ERR_CUDA);
+  c->phase_tasks.assign(plan.n_phases, 0);
+  for (int ph = 0; ph < plan.n_phases; ++ph)
+    for (int cc = 0; cc < plan.n_ctas; ++cc)
+      c->phase_tasks[ph] += plan.phase_counts[(size_t)ph * plan.n_ctas + cc];
+
+  Params& p = c->base;
+  std::memset(&p, 0, sizeof(p));
+  p.L = L; p.d = d; p.Hq = s.Hq; p.Hkv = s.Hkv; p.hd = s.hd; p.E = s.E; p.k = s.k; p.F = s.F;
+  p.V = s.V; p.B = B; p.S = S; p.G = G; p.NR = NR; p.qkvR = qkvR;
+  p.max_chunks = plan.max_chunks;
+  p.max_pages = max_pages_per_seq;
+  p.n_pages = s.n_pages;
+  p.part_stride = part_stride;
+  p.eps = s.eps;
+  p.actA_bytes = actA_bytes;
+  p.actA_frag_bytes = actA_frag;
+  p.ofrag_bytes = ofrag_bytes;
+  p.afrag_bytes = afrag_bytes;
+  p.route_words = rwords;
+  p.counters = c->d_counters;
+  p.tmaps = c->d_tmaps;
+  p.embed = static_cast<const uint16_t*>(c->embed);
+  p.final_norm = static_cast<const uint16_t*>(c->final_norm);
+  p.attn_norm = reinterpret_cast<const uint16_t* const*>(c->d_attn_norm);
+  p.router_bias = reinterpret_cast<const float* const*>(c->d_router_bias);
+  p.k_pool = reinterpret_cast<uint16_t* const*>(c->d_kpool);
+  p.v_pool = reinterpret_cast<uint16_t* const*>(c->d_vpool);
+  p.inv_freq = c->d_inv_freq;
+  p.x = static_cast<float*>(c->x.ptr);
+  p.actA = static_cast<uint8_t*>(c->actA.ptr);
+  p.qkv = static_cast<float*>(c->qkv.ptr);
+  p.cs = static_cast<float*>(c->cs.ptr);
+  p.attn_part = static_cast<float*>(c->attn_part.ptr);
+  p.attn_o = static_cast<float*>(c->attn_o.ptr);
+  p.ofrag = static_cast<uint8_t*>(c->ofrag.ptr);
+  p.o_part = static_cast<float*>(c->o_part.ptr);
+  p.rlogits = static_cast<float*>(c->rlogits.ptr);
+  p.route = static_cast<int32_t*>(c->route.ptr);
+  p.expert_a = static_cast<float*>(c->expert_a.ptr);
+  p.afrag = static_cast<uint8_t*>(c->afrag.ptr);
+  p.moe_part = static_cast<float*>(c->moe_part.ptr);
+  p.status = c->d_status;
+  p.n_stages = sl.n_stages;
+  p.nA = sl.nA;
+  p.actA_stride = sl.actA_stride;
+  p.off_bars = sl.off_bars;
+  p.off_fifo = sl.off_fifo;
+  p.off_scratch = sl.off_scratch;
+  p.off_actA = sl.off_actA;
+  p.off_actB = sl.off_actB;
+  p.actB_bytes = sl.actB_bytes;
+  p.off_ring = sl.off_ring;
+  p.smem_bytes = sl.dyn_bytes;
+
+  c->plan.release();
+  c->plan = plan;  // takes ownership of the host arrays
+  c->sl = sl;
+  c->B = B;
+  c->S = S;
+  c->max_chunks = plan.max_chunks;
+  c->max_pages = max_pages_per_seq;
+  c->epoch = 0;
+  c->have_schedule = true;
+  MK_CUDA(cudaDeviceSynchronize());
+  return MK_OK;
+}
+
+static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* positions,
+                             const int32_t* page_table, const int32_t* seq_lens, float* logits,
+                             void* stream, bool unfused) {
+  if (!c) return MK_ERR_INVALID;
+  if (!c->have_schedule) return MK_ERR_STATE;
+  if (!tokens || !positions || !page_table || !seq_lens || !logits) return MK_ERR_INVALID;
+  MK_CUDA(cudaSetDevice(c->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = c->base;
+  p.tokens = tokens;
+  p.positions = positions;
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.logits = logits;
+  p.timeout_ns = c->timeout_ns;
+  p.epoch = c->epoch + 1;
+  cudaError_t e = cudaSuccess;
+  if (!unfused) {
+    p.desc = static_cast<const int32_t*>(c->desc.ptr);
+    p.ntasks = static_cast<const int32_t*>(c->ntasks.ptr);
+    p.max_tasks = c->plan.max_tasks;
+    e = mk::launch_interp(p, c->plan.n_ctas, st);
+  } else {
+    const size_t stride = (size_t)c->plan.n_ctas * c->plan.phase_max_tasks * mk::kDescWords;
+    for (int ph = 0; ph < c->plan.n_phases && e == cudaSuccess; ++ph) {
+      if (c->phase_tasks[ph] == 0) continue;
+      p.desc = static_cast<const int32_t*>(c->phase_desc.ptr) + stride * ph;
+      p.ntasks = static_cast<const int32_t*>(c->phase_counts.ptr) + (size_t)ph * c->plan.n_ctas;
+      p.max_tasks = c->plan.phase_max_tasks;
+      e = mk::launch_interp(p, c->plan.n_ctas, st);
+    }
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  c->epoch += 1;
+  c->last_stream = st;
+  return MK_OK;
+}
+
+mk_status mk_decode_step(mk_ctx* c, const int32_t* tokens, const int32_t* positions,
+                         const int32_t* page_table, const int32_t* seq_lens, float* logits,
+                         void* stream) {
+  return launch_step(c, tokens, positions, page_table, seq_lens, logits, stream, false);
+}
+
+mk_status mk_decode_step_unfused(mk_ctx* c, const int32_t* tokens, const int32_t* positions,
+                                 const int32_t* page_table, const int32_t* seq_lens, float* logits,
+                                 void* stream) {
+  return launch_step(c, tokens, positions, page_table, seq_lens, logits, stream, true);
+}
+
+mk_status mk_check(mk_ctx* c, int32_t* device_status, int32_t* detail) {
+  if (!c) return MK_ERR_INVALID;
+  MK_CUDA(cudaSetDevice(c->device));
+  MK_CUDA(cudaDeviceSynchronize());
+  int32_t st[16];
+  MK_CUDA(cudaMemcpy(st, c->d_status, sizeof(st), cudaMemcpyDeviceToHost));
+  if (device_status) *device_status = st[mk::ST_CODE];
+  if (detail)
+    for (int i = 0; i < 8; ++i) detail[i] = st[i];
+  if (st[mk::ST_CODE] != 0 || st[mk::ST_ABORT] != 0) {
+    // a step that stopped part-way leaves counters short of their targets:
+    // restart the epochs so the next step begins from a clean state
+    MK_CUDA(cudaMemset(c->d_status, 0, sizeof(st)));
+    if (c->d_counters)
+      MK_CUDA(cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap));
+    c->epoch = 0;
+    return st[mk::ST_CODE] != 0 ? (mk_status)st[mk::ST_CODE] : MK_ERR_DEVICE;
+  }
+  return MK_OK;
+}
+
+size_t mk_debug_size(mk_ctx* c, int which) {
+  if (!c || !c->have_schedule) return 0;
+  const Shape& s = c->shape;
+  const size_t L = s.L, B = c->B, S = c->S;
+  switch (which) {
+    case MK_BUF_X: return (L + 1) * B * s.d * 4;
+    case MK_BUF_QKV: return L * B * (s.Hq + 2 * s.Hkv) * s.hd * 4;
+    case MK_BUF_ATTN_O: return L * B * s.Hq * s.hd * 4;
+    case MK_BUF_RLOGITS: return L * B * s.E * 4;
+    case MK_BUF_TOPK: return 2 * L * B * s.k * 4;
+    case MK_BUF_NSLOTS: return L * 4;
+    case MK_BUF_EXPERT_A: return L * S * B * s.F * 4;
+    case MK_BUF_MOE: return L * s.k * B * s.d * 4;
+    case MK_BUF_OPART: return L * s.Hkv * B * s.d * 4;
+  }
+  return 0;
+}
+
+mk_status mk_debug_read(mk_ctx* c, int which, void* dst, size_t bytes) {
+  if (!c || !dst) return MK_ERR_INVALID;
+  if (!c->have_schedule) return MK_ERR_STATE;
+  const size_t need = mk_debug_size(c, which);
+  if (need == 0 || bytes != need) return MK_ERR_INVALID;
+  MK_CUDA(cudaSetDevice(c->device));
+  MK_CUDA(cudaDeviceSynchronize());
+  const Shape& s = c->shape;
+  const int L = s.L, B = c->B, K = s.k, S = c->S;
+  const void* src = nullptr;
+  switch (which) {
+    case MK_BUF_X: src = c->x.ptr; break;
+    case MK_BUF_QKV: src = c->qkv.ptr; break;
+    case MK_BUF_ATTN_O: src = c->attn_o.ptr; break;
+    case MK_BUF_RLOGITS: src = c->rlogits.ptr; break;
+    case MK_BUF_EXPERT_A: src = c->expert_a.ptr; break;
+    case MK_BUF_MOE: src = c->moe_part.ptr; break;
+    case MK_BUF_OPART: src = c->o_part.ptr; break;
+    default: break;
+  }
+  if (src) {
+    MK_CUDA(cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost));
+    return MK_OK;
+  }
+  const int rw = mk::route_words(B, K, S);
+  std::vector<int32_t> rt((size_t)L * rw);
+  MK_CUDA(cudaMemcpy(rt.data(), c->route.ptr, rt.size() * 4, cudaMemcpyDeviceToHost));
+  int32_t* o = static_cast<int32_t*>(dst);
+  if (which == MK_BUF_NSLOTS) {
+    for (int l = 0; l < L; ++l) o[l] = rt[(size_t)l * rw];
+    return MK_OK;
+  }
+  // MK_BUF_TOPK: ids [L][B][k] then weights [L][B][k]
+  for (int l = 0; l < L; ++l)
+    for (int i = 0; i < B * K; ++i) {
+      o[(size_t)l * B * K + i] = rt[(size_t)l * rw + mk::route_topk_idx(B, K) + i];
+      o[(size_t)L * B * K + (size_t)l * B * K + i] = rt[(size_t)l * rw + mk::route_topk_w(B, K) + i];
+    }
+  return MK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+// mk_internal.h -- task descriptor format, opcodes, counter layout and the
+// kernel parameter block shared by the host planner, the host library and the
+// persistent interpreter.
+//
+// The descriptor format follows the pages' "uniform ABI" of fixed-size int32
+// task records (aimodeling.com, "Cohere open-sources a megakernel inference
+// engine", section "Caveats and takeaways": 32 int32 per task); the field
+// assignment below is this library's own.
+#pragma once
+
+#include <stdint.h>
+#include <stddef.h>
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+
+namespace mk {
+
+constexpr int kDescWords = 32;
+constexpr int kPage = 64;            // tokens per KV page
+constexpr int kMaxBatch = 8;         // mma N (token columns) and the pages' batch cap
+constexpr int kMaxTopK = 8;
+constexpr int kStageBytes = 16384;   // one ring stage = 8 units of 16 rows x 64 k (bf16)
+constexpr int kUnitBytes = 2048;
+constexpr int kConsumerWarps = 8;
+constexpr int kProducerWarp = 0;     // TMA weight/KV streamer + task resolver
+constexpr int kLoaderWarp = 1;       // dependency waits + activation loads
+constexpr int kSignalWarp = 2;       // completion signals (release adds)
+constexpr int kFirstConsumerWarp = 3;
+constexpr int kThreads = (kFirstConsumerWarp + kConsumerWarps) * 32;   // 352
+constexpr int kFifo = 16;            // task entries in flight per CTA
+constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words
+constexpr int kMapsPerLayer = 8;     // qkv, o, router, gate, up, down, kpool, vpool
+
+// ---------------------------------------------------------------- opcodes --
+enum Op : int32_t {
+  OP_NONE = 0,
+  OP_RN = 1,        // fused residual add + RMSNorm statistics for one 64-row tile
+  OP_QKV = 2,       // QKV projection tile (RoPE/append happen in OP_ATTN)
+  OP_ROUTER = 3,    // router logits tile
+  OP_TOPK = 4,      // top-k + softmax + expert-slot compaction
+  OP_ATTN = 5,      // paged GQA decode attention over one KV chunk (+RoPE, append)
+  OP_COMBINE = 6,   // log-sum-exp merge of the chunk partials of (b, g)
+  OP_OPROJ = 7,     // O-proj tile, split-K by KV group
+  OP_GATEUP = 8,    // expert gate+up tile with SwiGLU epilogue
+  OP_DOWN = 9,      // expert down tile with weighted scatter into rank slots
+  OP_LMHEAD = 10,   // LM head tile
+  OP_COUNT = 11
+};
+
+// ------------------------------------------------------- descriptor words --
+enum DescField : int {
+  D_OP = 0,
+  D_LAYER = 1,
+  D_A = 2,          // tile / batch index / slot
+  D_B = 3,          // tile / group
+  D_C = 4,          // chunk
+  D_D = 5,          // chunk count
+  D_FLAGS = 6,
+  D_NWAIT = 7,
+  D_W0 = 8, D_W0N = 9, D_W1 = 10, D_W1N = 11,   // loader waits (counter, arrivals/step)
+  D_PW = 12, D_PWN = 13,                        // producer wait (-1: none)
+  D_NSIG = 14, D_S0 = 15, D_S1 = 16,            // signalled counters
+  D_NSTAGE = 17,    // ring stages streamed (static part)
+  D_ROW0 = 18,      // GEMV: first row (per-expert offset added at run time)
+  D_K0 = 19,        // GEMV: first column
+  D_KCH = 20,       // GEMV: 64-column chunks
+  D_R = 21,         // GEMV: rows per tile (TMA box height)
+  D_NMAT = 22,      // GEMV: matrices per tile (2 = gate+up)
+  D_MAP0 = 23, D_MAP1 = 24,                     // tensor-map indices
+  D_BSLOT = 25,     // small-activation buffer (0/1)
+  D_SEQ = 26,       // position of this task in its CTA list
+  D_PPC = 27,       // attention: pages per chunk
+  D_PHASE = 28,     // operation phase (for the unfused launcher)
+  D_X0 = 29, D_X1 = 30, D_X2 = 31
+};
+
+enum Flags : int32_t {
+  F_LOAD_A = 1,      // loader fetches the normalized-input activation (slot A)
+  F_REL_A = 2,       // consumer releases slot A after this task
+  F_LOAD_B = 4,      // loader fetches this task's small activation (slot B[D_BSLOT])
+  F_LAST_CHUNK = 8,  // attention chunk that owns the new token (and appends it)
+  F_SINGLE = 16      // attention of (b, g) in one chunk: write the final output
+};
+
+// ------------------------------------------------- resolved entry words ---
+// Written by the producer into the FIFO entry after the 32 descriptor words.
+enum ResolvedField : int {
+  R_NSTAGE = 0,     // stages actually streamed for this task
+  R_EXPERT = 1,     // expert id (-1: empty slot)
+  R_NTOK = 2,       // tokens in the slot / pages in the chunk
+  R_P0 = 3,         // attention: first logical page of the chunk
+  R_SEQLEN = 4,     // attention: cached tokens of the sequence
+  R_PHYS_NEW = 5,   // attention: physical page receiving the new token
+  R_TOK = 8,        // [8] slot token ids
+  R_RANK = 16,      // [8] rank of the expert in each token's top-k
+  R_W = 24          // [8] routing weight (float bits)
+};
+
+// ------------------------------------------------------------- params -----
+struct Params {
+  // shape
+  int L, d, Hq, Hkv, hd, E, k, F, V, B, S, G, NR, qkvR;
+  int max_chunks, max_pages, n_pages, part_stride;
+  float eps;
+  // byte sizes of the activation formats
+  int actA_bytes;      // per level: B-fragment hi/lo of gamma*x + ss partials
+  int actA_frag_bytes; // per level: the fragment part
+  int ofrag_bytes;     // per (layer, group)
+  int afrag_bytes;     // per (layer, slot)
+  int route_words;     // per layer
+  // schedule
+  const int32_t* desc;     // [n_ctas][max_tasks][kDescWords]
+  const int32_t* ntasks;   // [n_ctas]
+  int max_tasks;
+  uint32_t* counters;
+  uint32_t epoch;
+  // tensors
+  const void* tmaps;       // CUtensorMap[L * kMapsPerLayer + 1]
+  const uint16_t* embed;
+  const uint16_t* final_norm;
+  const uint16_t* const* attn_norm;   // device array [L]
+  const float* const* router_bias;    // device array [L] (entries may be null)
+  uint16_t* const* k_pool;            // device array [L]
+  uint16_t* const* v_pool;            // device array [L]
+  const double* inv_freq;             // [hd/2]
+  // step inputs / output
+  const int32_t* tokens;
+  const int32_t* positions;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* logits;
+  // context buffers
+  float* x;          // [L+1][B][d]
+  uint8_t* actA;     // [L+1][actA_bytes]
+  float* qkv;        // [L][B][qkvR]
+  float* cs;         // [B][hd]  cos | sin
+  float* attn_part;  // [L][B][Hkv][max_chunks][part_stride]
+  float* attn_o;     // [L][B][Hq*hd]
+  uint8_t* ofrag;    // [L][Hkv][ofrag_bytes]
+  float* o_part;     // [L][Hkv][B][d]
+  float* rlogits;    // [L][B][E]
+  int32_t* route;    // [L][route_words]
+  float* expert_a;   // [L][S][B][F]
+  uint8_t* afrag;    // [L][S][afrag_bytes]
+  float* moe_part;   // [L][k][B][d]
+  int32_t* status;   // [16]
+  unsigned long long timeout_ns;
+  // shared-memory layout (byte offsets from the 1024-aligned base)
+  int n_stages, nA, actA_stride;
+  int off_bars, off_fifo, off_scratch, off_actA, off_actB, actB_bytes, off_ring;
+  int smem_bytes;
+};
+
+// status word layout
+enum StatusField : int {
+  ST_CODE = 0, ST_CTA = 1, ST_TASK = 2, ST_OP = 3, ST_COUNTER = 4,
+  ST_OBSERVED = 5, ST_TARGET = 6, ST_AUX = 7, ST_ABORT = 15
+};
+
+// routing table layout per layer (int32 words)
+MK_HD inline int route_topk_idx(int B, int k) { (void)B; (void)k; return 1; }
+MK_HD inline int route_topk_w(int B, int k) { return 1 + B * k; }
+MK_HD inline int route_slot_expert(int B, int k) { return 1 + 2 * B * k; }
+MK_HD inline int route_slot_ntok(int B, int k, int S) { return 1 + 2 * B * k + S; }
+MK_HD inline int route_slot_tok(int B, int k, int S) { return 1 + 2 * B * k + 2 * S; }
+MK_HD inline int route_slot_rank(int B, int k, int S) { return 1 + 2 * B * k + 2 * S + 8 * S; }
+MK_HD inline int route_slot_w(int B, int k, int S) { return 1 + 2 * B * k + 2 * S + 16 * S; }
+MK_HD inline int route_words(int B, int k, int S) {
+  int w = 1 + 2 * B * k + 2 * S + 24 * S;
+  return (w + 3) & ~3;
+}
+
+// ------------------------------------------------------------- planner ----
+struct Shape {
+  int L, d, Hq, Hkv, hd, E, k, F, V, page, max_batch, n_pages;
+  float theta, eps;
+};
+
+struct Plan {
+  int n_ctas = 0, B = 0, S = 0, max_chunks = 1, n_counters = 0, max_tasks = 0;
+  int n_phases = 0;
+  int r_qkv = 16, r_router = 16;
+  size_t total_tasks = 0;
+  // flat storage: CTA c has counts[c] descriptors
+  int32_t* desc = nullptr;           // [n_ctas][max_tasks][kDescWords]
+  int32_t* counts = nullptr;         // [n_ctas]
+  int32_t* targets = nullptr;        // [n_counters]
+  // per-phase lists for the unfused launcher: [n_phases][n_ctas][max_tasks_phase][32]
+  int32_t* phase_desc = nullptr;
+  int32_t* phase_counts = nullptr;   // [n_phases][n_ctas]
+  int phase_max_tasks = 0;
+  int nc[kMaxBatch] = {0};           // attention chunks per sequence
+  int ppc[kMaxBatch] = {0};          // pages per chunk per sequence
+  void release();
+};
+
+// Shared-memory carve-up of one CTA for a shape and batch.
+struct SmemLayout {
+  int nA;             // normalized-input activation buffers (1 or 2)
+  int actA_stride;    // bytes per A buffer
+  int actB_bytes;     // bytes per small-activation buffer (two of them)
+  int scratch_bytes;
+  int n_stages;       // ring stages of kStageBytes
+  int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring;
+  int total;          // bytes from the 1024-aligned base
+  int dyn_bytes;      // dynamic shared memory to request (total + alignment slack)
+};
+int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* out);
+
+// Returns MK_OK or MK_ERR_INVALID / MK_ERR_CAPACITY for an unsupported shape.
+int validate_shape(const Shape& s);
+
+// Validates the shape and builds the plan; returns 0 or an mk_status code.
+int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
+                  const int32_t* plan_len, bool with_phases, Plan* out);
+
+// GEMV tile geometry shared by planner and host (rows per tile for a K).
+int gemv_rows_for(int K, int n_mat);
+
+}  // namespace mk

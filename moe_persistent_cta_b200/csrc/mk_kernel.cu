@@ -1,0 +1,1275 @@
+// mk_kernel.cu -- the persistent decode interpreter for sm_100a.
+//
+// One CTA per SM stays resident for the whole decode step and walks its own
+// list of task descriptors (agenticcommons.xyz, "Cohere North Mini Code
+// megakernel serving engine", section "How the megakernel works").  Warp roles
+// inside a CTA:
+//   warp 0 (producer)  resolves each task (routing table for expert tiles,
+//                      page table for attention chunks) and streams its
+//                      immutable weight / KV tiles into a ring of 16 KB shared
+//                      memory stages with TMA, BEFORE the task's activation
+//                      dependency is known to be satisfied (section "Three
+//                      sources of speedup", item 3).  The ring's stage/phase
+//                      runs on across task boundaries, so consecutive tiles
+//                      never drain and refill the pipeline (section "Building
+//                      on Hazy Research": phase continuation across tiles and
+//                      weight loads issued before the cross-SM wait).
+//   warp 1 (loader)    spins on the task's global counters (bounded by a
+//                      deadline) and then bulk-copies the task's activation
+//                      vector into shared memory.
+//   warp 2 (signaler)  after the consumers finish a task, publishes it with a
+//                      release add on each of the task's counters.
+//   warps 3..10        compute: mma.sync bf16 tiles (weights as the 16-row A
+//                      operand read from the swizzled TMA tile with ldmatrix,
+//                      activations as the 8-column B operand split into bf16
+//                      hi + lo halves so the product keeps ~16 mantissa bits),
+//                      attention with an online softmax, and the epilogues.
+// Every wait is bounded by a globaltimer deadline; on expiry the CTA latches an
+// error in the status word, raises the abort flag and unwinds, waiting for its
+// own copies in flight before it exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---------------------------------------------------------------- PTX -----
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma1688(float* c, uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+// named barrier among the 8 consumer warps only
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ int cbar_or(int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred)
+      : "memory");
+  return r;
+}
+
+// bf16 helpers
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16r(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ float bf16_to_f(uint16_t u) {
+  return __uint_as_float(((uint32_t)u) << 16);
+}
+// B-operand fragment entry for 16 consecutive k of one column: hi and lo
+// bf16 halves of the four values this lane of the quad owns.
+__device__ __forceinline__ uint4 frag_entry(float v0, float v1, float v2, float v3) {
+  float h0 = bf16r(v0), h1 = bf16r(v1), h2 = bf16r(v2), h3 = bf16r(v3);
+  uint4 e;
+  e.x = pack_bf16(h0, h1);
+  e.y = pack_bf16(h2, h3);
+  e.z = pack_bf16(v0 - h0, v1 - h1);
+  e.w = pack_bf16(v2 - h2, v3 - h3);
+  return e;
+}
+
+// -------------------------------------------------------------- state -----
+struct Smem {
+  uint8_t* base;
+  uint8_t* ring;
+  uint64_t* bars;
+  int32_t* fifo;
+  uint8_t* scratch;
+  uint8_t* actA;
+  uint8_t* actB;
+  int NS;
+  int* abort_flag;
+  // barrier indices
+  __device__ uint32_t full(int s) const { return saddr(bars + s); }
+  __device__ uint32_t empty(int s) const { return saddr(bars + NS + s); }
+  __device__ uint32_t ready(int e) const { return saddr(bars + 2 * NS + e); }
+  __device__ uint32_t done(int e) const { return saddr(bars + 2 * NS + kFifo + e); }
+  __device__ uint32_t fempty(int e) const { return saddr(bars + 2 * NS + 2 * kFifo + e); }
+  __device__ uint32_t afullA(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + i); }
+  __device__ uint32_t aemptyA(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 2 + i); }
+  __device__ uint32_t afullB(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 4 + i); }
+  __device__ uint32_t aemptyB(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 6 + i); }
+};
+
+__device__ void raise_error(const Params& p, int code, int task, int op, int ctr, uint32_t obs,
+                            uint32_t tgt, int aux) {
+  if (atomicCAS(&p.status[ST_CODE], 0, code) == 0) {
+    p.status[ST_CTA] = blockIdx.x;
+    p.status[ST_TASK] = task;
+    p.status[ST_OP] = op;
+    p.status[ST_COUNTER] = ctr;
+    p.status[ST_OBSERVED] = (int)obs;
+    p.status[ST_TARGET] = (int)tgt;
+    p.status[ST_AUX] = aux;
+  }
+  __threadfence();
+  atomicExch(&p.status[ST_ABORT], 1);
+}
+
+__device__ __forceinline__ bool aborted(const Smem& sm) {
+  return *(volatile int*)sm.abort_flag != 0;
+}
+
+// Bounded spin on a global counter (one lane).
+__device__ bool wait_counter(const Params& p, const Smem& sm, int ctr, uint32_t target, int task,
+                             int op) {
+  const uint32_t* c = p.counters + ctr;
+  uint32_t v = ld_acquire(c);
+  if (v >= target) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t it = 1;; ++it) {
+    v = ld_acquire(c);
+    if (v >= target) return true;
+    if ((it & 7u) == 0) {
+      if (aborted(sm)) return false;
+      if (*(volatile int*)(p.status + ST_ABORT)) {
+        *(volatile int*)sm.abort_flag = 1;
+        return false;
+      }
+      if (gtimer() - t0 > p.timeout_ns) {
+        raise_error(p, MK_ERR_TIMEOUT, task, op, ctr, v, target, 0);
+        *(volatile int*)sm.abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait on a shared-memory mbarrier phase (every calling lane).
+__device__ bool wait_bar(const Params& p, const Smem& sm, uint32_t bar, uint32_t parity, int aux) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (;;) {
+    for (int i = 0; i < 8; ++i)
+      if (mbar_test(bar, parity)) return true;
+    if (aborted(sm)) return false;
+    if (gtimer() - t0 > p.timeout_ns) {
+      raise_error(p, MK_ERR_TIMEOUT, -1, -1, -1, 0, 0, aux);
+      *(volatile int*)sm.abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: lane 0 waits, the outcome is broadcast.
+__device__ bool warp_wait(const Params& p, const Smem& sm, uint32_t bar, uint32_t parity,
+                          int aux) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(p, sm, bar, parity, aux) ? 1 : 0;
+  ok = __shfl_sync(FULL, ok, 0);
+  return ok != 0;
+}
+
+// Wait for a phase that is known to complete (copies in flight), bounded.
+__device__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = gtimer();
+  while (!mbar_test(bar, parity)) {
+    if (gtimer() - t0 > p.timeout_ns) break;
+  }
+}
+
+__device__ __forceinline__ const void* tmap(const Params& p, int idx) {
+  return static_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
+}
+
+// ============================================================== producer ==
+__device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my, int ntasks) {
+  const int lane = threadIdx.x & 31;
+  uint32_t stage_ctr = 0;
+  int fills[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) fills[i] = 0;
+  const int NS = sm.NS;
+  for (int i = 0; i < ntasks; ++i) {
+    const int e = i % kFifo;
+    if (!warp_wait(p, sm, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 100)) break;
+    const int32_t dw = my[(size_t)i * kDescWords + lane];
+    const int op = __shfl_sync(FULL, dw, D_OP);
+    const int layer = __shfl_sync(FULL, dw, D_LAYER);
+    int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
+    int32_t rw = 0;  // resolved word `lane`
+    int expert = -1, ntok = 0, p0 = 0, seqlen = 0, phys_new = -1;
+    bool fail = false;
+    if (op == OP_GATEUP || op == OP_DOWN) {
+      const int ctr = __shfl_sync(FULL, dw, D_PW);
+      const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
+      int ok = 1;
+      if (lane == 0) ok = wait_counter(p, sm, ctr, tgt, i, op) ? 1 : 0;
+      ok = __shfl_sync(FULL, ok, 0);
+      if (!ok) break;
+      __syncwarp();
+      const int j = __shfl_sync(FULL, dw, D_A);
+      const int32_t* rt = p.route + (size_t)layer * p.route_words;
+      const int B = p.B, K = p.k, S = p.S;
+      expert = __ldcg(rt + route_slot_expert(B, K) + j);
+      ntok = __ldcg(rt + route_slot_ntok(B, K, S) + j);
+      if (expert < 0 || expert >= p.E || ntok < 0 || ntok > B) {
+        if (expert >= p.E || ntok < 0 || ntok > B) {
+          if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, expert, ntok, 1);
+          *(volatile int*)sm.abort_flag = 1;
+          break;
+        }
+        expert = -1;
+        ntok = 0;
+        nstage = 0;
+      }
+      if (lane >= R_TOK && lane < R_TOK + 8) {
+        int t = lane - R_TOK;
+        rw = t < ntok ? __ldcg(rt + route_slot_tok(B, K, S) + j * 8 + t) : 0;
+      } else if (lane >= R_RANK && lane < R_RANK + 8) {
+        int t = lane - R_RANK;
+        rw = t < ntok ? __ldcg(rt + route_slot_rank(B, K, S) + j * 8 + t) : 0;
+      } else if (lane >= R_W && lane < R_W + 8) {
+        int t = lane - R_W;
+        rw = t < ntok ? __ldcg(rt + route_slot_w(B, K, S) + j * 8 + t) : 0;
+      }
+    } else if (op == OP_ATTN) {
+      const int b = __shfl_sync(FULL, dw, D_A);
+      const int c = __shfl_sync(FULL, dw, D_C);
+      const int nc = __shfl_sync(FULL, dw, D_D);
+      const int ppc = __shfl_sync(FULL, dw, D_PPC);
+      seqlen = __ldg(p.seq_lens + b);
+      const int pages_now = (seqlen + kPage - 1) / kPage;
+      p0 = c * ppc;
+      int np = min(ppc, pages_now - p0);
+      if (np < 0) np = 0;
+      const bool last = (c == nc - 1);
+      if (seqlen < 0 || (last && p0 + ppc < pages_now) || (seqlen / kPage) >= p.max_pages) {
+        if (lane == 0) raise_error(p, MK_ERR_STATE, i, op, -1, seqlen, pages_now, b);
+        *(volatile int*)sm.abort_flag = 1;
+        fail = true;
+      }
+      if (!fail && last) {
+        phys_new = __ldg(p.page_table + (size_t)b * p.max_pages + seqlen / kPage);
+        if (phys_new < 0 || phys_new >= p.n_pages) {
+          if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, phys_new, p.n_pages, 2);
+          *(volatile int*)sm.abort_flag = 1;
+          fail = true;
+        }
+      }
+      if (fail) break;
+      nstage = 2 * np;
+      ntok = np;
+    }
+    if (lane == R_NSTAGE) rw = nstage;
+    if (lane == R_EXPERT) rw = expert;
+    if (lane == R_NTOK) rw = ntok;
+    if (lane == R_P0) rw = p0;
+    if (lane == R_SEQLEN) rw = seqlen;
+    if (lane == R_PHYS_NEW) rw = phys_new;
+    int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    ent[lane] = dw;
+    ent[32 + lane] = rw;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.ready(e));
+
+    // ---- stream the task's tiles
+    if (op == OP_ATTN) {
+      const int b = __shfl_sync(FULL, dw, D_A);
+      const int g = __shfl_sync(FULL, dw, D_B);
+      const void* mk_ = tmap(p, __shfl_sync(FULL, dw, D_MAP0));
+      const void* mv_ = tmap(p, __shfl_sync(FULL, dw, D_MAP1));
+      const int np = ntok;
+      int pg = -1;
+      const int* pt = p.page_table + (size_t)b * p.max_pages;
+      for (int s = 0; s < nstage; ++s) {
+        const int pi = s >> 1;
+        if ((pi & 31) == 0 && (s & 1) == 0) {
+          int idx = p0 + pi + lane;
+          pg = (pi + lane < np) ? __ldg(pt + idx) : 0;
+          int bad = (pi + lane < np) && (pg < 0 || pg >= p.n_pages);
+          if (__any_sync(FULL, bad)) {
+            if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, 0, 0, 3);
+            *(volatile int*)sm.abort_flag = 1;
+            fail = true;
+          }
+        }
+        if (fail) break;
+        const int phys = __shfl_sync(FULL, pg, pi & 31);
+        const uint32_t slot = stage_ctr % NS;
+        const uint32_t ph = (stage_ctr / NS) & 1;
+        if (!warp_wait(p, sm, sm.empty(slot), ph ^ 1, 101)) {
+          fail = true;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t bytes = (uint32_t)p.hd * kPage * 2;
+          const uint32_t fb = sm.full(slot);
+          mbar_expect_tx(fb, bytes);
+          const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
+          const int y = (phys * p.Hkv + g) * kPage;
+          const void* m = (s & 1) ? mv_ : mk_;
+          for (int xb = 0; xb < p.hd / 64; ++xb) tma_2d(dst + xb * 8192, m, xb * 64, y, fb);
+        }
+        fills[slot] += 1;
+        __syncwarp();
+        ++stage_ctr;
+      }
+      if (fail) break;
+    } else if (nstage > 0) {
+      const int nm = __shfl_sync(FULL, dw, D_NMAT);
+      const int R = __shfl_sync(FULL, dw, D_R);
+      const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
+      const int k0 = __shfl_sync(FULL, dw, D_K0);
+      int row0 = __shfl_sync(FULL, dw, D_ROW0);
+      if (op == OP_GATEUP) row0 += expert * p.F;
+      if (op == OP_DOWN) row0 += expert * p.d;
+      const void* m0 = tmap(p, __shfl_sync(FULL, dw, D_MAP0));
+      const void* m1 = nm > 1 ? tmap(p, __shfl_sync(FULL, dw, D_MAP1)) : m0;
+      for (int s = 0; s < nstage; ++s) {
+        const uint32_t slot = stage_ctr % NS;
+        const uint32_t ph = (stage_ctr / NS) & 1;
+        if (!warp_wait(p, sm, sm.empty(slot), ph ^ 1, 102)) {
+          fail = true;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = sm.full(slot);
+          mbar_expect_tx(fb, kStageBytes);
+          const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
+          for (int kl = 0; kl < kcps; ++kl) {
+            const int x = k0 + (s * kcps + kl) * 64;
+            tma_2d(dst + (kl * nm + 0) * MT * kUnitBytes, m0, x, row0, fb);
+            if (nm > 1) tma_2d(dst + (kl * nm + 1) * MT * kUnitBytes, m1, x, row0, fb);
+          }
+        }
+        fills[slot] += 1;
+        __syncwarp();
+        ++stage_ctr;
+      }
+      if (fail) break;
+    }
+  }
+  // drain: every fill issued must land before the CTA may exit
+  for (int s = 0; s < NS && s < 16; ++s)
+    if (fills[s] > 0) drain_bar(p, sm.full(s), (uint32_t)((fills[s] - 1) & 1));
+}
+
+// ================================================================ loader ==
+__device__ void loader_loop(const Params& p, const Smem& sm, const int32_t* my, int ntasks) {
+  const int lane = threadIdx.x & 31;
+  int nloadA[2] = {0, 0}, nloadB[2] = {0, 0};
+  for (int i = 0; i < ntasks; ++i) {
+    const int e = i % kFifo;
+    if (!warp_wait(p, sm, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 200)) break;
+    const int32_t dw = my[(size_t)i * kDescWords + lane];
+    const int op = __shfl_sync(FULL, dw, D_OP);
+    const int layer = __shfl_sync(FULL, dw, D_LAYER);
+    const int flags = __shfl_sync(FULL, dw, D_FLAGS);
+    const int nwait = __shfl_sync(FULL, dw, D_NWAIT);
+    int ok = 1;
+    for (int w = 0; w < nwait && ok; ++w) {
+      const int ctr = __shfl_sync(FULL, dw, D_W0 + 2 * w);
+      const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_W0N + 2 * w);
+      if (lane == 0) ok = wait_counter(p, sm, ctr, tgt, i, op) ? 1 : 0;
+      ok = __shfl_sync(FULL, ok, 0);
+    }
+    if (!ok) break;
+    if (flags & F_LOAD_A) {
+      const int buf = __shfl_sync(FULL, dw, D_X0);
+      if (!warp_wait(p, sm, sm.aemptyA(buf), (uint32_t)((nloadA[buf] & 1) ^ 1), 201)) break;
+      nloadA[buf]++;
+      if (lane == 0) {
+        fence_proxy_async_global();
+        const uint32_t fb = sm.afullA(buf);
+        mbar_expect_tx(fb, (uint32_t)p.actA_bytes);
+        bulk_g2s(saddr(sm.actA + (size_t)buf * p.actA_stride),
+                 p.actA + (size_t)layer * p.actA_bytes, (uint32_t)p.actA_bytes, fb);
+      }
+      __syncwarp();
+    }
+    if (flags & F_LOAD_B) {
+      const int buf = __shfl_sync(FULL, dw, D_BSLOT);
+      if (!warp_wait(p, sm, sm.aemptyB(buf), (uint32_t)((nloadB[buf] & 1) ^ 1), 202)) break;
+      nloadB[buf]++;
+      if (lane == 0) {
+        fence_proxy_async_global();
+        const uint32_t fb = sm.afullB(buf);
+        const uint32_t dst = saddr(sm.actB + (size_t)buf * p.actB_bytes);
+        const int a = __ldg(my + (size_t)i * kDescWords + D_A);
+        const int bb = __ldg(my + (size_t)i * kDescWords + D_B);
+        if (op == OP_ATTN) {
+          const int b = a, g = bb, G = p.G, hd = p.hd;
+          const float* row = p.qkv + ((size_t)layer * p.B + b) * p.qkvR;
+          const uint32_t qb = (uint32_t)(G * hd * 4), hb = (uint32_t)(hd * 4);
+          mbar_expect_tx(fb, qb + 3 * hb);
+          bulk_g2s(dst, row + (size_t)g * G * hd, qb, fb);
+          bulk_g2s(dst + qb, row + (size_t)p.Hq * hd + g * hd, hb, fb);
+          bulk_g2s(dst + qb + hb, row + (size_t)(p.Hq + p.Hkv) * hd + g * hd, hb, fb);
+          bulk_g2s(dst + qb + 2 * hb, p.cs + (size_t)b * hd, hb, fb);
+        } else if (op == OP_OPROJ) {
+          const int g = bb;
+          mbar_expect_tx(fb, (uint32_t)p.ofrag_bytes);
+          bulk_g2s(dst, p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes,
+                   (uint32_t)p.ofrag_bytes, fb);
+        } else {  // OP_DOWN
+          const int j = a;
+          mbar_expect_tx(fb, (uint32_t)p.afrag_bytes);
+          bulk_g2s(dst, p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes,
+                   (uint32_t)p.afrag_bytes, fb);
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mbar_arrive(sm.ready(e));
+    __syncwarp();
+  }
+  // drain activation copies in flight
+  for (int b = 0; b < 2; ++b) {
+    if (nloadA[b] > 0 && b < p.nA) drain_bar(p, sm.afullA(b), (uint32_t)((nloadA[b] - 1) & 1));
+    if (nloadB[b] > 0) drain_bar(p, sm.afullB(b), (uint32_t)((nloadB[b] - 1) & 1));
+  }
+}
+
+// ============================================================== signaler ==
+__device__ void signal_loop(const Params& p, const Smem& sm, int ntasks) {
+  const int lane = threadIdx.x & 31;
+  for (int i = 0; i < ntasks; ++i) {
+    const int e = i % kFifo;
+    if (!warp_wait(p, sm, sm.done(e), (i / kFifo) & 1, 300)) break;
+    if (lane == 0) {
+      const int32_t* ent = sm.fifo + e * kFifoEntryWords;
+      const int nsig = ent[D_NSIG];
+      for (int s = 0; s < nsig; ++s) red_release_add(p.counters + ent[D_S0 + s], 1u);
+      mbar_arrive(sm.fempty(e));
+    }
+    __syncwarp();
+  }
+}
+
+// ============================================================= consumers ==
+struct CCtx {
+  const Params* p;
+  const Smem* sm;
+  int ct;     // consumer thread 0..255
+  int cw;     // consumer warp 0..7
+  int lane;
+  uint32_t stage_ctr;
+};
+
+// rstd of each token from the level's sum-of-squares partials (slot A tail)
+__device__ __forceinline__ float level_rstd(const Params& p, const uint8_t* actA, int b) {
+  const float* ss = reinterpret_cast<const float*>(actA + p.actA_frag_bytes);
+  float acc = 0.f;
+  for (int r = 0; r < p.NR; ++r) acc += ss[r * p.B + b];
+  return 1.0f / sqrtf(acc / (float)p.d + p.eps);
+}
+
+// Generic skinny GEMV tile: n_mat matrices x R rows x (KCH*64) columns
+// against the <=8 activation columns in `act` ([kstep][B][4][16 B] hi/lo
+// fragment layout).  Leaves the result in scratch res[m][row][n] (floats).
+__device__ void gemv_tile(CCtx& c, const int32_t* ent, const uint8_t* act, int colsel,
+                          float* res) {
+  const Params& p = *c.p;
+  const Smem& sm = *c.sm;
+  const int nstage = ent[32 + R_NSTAGE];
+  const int nm = ent[D_NMAT], R = ent[D_R];
+  const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
+  const int kl = c.cw / MTn;
+  const int lane = c.lane;
+  const int g8 = lane >> 2, q = lane & 3;
+  const int B = p.B;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // A-operand row/chunk of this lane inside a 16x64 unit (128B-swizzled)
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int achunk_hi = lane >> 4;
+  for (int s = 0; s < nstage; ++s) {
+    const uint32_t slot = c.stage_ctr % sm.NS;
+    const uint32_t ph = (c.stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm, sm.full(slot), ph, 400);
+    __syncwarp();
+    const uint32_t ubase = saddr(sm.ring + (size_t)slot * kStageBytes + c.cw * kUnitBytes);
+    const int kc = s * kcps + kl;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t a0, a1, a2, a3;
+      const int chunk = 2 * i + achunk_hi;
+      ldsm_x4(ubase + arow * 128 + ((chunk ^ (arow & 7)) << 4), a0, a1, a2, a3);
+      const int ks = kc * 4 + i;
+      uint4 bf = make_uint4(0u, 0u, 0u, 0u);
+      if (colsel >= 0)
+        bf = *reinterpret_cast<const uint4*>(act + (((size_t)ks * B + colsel) * 4 + q) * 16);
+      mma16816(acc, a0, a1, a2, a3, bf.x, bf.y);
+      mma16816(acc, a0, a1, a2, a3, bf.z, bf.w);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(slot));
+    ++c.stage_ctr;
+  }
+  // cross-warp reduction over the column chunks that shared a row tile
+  float* part = reinterpret_cast<float*>(sm.scratch);  // [8][16][8]
+  float* pw = part + c.cw * 128;
+  pw[g8 * 8 + 2 * q] = acc[0];
+  pw[g8 * 8 + 2 * q + 1] = acc[1];
+  pw[(g8 + 8) * 8 + 2 * q] = acc[2];
+  pw[(g8 + 8) * 8 + 2 * q + 1] = acc[3];
+  cbar();
+  const int nout = nm * R * 8;
+  for (int idx = c.ct; idx < nout; idx += 256) {
+    const int n = idx & 7;
+    const int row = (idx >> 3) % R;
+    const int m = (idx >> 3) / R;
+    const int mt = row >> 4, r16 = row & 15;
+    float v = 0.f;
+    for (int k2 = 0; k2 < kcps; ++k2) v += part[(k2 * MTn + m * MT + mt) * 128 + r16 * 8 + n];
+    res[idx] = v;  // res[(m*R + row)*8 + n]
+  }
+  cbar();
+}
+
+// Write the normalized attention output o[G][hd] (smem) of token b, group g:
+// fp32 copy and the O-proj B-operand fragments.
+__device__ void write_attn_out(CCtx& c, int layer, int b, int g, const float* o) {
+  const Params& p = *c.p;
+  const int G = p.G, hd = p.hd, B = p.B;
+  float* dst = p.attn_o + ((size_t)layer * B + b) * (size_t)p.Hq * hd + (size_t)g * G * hd;
+  for (int idx = c.ct; idx < G * hd; idx += 256) dst[idx] = o[idx];
+  uint8_t* fr = p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes;
+  const int nent = (G * hd / 16) * 4;
+  for (int t = c.ct; t < nent; t += 256) {
+    const int ks = t >> 2, q = t & 3;
+    const float* v = o + ks * 16 + 2 * q;
+    *reinterpret_cast<uint4*>(fr + (((size_t)ks * B + b) * 4 + q) * 16) =
+        frag_entry(v[0], v[1], v[8], v[9]);
+  }
+}
+
+template <int HD>
+__device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
+  const Params& p = *c.p;
+  const Smem& sm = *c.sm;
+  const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], chunk = ent[D_C];
+  const int flags = ent[D_FLAGS];
+  const int np = ent[32 + R_NTOK], p0 = ent[32 + R_P0], seqlen = ent[32 + R_SEQLEN];
+  const int phys_new = ent[32 + R_PHYS_NEW];
+  const int G = p.G;
+  const int lane = c.lane, g8 = lane >> 2, q = lane & 3;
+  constexpr int HALF = HD / 2;
+  const float* q_raw = reinterpret_cast<const float*>(act);
+  const float* k_raw = q_raw + G * HD;
+  const float* v_raw = k_raw + HD;
+  const float* csv = v_raw + HD;
+  float* mrg = reinterpret_cast<float*>(sm.scratch);       // [8][G][HD+4]
+  float* qs = mrg + 8 * G * (HD + 4);                      // [G][HD]
+  float* kn = qs + G * HD;                                 // [HD]
+  float* vn = kn + HD;                                     // [HD]
+  const float qscale = 1.4426950408889634f / sqrtf((float)HD);
+  for (int idx = c.ct; idx < G * HD; idx += 256) {
+    const int h = idx / HD, i = idx % HD, i1 = i % HALF;
+    const float co = csv[i1], si = csv[HALF + i1];
+    const float x = q_raw[h * HD + i];
+    const float y = (i < HALF) ? q_raw[h * HD + i + HALF] : q_raw[h * HD + i - HALF];
+    const float r = (i < HALF) ? (x * co - y * si) : (x * co + y * si);
+    qs[idx] = r * qscale;
+  }
+  for (int i = c.ct; i < HD; i += 256) {
+    const int i1 = i % HALF;
+    const float co = csv[i1], si = csv[HALF + i1];
+    const float x = k_raw[i];
+    const float y = (i < HALF) ? k_raw[i + HALF] : k_raw[i - HALF];
+    const float r = (i < HALF) ? (x * co - y * si) : (x * co + y * si);
+    const __nv_bfloat16 kb = __float2bfloat16_rn(r);
+    const __nv_bfloat16 vb = __float2bfloat16_rn(v_raw[i]);
+    kn[i] = __bfloat162float(kb);
+    vn[i] = __bfloat162float(vb);
+    if (flags & F_LAST_CHUNK) {
+      const size_t off = (((size_t)phys_new * p.Hkv + g) * kPage + (seqlen % kPage)) * HD + i;
+      reinterpret_cast<__nv_bfloat16*>(p.k_pool[layer])[off] = kb;
+      reinterpret_cast<__nv_bfloat16*>(p.v_pool[layer])[off] = vb;
+    }
+  }
+  cbar();
+  // Q as the A operand: rows [0,G) hi halves, rows [G,2G) lo halves
+  uint32_t qa[HD / 16][2];
+  {
+    const int row = g8;
+    const int h = row < G ? row : (row < 2 * G ? row - G : -1);
+#pragma unroll
+    for (int ks = 0; ks < HD / 16; ++ks) {
+      if (h < 0) {
+        qa[ks][0] = qa[ks][1] = 0u;
+      } else {
+        const float* v = qs + h * HD + ks * 16 + 2 * q;
+        float v0 = v[0], v1 = v[1], v2 = v[8], v3 = v[9];
+        if (row >= G) {
+          v0 -= bf16r(v0);
+          v1 -= bf16r(v1);
+          v2 -= bf16r(v2);
+          v3 -= bf16r(v3);
+        }
+        qa[ks][0] = pack_bf16(v0, v1);
+        qa[ks][1] = pack_bf16(v2, v3);
+      }
+    }
+  }
+  float m_run = -1e30f, l_run = 0.f;
+  float acc[HD / 8][4];
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  // the new token joins the softmax of the chunk that owns it (warp 0)
+  if ((flags & F_LAST_CHUNK) && c.cw == 0) {
+    float sn[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = lane; i < HD; i += 32)
+      for (int h = 0; h < G; ++h) sn[h] += qs[h * HD + i] * kn[i];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      for (int o = 16; o > 0; o >>= 1) sn[h] += __shfl_xor_sync(FULL, sn[h], o);
+    if (g8 < G) {
+      m_run = sn[g8];
+      l_run = 1.f;
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        acc[j][0] = vn[8 * j + 2 * q];
+        acc[j][1] = vn[8 * j + 2 * q + 1];
+      }
+    }
+  }
+  const int key8 = 8 * c.cw;
+  const int krow = key8 + (lane & 7);
+  for (int pi = 0; pi < np; ++pi) {
+    // ---- K page: scores of this warp's 8 keys for the G heads
+    uint32_t slot = c.stage_ctr % sm.NS;
+    uint32_t ph = (c.stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm, sm.full(slot), ph, 401);
+    __syncwarp();
+    uint32_t kb = saddr(sm.ring + (size_t)slot * kStageBytes);
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k2 = 0; k2 < HD / 32; ++k2) {
+      const int hd0 = k2 * 32;
+      const int box = hd0 / 64;
+      const int chunk = ((hd0 % 64) >> 3) + (lane >> 3);
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4(kb + box * 8192 + krow * 128 + ((chunk ^ (krow & 7)) << 4), r0, r1, r2, r3);
+      mma16816(sc, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, r0, r1);
+      mma16816(sc, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, r2, r3);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(slot));
+    ++c.stage_ctr;
+    float s0 = sc[0] + __shfl_down_sync(FULL, sc[0], 4 * G);
+    float s1 = sc[1] + __shfl_down_sync(FULL, sc[1], 4 * G);
+    const int kidx = (p0 + pi) * kPage + key8 + 2 * q;
+    if (kidx >= seqlen) s0 = -INFINITY;
+    if (kidx + 1 >= seqlen) s1 = -INFINITY;
+    float mx = fmaxf(s0, s1);
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = exp2f(m_run - m_new);
+    const float e0 = exp2f(s0 - m_new), e1 = exp2f(s1 - m_new);
+    float ps = e0 + e1;
+    ps += __shfl_xor_sync(FULL, ps, 1);
+    ps += __shfl_xor_sync(FULL, ps, 2);
+    l_run = l_run * alpha + ps;
+    m_run = m_new;
+    // lanes holding the lo rows take their head's scale and probabilities
+    const float alpha_lo = __shfl_up_sync(FULL, alpha, 4 * G);
+    const float e0_lo = __shfl_up_sync(FULL, e0, 4 * G);
+    const float e1_lo = __shfl_up_sync(FULL, e1, 4 * G);
+    float my_alpha = 1.f;
+    uint32_t pa = 0u;
+    if (g8 < G) {
+      my_alpha = alpha;
+      pa = pack_bf16(e0, e1);
+    } else if (g8 < 2 * G) {
+      my_alpha = alpha_lo;
+      pa = pack_bf16(e0_lo - bf16r(e0_lo), e1_lo - bf16r(e1_lo));
+    }
+#pragma unroll
+    for (int j = 0; j < HD / 8; ++j) {
+      acc[j][0] *= my_alpha;
+      acc[j][1] *= my_alpha;
+    }
+    // ---- V page: acc += P V
+    slot = c.stage_ctr % sm.NS;
+    ph = (c.stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm, sm.full(slot), ph, 402);
+    __syncwarp();
+    const uint32_t vb = saddr(sm.ring + (size_t)slot * kStageBytes);
+#pragma unroll
+    for (int j4 = 0; j4 < HD / 32; ++j4) {
+      const int hd0 = j4 * 32;
+      const int box = hd0 / 64;
+      const int chunk = ((hd0 % 64) >> 3) + (lane >> 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(vb + box * 8192 + krow * 128 + ((chunk ^ (krow & 7)) << 4), b0, b1, b2, b3);
+      mma1688(acc[4 * j4 + 0], pa, 0u, b0);
+      mma1688(acc[4 * j4 + 1], pa, 0u, b1);
+      mma1688(acc[4 * j4 + 2], pa, 0u, b2);
+      mma1688(acc[4 * j4 + 3], pa, 0u, b3);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(slot));
+    ++c.stage_ctr;
+  }
+  // ---- per-warp state -> shared memory: O = hi rows + lo rows
+  float* mw = mrg + c.cw * G * (HD + 4);
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) {
+    const float o0 = acc[j][0] + __shfl_down_sync(FULL, acc[j][0], 4 * G);
+    const float o1 = acc[j][1] + __shfl_down_sync(FULL, acc[j][1], 4 * G);
+    if (g8 < G) {
+      mw[g8 * (HD + 4) + 8 * j + 2 * q] = o0;
+      mw[g8 * (HD + 4) + 8 * j + 2 * q + 1] = o1;
+    }
+  }
+  if (g8 < G && q == 0) {
+    mw[g8 * (HD + 4) + HD] = m_run;
+    mw[g8 * (HD + 4) + HD + 1] = l_run;
+  }
+  cbar();
+  // ---- merge the 8 warps
+  float* osm = qs;  // reuse: [G][HD]
+  const bool single = (flags & F_SINGLE) != 0;
+  float* part = p.attn_part +
+                ((((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks + chunk) * p.part_stride;
+  for (int idx = c.ct; idx < G * HD; idx += 256) {
+    const int h = idx / HD, i = idx % HD;
+    float M = -1e30f;
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, mrg[(w * G + h) * (HD + 4) + HD]);
+    float Lsum = 0.f, O = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      const float* mwp = mrg + (w * G + h) * (HD + 4);
+      const float sc = exp2f(mwp[HD] - M);
+      Lsum += sc * mwp[HD + 1];
+      O += sc * mwp[i];
+    }
+    if (single) {
+      osm[idx] = O / Lsum;
+    } else {
+      part[2 * G + idx] = O;
+      if (i == 0) {
+        part[h] = M;
+        part[G + h] = Lsum;
+      }
+    }
+  }
+  if (single) {
+    cbar();
+    write_attn_out(c, layer, b, g, osm);
+  }
+}
+
+__device__ void combine_task(CCtx& c, const int32_t* ent) {
+  const Params& p = *c.p;
+  const Smem& sm = *c.sm;
+  const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], nc = ent[D_D];
+  const int G = p.G, hd = p.hd;
+  const float* parts =
+      p.attn_part + (((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks * (size_t)p.part_stride;
+  float* wsm = reinterpret_cast<float*>(sm.scratch);  // [nc][G]
+  float* ML = wsm + p.max_chunks * G;                 // [2][G]
+  float* osm = ML + 2 * G;                            // [G][hd]
+  if (c.ct < G) {
+    const int h = c.ct;
+    float M = -1e30f;
+    for (int ch = 0; ch < nc; ++ch) M = fmaxf(M, __ldcg(parts + (size_t)ch * p.part_stride + h));
+    float Ls = 0.f;
+    for (int ch = 0; ch < nc; ++ch) {
+      const float* pp = parts + (size_t)ch * p.part_stride;
+      Ls += exp2f(__ldcg(pp + h) - M) * __ldcg(pp + G + h);
+    }
+    ML[h] = M;
+    ML[G + h] = 1.0f / Ls;
+  }
+  cbar();
+  for (int t = c.ct; t < nc * G; t += 256) {
+    const int ch = t / G, h = t % G;
+    wsm[t] = exp2f(__ldcg(parts + (size_t)ch * p.part_stride + h) - ML[h]) * ML[G + h];
+  }
+  cbar();
+  for (int idx = c.ct; idx < G * hd; idx += 256) {
+    const int h = idx / hd;
+    float o = 0.f;
+    for (int ch = 0; ch < nc; ++ch)
+      o += wsm[ch * G + h] * __ldcg(parts + (size_t)ch * p.part_stride + 2 * G + idx);
+    osm[idx] = o;
+  }
+  cbar();
+  write_attn_out(c, layer, b, g, osm);
+}
+
+// fused residual add + RMSNorm statistics for one 64-row tile of level l
+__device__ void rn_task(CCtx& c, const int32_t* ent) {
+  const Params& p = *c.p;
+  const Smem& sm = *c.sm;
+  const int l = ent[D_LAYER], r = ent[D_A];
+  const int B = p.B, d = p.d;
+  float* xs = reinterpret_cast<float*>(sm.scratch);  // [B][64] gamma * x
+  const int b = c.cw;
+  const int col = r * 64 + 2 * c.lane;
+  if (b < B) {
+    float x0, x1;
+    if (l == 0) {
+      int tok = __ldg(p.tokens + b);
+      if (tok < 0 || tok >= p.V) {
+        if (c.lane == 0) raise_error(p, MK_ERR_DEVICE, ent[D_SEQ], OP_RN, -1, tok, p.V, 4);
+        tok = 0;
+      }
+      const uint16_t* er = p.embed + (size_t)tok * d + col;
+      x0 = bf16_to_f(__ldg(er));
+      x1 = bf16_to_f(__ldg(er + 1));
+    } else {
+      const size_t o = (size_t)b * d + col;
+      const float* xp = p.x + (size_t)(l - 1) * B * d;
+      x0 = __ldcg(xp + o);
+      x1 = __ldcg(xp + o + 1);
+      for (int g = 0; g < p.Hkv; ++g) {
+        const float* op = p.o_part + ((size_t)(l - 1) * p.Hkv + g) * B * d;
+        x0 += __ldcg(op + o);
+        x1 += __ldcg(op + o + 1);
+      }
+      for (int j = 0; j < p.k; ++j) {
+        const float* mp = p.moe_part + ((size_t)(l - 1) * p.k + j) * B * d;
+        x0 += __ldcg(mp + o);
+        x1 += __ldcg(mp + o + 1);
+      }
+    }
+    float* xo = p.x + ((size_t)l * B + b) * d + col;
+    xo[0] = x0;
+    xo[1] = x1;
+    const uint16_t* gam = (l < p.L) ? p.attn_norm[l] : p.final_norm;
+    xs[b * 64 + 2 * c.lane] = x0 * bf16_to_f(__ldg(gam + col));
+    xs[b * 64 + 2 * c.lane + 1] = x1 * bf16_to_f(__ldg(gam + col + 1));
+    float ss = x0 * x0 + x1 * x1;
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
+    if (c.lane == 0) {
+      float* ssd = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_frag_bytes);
+      ssd[r * B + b] = ss;
+    }
+  }
+  cbar();
+  uint8_t* fr = p.actA + (size_t)l * p.actA_bytes;
+  for (int t = c.ct; t < 16 * B; t += 256) {
+    const int ksl = t / (4 * B), n = (t >> 2) % B, q = t & 3;
+    const float* v = xs + n * 64 + ksl * 16 + 2 * q;
+    *reinterpret_cast<uint4*>(fr + (((size_t)(4 * r + ksl) * B + n) * 4 + q) * 16) =
+        frag_entry(v[0], v[1], v[8], v[9]);
+  }
+  if (l == 0 && r == 0) {
+    const int half = p.hd / 2;
+    for (int t = c.ct; t < B * half; t += 256) {
+      const int bb = t / half, i = t % half;
+      const int pos = __ldg(p.positions + bb);
+      const int sl = __ldg(p.seq_lens + bb);
+      if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, ent[D_SEQ], OP_RN, -1, pos, sl, 5);
+      double sv, cv;
+      sincos((double)pos * p.inv_freq[i], &sv, &cv);
+      p.cs[(size_t)bb * p.hd + i] = (float)cv;
+      p.cs[(size_t)bb * p.hd + half + i] = (float)sv;
+    }
+  }
+}
+
+// top-k (logit desc, index asc) + softmax over the selected + slot compaction
+__device__ void topk_task(CCtx& c, const int32_t* ent) {
+  const Params& p = *c.p;
+  const Smem& sm = *c.sm;
+  const int l = ent[D_LAYER];
+  const int B = p.B, E = p.E, K = p.k, S = p.S;
+  int32_t* rt = p.route + (size_t)l * p.route_words;
+  int* sel = reinterpret_cast<int*>(sm.scratch);               // [B][8]
+  float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [B][8]
+  int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8); // [E]
+  uint32_t* used = reinterpret_cast<uint32_t*>(slot_of + 256); // [8]
+  if (c.ct < 8) used[c.ct] = 0u;
+  cbar();
+  const int b = c.cw;
+  if (b < B) {
+    const float* lg = p.rlogits + ((size_t)l * B + b) * E;
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int e = c.lane + 32 * t;
+      v[t] = (e < E) ? __ldcg(lg + e) : -INFINITY;
+    }
+    float selv[8];
+    for (int j = 0; j < K; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int e = c.lane + 32 * t;
+        if (e < E && (v[t] > bv || (v[t] == bv && e < bi))) {
+          bv = v[t];
+          bi = e;
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(FULL, bv, o);
+        const int oi = __shfl_xor_sync(FULL, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      selv[j] = bv;
+      if (c.lane == 0) sel[b * 8 + j] = bi;
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (c.lane + 32 * t == bi) v[t] = -INFINITY;
+    }
+    if (c.lane == 0) {
+      float ws[8], sum = 0.f;
+      for (int j = 0; j < K; ++j) {
+        ws[j] = expf(selv[j] - selv[0]);
+        sum += ws[j];
+      }
+      for (int j = 0; j < K; ++j) {
+        const float w = ws[j] / sum;
+        wsel[b * 8 + j] = w;
+        rt[route_topk_idx(B, K) + b * K + j] = sel[b * 8 + j];
+        reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + j] = w;
+        atomicOr(&used[sel[b * 8 + j] >> 5], 1u << (sel[b * 8 + j] & 31));
+      }
+    }
+  }
+  cbar();
+  // slot of each used expert = number of used experts below it
+  for (int e = c.ct; e < E; e += 256) {
+    int cnt = 0;
+    for (int w = 0; w < (e >> 5); ++w) cnt += __popc(used[w]);
+    cnt += __popc(used[e >> 5] & ((1u << (e & 31)) - 1u));
+    slot_of[e] = ((used[e >> 5] >> (e & 31)) & 1u) ? cnt : -1;
+  }
+  cbar();
+  int n_used = 0;
+  for (int w = 0; w < 8; ++w) n_used += __popc(used[w]);
+  for (int s = c.ct; s < S; s += 256) {
+    if (s >= n_used) {
+      rt[route_slot_expert(B, K) + s] = -1;
+      rt[route_slot_ntok(B, K, S) + s] = 0;
+    }
+  }
+  if (c.ct == 0) rt[0] = n_used;
+  // one thread per (token, rank): its position in the slot's token list
+  if (c.ct < B * K) {
+    const int bb = c.ct / K, j = c.ct % K;
+    const int e = sel[bb * 8 + j];
+    const int s = slot_of[e];
+    int pos = 0;
+    for (int b2 = 0; b2 < bb; ++b2)
+      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
+    rt[route_slot_tok(B, K, S) + s * 8 + pos] = bb;
+    rt[route_slot_rank(B, K, S) + s * 8 + pos] = j;
+    reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s * 8 + pos] = wsel[bb * 8 + j];
+    if (pos == 0) {
+      int cnt = 0;
+      for (int b2 = 0; b2 < B; ++b2)
+        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
+      rt[route_slot_expert(B, K) + s] = e;
+      rt[route_slot_ntok(B, K, S) + s] = cnt;
+    }
+  }
+}
+
+__device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
+  CCtx c;
+  c.p = &p;
+  c.sm = &sm;
+  c.ct = threadIdx.x - kFirstConsumerWarp * 32;
+  c.cw = c.ct >> 5;
+  c.lane = threadIdx.x & 31;
+  c.stage_ctr = 0;
+  int nA[2] = {0, 0}, nB[2] = {0, 0};
+  float* res = reinterpret_cast<float*>(sm.scratch) + 8 * 128;  // after the partials
+  for (int i = 0; i < ntasks; ++i) {
+    const int e = i % kFifo;
+    const bool ok = wait_bar(p, sm, sm.ready(e), (i / kFifo) & 1, 500);
+    if (cbar_or(!ok || aborted(sm))) break;
+    const int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    const int op = ent[D_OP];
+    const int flags = ent[D_FLAGS];
+    const int bufA = ent[D_X0], bufB = ent[D_BSLOT];
+    if (flags & F_LOAD_A) {
+      wait_bar(p, sm, sm.afullA(bufA), (uint32_t)(nA[bufA] & 1), 501);
+      nA[bufA]++;
+    }
+    if (flags & F_LOAD_B) {
+      wait_bar(p, sm, sm.afullB(bufB), (uint32_t)(nB[bufB] & 1), 502);
+      nB[bufB]++;
+    }
+    const uint8_t* actA = sm.actA + (size_t)bufA * p.actA_stride;
+    const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
+    const int layer = ent[D_LAYER];
+    const int n = c.lane >> 2;
+    switch (op) {
+      case OP_RN:
+        rn_task(c, ent);
+        break;
+      case OP_TOPK:
+        topk_task(c, ent);
+        break;
+      case OP_COMBINE:
+        combine_task(c, ent);
+        break;
+      case OP_ATTN:
+        if (p.hd == 128)
+          attn_task<128>(c, ent, actB);
+        else
+          attn_task<64>(c, ent, actB);
+        break;
+      case OP_QKV:
+      case OP_ROUTER:
+      case OP_LMHEAD: {
+        gemv_tile(c, ent, actA, n < p.B ? n : -1, res);
+        const int R = ent[D_R], row0 = ent[D_ROW0];
+        for (int idx = c.ct; idx < R * 8; idx += 256) {
+          const int nn = idx / R, r = idx % R;  // r fastest: coalesced rows
+          if (nn >= p.B) continue;
+          const float v = res[r * 8 + nn] * level_rstd(p, actA, nn);
+          const int row = row0 + r;
+          if (op == OP_QKV) {
+            p.qkv[((size_t)layer * p.B + nn) * p.qkvR + row] = v;
+          } else if (op == OP_ROUTER) {
+            if (row < p.E) {
+              const float* bias = p.router_bias[layer];
+              p.rlogits[((size_t)layer * p.B + nn) * p.E + row] = v + (bias ? bias[row] : 0.f);
+            }
+          } else {
+            if (row < p.V) p.logits[(size_t)nn * p.V + row] = v;
+          }
+        }
+        break;
+      }
+      case OP_OPROJ: {
+        gemv_tile(c, ent, actB, n < p.B ? n : -1, res);
+        const int g = ent[D_B], row0 = ent[D_ROW0];
+        for (int idx = c.ct; idx < 64 * 8; idx += 256) {
+          const int nn = idx / 64, r = idx % 64;
+          if (nn >= p.B) continue;
+          p.o_part[(((size_t)layer * p.Hkv + g) * p.B + nn) * p.d + row0 + r] = res[r * 8 + nn];
+        }
+        break;
+      }
+      case OP_GATEUP: {
+        const int ntok = ent[32 + R_NTOK];
+        if (ent[32 + R_EXPERT] < 0) break;
+        const int col = n < ntok ? ent[32 + R_TOK + n] : -1;
+        gemv_tile(c, ent, actA, col, res);
+        const int R = ent[D_R], f = ent[D_B], j = ent[D_A];
+        float* asm_ = res + 2 * R * 8;  // [R][8] activations
+        for (int idx = c.ct; idx < R * 8; idx += 256) {
+          const int nn = idx / R, r = idx % R;
+          float a = 0.f;
+          if (nn < ntok) {
+            const float rs = level_rstd(p, actA, ent[32 + R_TOK + nn]);
+            const float gt = res[r * 8 + nn] * rs;
+            const float ut = res[(R + r) * 8 + nn] * rs;
+            a = gt / (1.0f + expf(-gt)) * ut;
+            p.expert_a[(((size_t)layer * p.S + j) * p.B + nn) * p.F + f * R + r] = a;
+          }
+          asm_[r * 8 + nn] = a;
+        }
+        cbar();
+        uint8_t* fr = p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes;
+        const int nent = (R / 16) * ntok * 4;
+        for (int t = c.ct; t < nent; t += 256) {
+          const int ksl = t / (4 * ntok), nn = (t >> 2) % ntok, q = t & 3;
+          const int r0 = ksl * 16 + 2 * q;
+          const uint4 fe = frag_entry(asm_[r0 * 8 + nn], asm_[(r0 + 1) * 8 + nn],
+                                      asm_[(r0 + 8) * 8 + nn], asm_[(r0 + 9) * 8 + nn]);
+          const int ks = f * (R / 16) + ksl;
+          *reinterpret_cast<uint4*>(fr + (((size_t)ks * p.B + nn) * 4 + q) * 16) = fe;
+        }
+        break;
+      }
+      case OP_DOWN: {
+        const int ntok = ent[32 + R_NTOK];
+        if (ent[32 + R_EXPERT] < 0) break;
+        gemv_tile(c, ent, actB, n < ntok ? n : -1, res);
+        const int row0 = ent[D_ROW0];
+        for (int idx = c.ct; idx < 64 * 8; idx += 256) {
+          const int nn = idx / 64, r = idx % 64;
+          if (nn >= ntok) continue;
+          const int tok = ent[32 + R_TOK + nn];
+          const int rank = ent[32 + R_RANK + nn];
+          const float w = __int_as_float(ent[32 + R_W + nn]);
+          p.moe_part[(((size_t)layer * p.k + rank) * p.B + tok) * p.d + row0 + r] =
+              w * res[r * 8 + nn];
+        }
+        break;
+      }
+      default:
+        break;
+    }
+    cbar();
+    if (c.ct == 0) {
+      if (flags & F_REL_A) mbar_arrive(sm.aemptyA(bufA));
+      if (flags & F_LOAD_B) mbar_arrive(sm.aemptyB(bufB));
+      mbar_arrive(sm.done(e));
+    }
+    if (cbar_or(aborted(sm))) break;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_abort;
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Smem sm;
+  sm.base = base;
+  sm.ring = base + p.off_ring;
+  sm.bars = reinterpret_cast<uint64_t*>(base + p.off_bars);
+  sm.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
+  sm.scratch = base + p.off_scratch;
+  sm.actA = base + p.off_actA;
+  sm.actB = base + p.off_actB;
+  sm.NS = p.n_stages;
+  sm.abort_flag = &s_abort;
+  const int warp = threadIdx.x >> 5;
+  const int cta = blockIdx.x;
+  const int ntasks = p.ntasks[cta];
+  const int32_t* my = p.desc + (size_t)cta * p.max_tasks * kDescWords;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < sm.NS; ++s) {
+      mbar_init(sm.full(s), 1);
+      mbar_init(sm.empty(s), kConsumerWarps);
+    }
+    for (int e = 0; e < kFifo; ++e) {
+      mbar_init(sm.ready(e), 2);
+      mbar_init(sm.done(e), 1);
+      mbar_init(sm.fempty(e), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sm.afullA(b), 1);
+      mbar_init(sm.aemptyA(b), 1);
+      mbar_init(sm.afullB(b), 1);
+      mbar_init(sm.aemptyB(b), 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == kProducerWarp) {
+    producer_loop(p, sm, my, ntasks);
+  } else if (warp == kLoaderWarp) {
+    loader_loop(p, sm, my, ntasks);
+  } else if (warp == kSignalWarp) {
+    signal_loop(p, sm, ntasks);
+  } else {
+    consumer_loop(p, sm, ntasks);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+// Launch one step (or one phase) of the interpreter: cooperative, so that all
+// CTAs are guaranteed co-resident (the counter waits rely on it).
+cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream) {
+  static int configured_bytes = -1;
+  if (configured_bytes != p.smem_bytes) {
+    cudaError_t e =
+        cudaFuncSetAttribute(mk_interp, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+    if (e != cudaSuccess) return e;
+    configured_bytes = p.smem_bytes;
+  }
+  void* args[] = {const_cast<Params*>(&p)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(mk_interp), dim3(grid),
+                                     dim3(kThreads), args, (size_t)p.smem_bytes, stream);
+}
+
+cudaError_t max_coresident(int smem_bytes, int* blocks_per_sm) {
+  cudaError_t e =
+      cudaFuncSetAttribute(mk_interp, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_interp, kThreads,
+                                                       (size_t)smem_bytes);
+}
+
+}  // namespace mk

@@ -1,0 +1,646 @@
+// mk_plan.cpp -- host schedule builder: decode step -> per-CTA task lists.
+//
+// Every operation of the step is cut into tiles, one task per tile, emitted in
+// one global topological order (per layer: residual/norm tiles, QKV and router
+// tiles, top-k, attention chunks, combines, O-proj, expert gate/up, expert
+// down; then the final norm and the LM head).  Each task is appended to the
+// list of the CTA that a small list-scheduling simulation says finishes it
+// first, so any free SM picks up any ready tile and no work is rounded up to
+// whole waves (agenticcommons.xyz, "Cohere North Mini Code megakernel serving
+// engine", section "Three sources of speedup", item 1).  Because every list is
+// a subsequence of one topological order and all CTAs are co-resident, every
+// wait is on work that is earlier in that order, so the step cannot deadlock.
+//
+// Dependencies are counters, one per producer group, with per-step arrival
+// counts; a task waits until counter >= epoch * arrivals (section "How the
+// megakernel works": increment on completion, spin on the producer).  The
+// O-proj of one KV group waits only for that group's attention, and the down
+// projection of one expert only for that expert's gate/up tiles (section
+// "Three sources of speedup", item 2).
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+
+void Plan::release() {
+  std::free(desc);
+  std::free(counts);
+  std::free(targets);
+  std::free(phase_desc);
+  std::free(phase_counts);
+  desc = counts = targets = phase_desc = phase_counts = nullptr;
+}
+
+static int gcd_int(int a, int b) {
+  while (b) {
+    int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+// Rows per GEMV tile: a ring stage holds 8 units of 16 rows x 64 columns; a
+// tile of n_mat matrices x R rows consumes stages of (8 / (n_mat*R/16)) column
+// chunks each, which must divide the K/64 chunks of the row.
+int gemv_rows_for(int K, int n_mat) {
+  int kc = K / 64;
+  int per_stage = 8 / n_mat;                  // units per stage per matrix
+  int kcps = gcd_int(per_stage, kc);          // column chunks per stage
+  int mt = per_stage / kcps;                  // 16-row tiles per matrix
+  return 16 * mt;
+}
+
+int validate_shape(const Shape& s) {
+  if (s.L < 1 || s.d < 128 || s.d % 64 != 0 || s.d > 16384) return MK_ERR_INVALID;
+  if (s.hd != 64 && s.hd != 128) return MK_ERR_INVALID;
+  if (s.Hkv < 1 || s.Hq < s.Hkv || s.Hq % s.Hkv != 0) return MK_ERR_INVALID;
+  const int G = s.Hq / s.Hkv;
+  if (G > 4) return MK_ERR_CAPACITY;
+  if ((G * s.hd) % 128 != 0) return MK_ERR_INVALID;
+  const int r_qkv = gemv_rows_for(s.d, 1);
+  if (r_qkv > s.hd || s.hd % r_qkv != 0) return MK_ERR_INVALID;
+  if (s.E < 1 || s.E > 256) return MK_ERR_CAPACITY;
+  if (s.k < 1 || s.k > kMaxTopK || s.k > s.E) return MK_ERR_INVALID;
+  if (s.F < 128 || s.F % 128 != 0) return MK_ERR_INVALID;
+  if (s.F % gemv_rows_for(s.d, 2) != 0) return MK_ERR_INVALID;
+  if (s.V < 1) return MK_ERR_INVALID;
+  if (s.page != kPage) return MK_ERR_INVALID;
+  if (s.max_batch < 1 || s.max_batch > kMaxBatch) return MK_ERR_INVALID;
+  if (s.n_pages < 1) return MK_ERR_INVALID;
+  if (!(s.eps > 0.0f) || !(s.theta > 0.0f)) return MK_ERR_INVALID;
+  return MK_OK;
+}
+
+static int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
+  const int G = s.Hq / s.Hkv;
+  const int NR = s.d / 64;
+  const int actA_bytes = 4 * s.d * B + round_up(NR * B * 4, 16);
+  o->actA_stride = round_up(actA_bytes, 128);
+  int b_need = std::max(4 * G * s.hd * B, std::max(4 * s.F * B, (G + 3) * s.hd * 4));
+  o->actB_bytes = round_up(b_need, 128);
+  int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
+  int sc_gemv = 8 * 512 + 1024 * 4 + 64;
+  int sc_topk = B * s.E * 4 + B * 8 * 8 + s.E * 4 + 256;
+  int sc_rn = B * 64 * 4 + 64;
+  int sc_comb = max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
+  int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
+  o->scratch_bytes = round_up(sc, 1024);
+  const int fifo = kFifo * kFifoEntryWords * 4;
+  const int max_stages = 14;
+  const int bars = round_up((2 * max_stages + 3 * kFifo + 8) * 8, 1024);
+  const int budget = 232448 - 1024;
+  int rest1 = bars + fifo + o->scratch_bytes + o->actA_stride + 2 * o->actB_bytes;
+  int rest2 = rest1 + o->actA_stride;
+  int nA = ((budget - rest2) / kStageBytes >= 8) ? 2 : 1;
+  int rest = nA == 2 ? rest2 : rest1;
+  int ns = std::min(max_stages, (budget - rest) / kStageBytes);
+  if (ns < 2) return MK_ERR_CAPACITY;
+  o->nA = nA;
+  o->n_stages = ns;
+  o->off_ring = 0;
+  o->off_bars = ns * kStageBytes;
+  o->off_fifo = o->off_bars + bars;
+  o->off_scratch = o->off_fifo + fifo;
+  o->off_actA = o->off_scratch + o->scratch_bytes;
+  o->off_actB = o->off_actA + nA * o->actA_stride;
+  o->total = o->off_actB + 2 * o->actB_bytes;
+  o->dyn_bytes = o->total + 1024;
+  return MK_OK;
+}
+
+namespace {
+
+enum ActKind { ACT_NONE = 0, ACT_A = 1, ACT_B = 2 };
+
+struct Task {
+  int32_t w[kDescWords];
+  double bytes;
+  int act;
+  int keyA;
+};
+
+struct Layout {
+  int L, B, S, Hkv, NR;
+  int norm0, qkv0, rpart0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
+  void build(int L_, int B_, int S_, int Hkv_, int NR_) {
+    L = L_; B = B_; S = S_; Hkv = Hkv_; NR = NR_;
+    int c = 0;
+    norm0 = c; c += L + 1;
+    qkv0 = c; c += L * Hkv;
+    rpart0 = c; c += L;
+    rtr0 = c; c += L;
+    attp0 = c; c += L * B * Hkv;
+    atto0 = c; c += L * Hkv;
+    slot0 = c; c += L * S;
+    dt0 = c; c += L * NR;
+    lmdone = c; c += 1;
+    total = c;
+  }
+  int norm(int l) const { return norm0 + l; }
+  int qkv(int l, int g) const { return qkv0 + l * Hkv + g; }
+  int rpart(int l) const { return rpart0 + l; }
+  int rtr(int l) const { return rtr0 + l; }
+  int attp(int l, int b, int g) const { return attp0 + (l * B + b) * Hkv + g; }
+  int atto(int l, int g) const { return atto0 + l * Hkv + g; }
+  int slot(int l, int j) const { return slot0 + l * S + j; }
+  int dt(int l, int r) const { return dt0 + l * NR + r; }
+};
+
+Task make_task(int op, int layer, int phase) {
+  Task t;
+  std::memset(t.w, 0, sizeof(t.w));
+  t.w[D_OP] = op;
+  t.w[D_LAYER] = layer;
+  t.w[D_PW] = -1;
+  t.w[D_PWN] = 0;
+  t.w[D_W0] = -1;
+  t.w[D_W1] = -1;
+  t.w[D_S0] = -1;
+  t.w[D_S1] = -1;
+  t.w[D_MAP0] = -1;
+  t.w[D_MAP1] = -1;
+  t.w[D_PHASE] = phase;
+  t.bytes = 0.0;
+  t.act = ACT_NONE;
+  t.keyA = -1;
+  return t;
+}
+
+void add_wait(Task& t, int ctr, int n) {
+  int i = t.w[D_NWAIT]++;
+  t.w[D_W0 + 2 * i] = ctr;
+  t.w[D_W0N + 2 * i] = n;
+}
+void add_signal(Task& t, int ctr) {
+  int i = t.w[D_NSIG]++;
+  t.w[D_S0 + i] = ctr;
+}
+
+// Simulated list scheduling: place each task on the CTA where it would
+// finish first, given per-CTA HBM stream time and consumer time, a ring that
+// lets the stream run ahead of the consumer, and counter-dependency times.
+struct Sim {
+  int n;
+  double bw;        // bytes per microsecond per CTA
+  double hop;       // counter visibility latency
+  double ovh;       // per-task consumer overhead
+  double ring_us;   // how far the stream may run ahead of the consumer
+  std::vector<double> t_stream, t_done;
+  std::vector<double> ctr_time;
+
+  int place(const Task& t) {
+    double dep = 0.0;
+    for (int i = 0; i < t.w[D_NWAIT]; ++i)
+      dep = std::max(dep, ctr_time[t.w[D_W0 + 2 * i]] + hop);
+    double pdep = 0.0;
+    if (t.w[D_PW] >= 0) pdep = ctr_time[t.w[D_PW]] + hop;
+    int best = 0;
+    double best_fin = 1e300, best_ss = 1e300, best_se = 0.0;
+    for (int c = 0; c < n; ++c) {
+      double ss = std::max(std::max(t_stream[c], t_done[c] - ring_us), pdep);
+      double se = ss + t.bytes / bw;
+      double fin = std::max(std::max(se, dep), t_done[c]) + ovh;
+      if (fin < best_fin - 1e-9 || (fin < best_fin + 1e-9 && t_stream[c] < best_ss)) {
+        best = c;
+        best_fin = fin;
+        best_ss = t_stream[c];
+        best_se = se;
+      }
+    }
+    t_stream[best] = std::max(t_stream[best], best_se);
+    t_done[best] = best_fin;
+    for (int i = 0; i < t.w[D_NSIG]; ++i) {
+      int s = t.w[D_S0 + i];
+      ctr_time[s] = std::max(ctr_time[s], best_fin);
+    }
+    return best;
+  }
+};
+
+// Mark slot usage along one CTA list: a normalized-input activation is loaded
+// when its level changes (into alternating buffers when two fit) and released
+// after its last use; every small activation is loaded into the next of two
+// buffers and released after its task.
+void mark_list(std::vector<Task*>& lst, int nA) {
+  int cur_key = -1, cur_buf = -1, n_loads = 0;
+  Task* last_a = nullptr;
+  int nb = 0;
+  for (size_t i = 0; i < lst.size(); ++i) {
+    Task& t = *lst[i];
+    t.w[D_SEQ] = (int32_t)i;
+    t.w[D_FLAGS] &= ~(F_LOAD_A | F_REL_A | F_LOAD_B);
+    if (t.act == ACT_A) {
+      if (t.keyA != cur_key) {
+        if (last_a) last_a->w[D_FLAGS] |= F_REL_A;
+        cur_buf = n_loads % nA;
+        ++n_loads;
+        cur_key = t.keyA;
+        t.w[D_FLAGS] |= F_LOAD_A;
+      }
+      t.w[D_X0] = cur_buf;
+      last_a = &t;
+    } else if (t.act == ACT_B) {
+      t.w[D_FLAGS] |= F_LOAD_B;
+      t.w[D_BSLOT] = nb & 1;
+      ++nb;
+    }
+  }
+  if (last_a) last_a->w[D_FLAGS] |= F_REL_A;
+}
+
+}  // namespace
+
+int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
+                  const int32_t* plan_len, bool with_phases, Plan* out) {
+  if (!out || n_ctas < 1 || B < 1 || B > s.max_batch || B > kMaxBatch) return MK_ERR_INVALID;
+  if (!seq_lens) return MK_ERR_INVALID;
+  const int L = s.L, d = s.d, hd = s.hd, Hq = s.Hq, Hkv = s.Hkv, E = s.E, k = s.k, F = s.F;
+  const int G = Hq / Hkv;
+  const int NR = d / 64;
+  const int S = std::min(E, B * k);
+  const int qkvR = (Hq + 2 * Hkv) * hd;
+  const int r_qkv = gemv_rows_for(d, 1);
+  const int r_ff = gemv_rows_for(d, 2);
+  const int n_qkv = qkvR / r_qkv;
+  const int n_rt = (E + r_qkv - 1) / r_qkv;
+  const int n_ff = F / r_ff;
+  const int n_lm = (s.V + 127) / 128;
+  if (r_qkv > hd || hd % r_qkv != 0) return MK_ERR_INVALID;
+
+  // ---- attention chunk plan: whole pages, chunks sized so that the step's
+  // KV stream spreads over all CTAs.
+  int cap_pages[kMaxBatch];
+  long total_pages = 0;
+  for (int b = 0; b < B; ++b) {
+    if (seq_lens[b] < 0) return MK_ERR_INVALID;
+    long pl = plan_len ? (long)plan_len[b] : (long)seq_lens[b] + kPage;
+    if (pl < seq_lens[b]) return MK_ERR_INVALID;
+    cap_pages[b] = (int)((pl + kPage - 1) / kPage);
+    total_pages += (long)cap_pages[b] * Hkv;
+  }
+  long ppc_all = std::max(1L, (total_pages + n_ctas - 1) / n_ctas);
+  int max_chunks = 1;
+  for (int b = 0; b < B; ++b) {
+    out->ppc[b] = (int)ppc_all;
+    out->nc[b] = std::max(1, (int)((cap_pages[b] + ppc_all - 1) / ppc_all));
+    max_chunks = std::max(max_chunks, out->nc[b]);
+  }
+
+  Layout lay;
+  lay.build(L, B, S, Hkv, NR);
+  std::vector<int32_t> targets(lay.total, 0);
+
+  // Expected use of expert slot j: slots are compacted in expert order, so
+  // low slots fill first; estimate E[#distinct experts] under uniform routing.
+  double exp_used = E * (1.0 - std::pow(1.0 - (double)k / E, (double)B));
+  auto p_slot = [&](int j) {
+    double p = exp_used - j;
+    return p >= 1.0 ? 1.0 : (p <= 0.0 ? 0.05 : std::max(0.05, p));
+  };
+
+  std::vector<Task> tasks;
+  tasks.reserve((size_t)L * (NR + n_qkv + n_rt + 1 + 2 * B * Hkv * max_chunks + NR * Hkv +
+                             S * (n_ff + NR)) + NR + n_lm + 16);
+  const int PH = 8;  // phases per layer
+  auto map_of = [&](int l, int which) { return l * kMapsPerLayer + which; };
+
+  for (int l = 0; l <= L; ++l) {
+    // -- fused residual add + RMSNorm tiles producing level l
+    for (int r = 0; r < NR; ++r) {
+      Task t = make_task(OP_RN, l, l * PH + 0);
+      t.w[D_A] = r;
+      if (l > 0) add_wait(t, lay.dt(l - 1, r), Hkv + S);
+      add_signal(t, lay.norm(l));
+      targets[lay.norm(l)] += 1;
+      tasks.push_back(t);
+    }
+    if (l == L) break;
+    // -- QKV tiles (grouped by KV group so attention of a group starts early)
+    for (int g = 0; g < Hkv; ++g) {
+      auto emit_rows = [&](int row_begin, int rows) {
+        for (int r0 = row_begin; r0 < row_begin + rows; r0 += r_qkv) {
+          Task t = make_task(OP_QKV, l, l * PH + 1);
+          t.w[D_A] = r0 / r_qkv;
+          t.w[D_B] = g;
+          t.w[D_ROW0] = r0;
+          t.w[D_K0] = 0;
+          t.w[D_KCH] = d / 64;
+          t.w[D_R] = r_qkv;
+          t.w[D_NMAT] = 1;
+          t.w[D_MAP0] = map_of(l, 0);
+          t.w[D_NSTAGE] = (r_qkv / 16) * (d / 64) / 8;
+          add_wait(t, lay.norm(l), NR);
+          add_signal(t, lay.qkv(l, g));
+          targets[lay.qkv(l, g)] += 1;
+          t.bytes = (double)r_qkv * d * 2;
+          t.act = ACT_A;
+          t.keyA = l;
+          tasks.push_back(t);
+        }
+      };
+      emit_rows(g * G * hd, G * hd);            // q heads of the group
+      emit_rows(Hq * hd + g * hd, hd);          // k head
+      emit_rows((Hq + Hkv) * hd + g * hd, hd);  // v head
+    }
+    // -- router tiles
+    for (int t_i = 0; t_i < n_rt; ++t_i) {
+      Task t = make_task(OP_ROUTER, l, l * PH + 1);
+      t.w[D_A] = t_i;
+      t.w[D_ROW0] = t_i * r_qkv;
+      t.w[D_K0] = 0;
+      t.w[D_KCH] = d / 64;
+      t.w[D_R] = r_qkv;
+      t.w[D_NMAT] = 1;
+      t.w[D_MAP0] = map_of(l, 2);
+      t.w[D_NSTAGE] = (r_qkv / 16) * (d / 64) / 8;
+      add_wait(t, lay.norm(l), NR);
+      add_signal(t, lay.rpart(l));
+      targets[lay.rpart(l)] += 1;
+      t.bytes = (double)std::min(r_qkv, E - t_i * r_qkv) * d * 2;
+      t.act = ACT_A;
+      t.keyA = l;
+      tasks.push_back(t);
+    }
+    {
+      Task t = make_task(OP_TOPK, l, l * PH + 2);
+      add_wait(t, lay.rpart(l), n_rt);
+      add_signal(t, lay.rtr(l));
+      targets[lay.rtr(l)] += 1;
+      tasks.push_back(t);
+    }
+    // -- attention chunks, then combines
+    for (int g = 0; g < Hkv; ++g) {
+      for (int b = 0; b < B; ++b) {
+        int nc = out->nc[b];
+        for (int c = 0; c < nc; ++c) {
+          Task t = make_task(OP_ATTN, l, l * PH + 3);
+          t.w[D_A] = b;
+          t.w[D_B] = g;
+          t.w[D_C] = c;
+          t.w[D_D] = nc;
+          t.w[D_PPC] = out->ppc[b];
+          t.w[D_MAP0] = map_of(l, 6);
+          t.w[D_MAP1] = map_of(l, 7);
+          if (c == nc - 1) t.w[D_FLAGS] |= F_LAST_CHUNK;
+          if (nc == 1) t.w[D_FLAGS] |= F_SINGLE;
+          add_wait(t, lay.qkv(l, g), (G * hd + 2 * hd) / r_qkv);
+          int sig = nc > 1 ? lay.attp(l, b, g) : lay.atto(l, g);
+          add_signal(t, sig);
+          targets[sig] += 1;
+          long p0 = (long)c * out->ppc[b];
+          long pages_now = ((long)seq_lens[b] + kPage - 1) / kPage;
+          long np = std::max(0L, std::min((long)out->ppc[b], pages_now - p0));
+          t.bytes = (double)np * 2.0 * kPage * hd * 2.0;
+          t.act = ACT_B;
+          tasks.push_back(t);
+        }
+      }
+    }
+    for (int g = 0; g < Hkv; ++g) {
+      for (int b = 0; b < B; ++b) {
+        if (out->nc[b] <= 1) continue;
+        Task t = make_task(OP_COMBINE, l, l * PH + 4);
+        t.w[D_A] = b;
+        t.w[D_B] = g;
+        t.w[D_D] = out->nc[b];
+        add_wait(t, lay.attp(l, b, g), out->nc[b]);
+        add_signal(t, lay.atto(l, g));
+        targets[lay.atto(l, g)] += 1;
+        tasks.push_back(t);
+      }
+    }
+    // -- O-proj: (64-row tile, KV group)
+    for (int g = 0; g < Hkv; ++g) {
+      for (int r = 0; r < NR; ++r) {
+        Task t = make_task(OP_OPROJ, l, l * PH + 5);
+        t.w[D_A] = r;
+        t.w[D_B] = g;
+        t.w[D_ROW0] = r * 64;
+        t.w[D_K0] = g * G * hd;
+        t.w[D_KCH] = G * hd / 64;
+        t.w[D_R] = 64;
+        t.w[D_NMAT] = 1;
+        t.w[D_MAP0] = map_of(l, 1);
+        t.w[D_NSTAGE] = 4 * (G * hd / 64) / 8;
+        add_wait(t, lay.atto(l, g), B);
+        add_signal(t, lay.dt(l, r));
+        targets[lay.dt(l, r)] += 1;
+        t.bytes = 64.0 * G * hd * 2;
+        t.act = ACT_B;
+        tasks.push_back(t);
+      }
+    }
+    // -- experts: gate/up tiles per slot, then down tiles per slot
+    for (int j = 0; j < S; ++j) {
+      for (int f = 0; f < n_ff; ++f) {
+        Task t = make_task(OP_GATEUP, l, l * PH + 6);
+        t.w[D_A] = j;
+        t.w[D_B] = f;
+        t.w[D_ROW0] = f * r_ff;
+        t.w[D_K0] = 0;
+        t.w[D_KCH] = d / 64;
+        t.w[D_R] = r_ff;
+        t.w[D_NMAT] = 2;
+        t.w[D_MAP0] = map_of(l, 3);
+        t.w[D_MAP1] = map_of(l, 4);
+        t.w[D_NSTAGE] = 2 * (r_ff / 16) * (d / 64) / 8;
+        t.w[D_PW] = lay.rtr(l);
+        t.w[D_PWN] = 1;
+        add_wait(t, lay.norm(l), NR);
+        add_signal(t, lay.slot(l, j));
+        targets[lay.slot(l, j)] += 1;
+        t.bytes = 2.0 * r_ff * d * 2 * p_slot(j);
+        t.act = ACT_A;
+        t.keyA = l;
+        tasks.push_back(t);
+      }
+    }
+    for (int j = 0; j < S; ++j) {
+      for (int r = 0; r < NR; ++r) {
+        Task t = make_task(OP_DOWN, l, l * PH + 7);
+        t.w[D_A] = j;
+        t.w[D_B] = r;
+        t.w[D_ROW0] = r * 64;
+        t.w[D_K0] = 0;
+        t.w[D_KCH] = F / 64;
+        t.w[D_R] = 64;
+        t.w[D_NMAT] = 1;
+        t.w[D_MAP0] = map_of(l, 5);
+        t.w[D_NSTAGE] = 4 * (F / 64) / 8;
+        t.w[D_PW] = lay.rtr(l);
+        t.w[D_PWN] = 1;
+        add_wait(t, lay.slot(l, j), n_ff);
+        add_signal(t, lay.dt(l, r));
+        targets[lay.dt(l, r)] += 1;
+        t.bytes = 64.0 * F * 2 * p_slot(j);
+        t.act = ACT_B;
+        tasks.push_back(t);
+      }
+    }
+  }
+  // -- LM head
+  for (int t_i = 0; t_i < n_lm; ++t_i) {
+    Task t = make_task(OP_LMHEAD, L, L * PH + 1);
+    t.w[D_A] = t_i;
+    t.w[D_ROW0] = t_i * 128;
+    t.w[D_K0] = 0;
+    t.w[D_KCH] = d / 64;
+    t.w[D_R] = 128;
+    t.w[D_NMAT] = 1;
+    t.w[D_MAP0] = L * kMapsPerLayer;
+    t.w[D_NSTAGE] = 8 * (d / 64) / 8;
+    add_wait(t, lay.norm(L), NR);
+    add_signal(t, lay.lmdone);
+    targets[lay.lmdone] += 1;
+    t.bytes = 128.0 * d * 2;
+    t.act = ACT_A;
+    t.keyA = L;
+    tasks.push_back(t);
+  }
+
+  // ---- placement
+  Sim sim;
+  sim.n = n_ctas;
+  sim.bw = 6.5e12 / 1e6 / n_ctas;
+  sim.hop = 1.0;
+  sim.ovh = 0.25;
+  sim.ring_us = 160.0 * 1024.0 / sim.bw;
+  sim.t_stream.assign(n_ctas, 0.0);
+  sim.t_done.assign(n_ctas, 0.0);
+  sim.ctr_time.assign(lay.total, 0.0);
+  std::vector<std::vector<Task*>> lists(n_ctas);
+  for (auto& t : tasks) lists[sim.place(t)].push_back(&t);
+
+  // A-slot double buffering only where two buffers fit in shared memory.
+  SmemLayout sl;
+  int slrc = smem_layout(s, B, max_chunks, &sl);
+  if (slrc != MK_OK) return slrc;
+  const int nA = sl.nA;
+  int max_tasks = 0;
+  for (auto& lst : lists) {
+    mark_list(lst, nA);
+    max_tasks = std::max(max_tasks, (int)lst.size());
+  }
+  max_tasks = std::max(max_tasks, 1);
+
+  out->release();
+  out->n_ctas = n_ctas;
+  out->B = B;
+  out->S = S;
+  out->max_chunks = max_chunks;
+  out->n_counters = lay.total;
+  out->max_tasks = max_tasks;
+  out->total_tasks = tasks.size();
+  out->r_qkv = r_qkv;
+  out->r_router = r_qkv;
+  out->n_phases = L * PH + 2;
+  out->desc = (int32_t*)std::calloc((size_t)n_ctas * max_tasks * kDescWords, sizeof(int32_t));
+  out->counts = (int32_t*)std::calloc((size_t)n_ctas, sizeof(int32_t));
+  out->targets = (int32_t*)std::calloc((size_t)lay.total, sizeof(int32_t));
+  if (!out->desc || !out->counts || !out->targets) {
+    out->release();
+    return MK_ERR_OOM;
+  }
+  for (int c = 0; c < n_ctas; ++c) {
+    out->counts[c] = (int32_t)lists[c].size();
+    for (size_t i = 0; i < lists[c].size(); ++i)
+      std::memcpy(out->desc + ((size_t)c * max_tasks + i) * kDescWords, lists[c][i]->w,
+                  sizeof(int32_t) * kDescWords);
+  }
+  std::memcpy(out->targets, targets.data(), sizeof(int32_t) * lay.total);
+
+  if (with_phases) {
+    // one launch per phase; inside a phase the tiles are spread like a
+    // conventional kernel's grid: least-loaded CTA by bytes.
+    const int nph = out->n_phases;
+    std::vector<std::vector<std::vector<Task*>>> pl(nph, std::vector<std::vector<Task*>>(n_ctas));
+    std::vector<std::vector<double>> load(nph, std::vector<double>(n_ctas, 0.0));
+    std::vector<int> rr(nph, 0);
+    for (auto& t : tasks) {
+      int ph = t.w[D_PHASE];
+      int best = 0;
+      double bl = 1e300;
+      for (int c = 0; c < n_ctas; ++c) {
+        int cc = (rr[ph] + c) % n_ctas;
+        if (load[ph][cc] < bl - 1e-9) {
+          bl = load[ph][cc];
+          best = cc;
+        }
+      }
+      rr[ph] = (best + 1) % n_ctas;
+      load[ph][best] += t.bytes + 4096.0;
+      pl[ph][best].push_back(&t);
+    }
+    int pmax = 1;
+    for (int ph = 0; ph < nph; ++ph)
+      for (int c = 0; c < n_ctas; ++c) pmax = std::max(pmax, (int)pl[ph][c].size());
+    out->phase_max_tasks = pmax;
+    out->phase_desc =
+        (int32_t*)std::calloc((size_t)nph * n_ctas * pmax * kDescWords, sizeof(int32_t));
+    out->phase_counts = (int32_t*)std::calloc((size_t)nph * n_ctas, sizeof(int32_t));
+    if (!out->phase_desc || !out->phase_counts) {
+      out->release();
+      return MK_ERR_OOM;
+    }
+    for (int ph = 0; ph < nph; ++ph) {
+      for (int c = 0; c < n_ctas; ++c) {
+        auto& lst = pl[ph][c];
+        // flags depend on list order: mark a private copy
+        std::vector<Task> copy;
+        copy.reserve(lst.size());
+        for (auto* t : lst) copy.push_back(*t);
+        std::vector<Task*> ptrs;
+        for (auto& t : copy) ptrs.push_back(&t);
+        mark_list(ptrs, nA);
+        out->phase_counts[(size_t)ph * n_ctas + c] = (int32_t)copy.size();
+        for (size_t i = 0; i < copy.size(); ++i)
+          std::memcpy(out->phase_desc + (((size_t)ph * n_ctas + c) * pmax + i) * kDescWords,
+                      copy[i].w, sizeof(int32_t) * kDescWords);
+      }
+    }
+  }
+  return MK_OK;
+}
+
+}  // namespace mk
+
+extern "C" mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batch,
+                                      const int32_t* seq_lens, const int32_t* plan_len,
+                                      int32_t* meta, int32_t* counts, int32_t* desc,
+                                      int32_t* targets) {
+  if (!cfg || !meta) return MK_ERR_INVALID;
+  mk::Shape s{cfg->n_layers, cfg->d_model, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+              cfg->n_experts, cfg->top_k, cfg->d_ff, cfg->vocab, cfg->page_size,
+              cfg->max_batch, cfg->n_pages, cfg->rope_theta, cfg->rms_eps};
+  int v = mk::validate_shape(s);
+  if (v != MK_OK) return (mk_status)v;
+  mk::Plan p;
+  int rc = mk::plan_schedule(s, n_ctas, batch, seq_lens, plan_len, false, &p);
+  if (rc != MK_OK) return (mk_status)rc;
+  std::memset(meta, 0, 16 * sizeof(int32_t));
+  meta[0] = p.n_ctas;
+  meta[1] = p.max_tasks;
+  meta[2] = (int32_t)p.total_tasks;
+  meta[3] = p.n_counters;
+  meta[4] = p.S;
+  meta[5] = p.max_chunks;
+  meta[6] = mk::kDescWords;
+  meta[7] = p.n_phases;
+  meta[8] = p.r_qkv;
+  meta[9] = p.ppc[0];
+  if (counts) std::memcpy(counts, p.counts, sizeof(int32_t) * p.n_ctas);
+  if (desc)
+    std::memcpy(desc, p.desc, sizeof(int32_t) * (size_t)p.n_ctas * p.max_tasks * mk::kDescWords);
+  if (targets) std::memcpy(targets, p.targets, sizeof(int32_t) * p.n_counters);
+  p.release();
+  return MK_OK;
+}

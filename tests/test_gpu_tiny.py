@@ -1,0 +1,168 @@
+"""GPU parity on the tiny model: the CUDA path vs the CPU oracle, element by
+element, through the C ABI (sizes that span several tiles and ragged tails)."""
+
+import numpy as np
+import pytest
+import torch
+
+from moe_persistent_cta_b200 import configs, mk
+from tests.gpu_common import (MAX_ABS, REL_L2, TinyRig, compare_logits, router_gap)
+from tests.oracle_io import array_kv
+
+pytestmark = pytest.mark.gpu
+
+# Tighter internal bound than the contract: the hi/lo bf16 split keeps about
+# 16 mantissa bits of every matmul input and all accumulation is fp32, so the
+# tiny model agrees with the float64 oracle to ~1e-5.
+TIGHT = 2e-3
+
+
+@pytest.fixture(scope="module")
+def rig():
+    r = TinyRig(configs.TINY, [128], shuffled=False)
+    yield r
+    r.close()
+
+
+def test_one_step_logits(rig):
+    got = rig.step()
+    ref = rig.oracle_step()
+    err, rel = compare_logits(got, ref)
+    assert err <= MAX_ABS and rel <= REL_L2
+    assert err <= TIGHT, f"max_abs {err:.3e}"
+    assert np.argmax(got[0]) == np.argmax(ref[0])
+
+
+def test_intermediates_per_op(rig):
+    """Per-operation parity from the step's own buffers: residual entering
+    every layer, QKV, attention output, router logits and selection, expert
+    activations, weighted expert outputs, O-proj partials."""
+    rec = {}
+    rig.step()
+    rig.oracle_step(record=rec)
+    shape = rig.shape
+    L, B, d = shape["n_layers"], rig.B, shape["d_model"]
+    Hq, Hkv, hd, E, K, F = (shape[x] for x in ("n_q_heads", "n_kv_heads", "head_dim",
+                                               "n_experts", "top_k", "d_ff"))
+    X = rig.dec.debug(mk.MK_BUF_X).reshape(L + 1, B, d)
+    QKV = rig.dec.debug(mk.MK_BUF_QKV).reshape(L, B, -1)
+    AO = rig.dec.debug(mk.MK_BUF_ATTN_O).reshape(L, B, Hq, hd)
+    RL = rig.dec.debug(mk.MK_BUF_RLOGITS).reshape(L, B, E)
+    TK = rig.dec.debug(mk.MK_BUF_TOPK)
+    ids = TK[: L * B * K].reshape(L, B, K)
+    wts = TK[L * B * K:].view(np.float32).reshape(L, B, K)
+    OP = rig.dec.debug(mk.MK_BUF_OPART).reshape(L, Hkv, B, d)
+    MO = rig.dec.debug(mk.MK_BUF_MOE).reshape(L, K, B, d)
+    for l in range(L):
+        r = rec[(l, 0)]
+        assert np.allclose(X[l, 0], r["x_in"], atol=1e-4, rtol=1e-4)
+        assert np.allclose(QKV[l, 0], r["qkv"], atol=1e-4, rtol=1e-4)
+        assert np.allclose(AO[l, 0], r["o"], atol=1e-4, rtol=1e-4)
+        assert np.allclose(RL[l, 0], r["router_logits"], atol=1e-4, rtol=1e-4)
+        assert list(ids[l, 0]) == list(r["topk_idx"])
+        assert np.allclose(wts[l, 0], r["topk_w"], atol=1e-5)
+        assert np.allclose(OP[l, :, 0].sum(axis=0), r["attn_out"], atol=1e-4, rtol=1e-4)
+        assert np.allclose(MO[l, :, 0].sum(axis=0), r["moe_out"], atol=1e-4, rtol=1e-4)
+    assert np.allclose(X[L, 0], rec[(L - 1, 0)]["x_out"], atol=1e-4, rtol=1e-4)
+
+
+def test_unfused_equals_fused(rig):
+    a = rig.step()
+    b = rig.step(unfused=True)
+    assert np.array_equal(a, b)
+
+
+def test_deterministic(rig):
+    a = rig.step()
+    b = rig.step()
+    assert np.array_equal(a, b)
+
+
+def test_kv_append_matches_oracle_bits(rig):
+    rec = {}
+    rig.step()
+    rig.oracle_step(record=rec)
+    pos = rig.lens[0]
+    page = int(rig.table[0][pos // 64])
+    kd = rig.kd.view(torch.int16).cpu().numpy().view(np.uint16)
+    vd = rig.vd.view(torch.int16).cpu().numpy().view(np.uint16)
+    for l in range(rig.shape["n_layers"]):
+        for ours, ref in ((kd[l, page, :, pos % 64, :], rec[(l, 0)]["k_bits"]),
+                          (vd[l, page, :, pos % 64, :], rec[(l, 0)]["v_bits"])):
+            diff = np.abs(ours.astype(np.int32) - ref.astype(np.int32))
+            assert diff.max() <= 1            # at most one bf16 ulp (fp32 vs fp64 rounding)
+            assert (diff > 0).mean() < 0.02
+
+
+@pytest.mark.parametrize("lens,shuffled", [([5, 64, 200], True), ([0, 1, 63, 64, 65, 127, 128, 129], True)])
+def test_ragged_batch(lens, shuffled):
+    rig = TinyRig(configs.TINY, lens, seed=3, shuffled=shuffled)
+    try:
+        got = rig.step()
+        ref = rig.oracle_step()
+        err, rel = compare_logits(got, ref)
+        assert err <= TIGHT and rel <= REL_L2, (err, rel)
+        assert list(np.argmax(got, axis=1)) == list(np.argmax(ref, axis=1))
+    finally:
+        rig.close()
+
+
+def test_zipf_routing_batch8():
+    lens = [100, 200, 300, 400, 500, 600, 700, 800]
+    rig = TinyRig(configs.TINY, lens, seed=5, routing="zipf")
+    try:
+        got = rig.step()
+        rec = {}
+        ref = rig.oracle_step(record=rec)
+        err, rel = compare_logits(got, ref)
+        assert err <= TIGHT and rel <= REL_L2, (err, rel)
+        nslots = rig.dec.debug(mk.MK_BUF_NSLOTS)
+        for l in range(rig.shape["n_layers"]):
+            union = set()
+            for b in range(len(lens)):
+                union |= set(rec[(l, b)]["topk_idx"].tolist())
+            assert nslots[l] == len(union)
+    finally:
+        rig.close()
+
+
+def test_greedy_16_steps():
+    """16 greedy steps: identical tokens, logits within tolerance each step,
+    the GPU appending K/V into its own pool and the oracle into its copy."""
+    rig = TinyRig(configs.TINY, [128], shuffled=False)
+    try:
+        kv = array_kv(rig.k, rig.v)
+        import oracle as orc
+        from tests.oracle_io import array_weights, oracle_shape
+        ref_logits, fed = orc.greedy_decode(oracle_shape(rig.shape), array_weights(rig.W), kv,
+                                            rig.tokens, rig.lens, rig.table.numpy(), 16)
+        toks = list(rig.tokens)
+        lens = list(rig.lens)
+        for s in range(16):
+            got = rig.step(toks, lens)
+            assert toks == fed[s], f"step {s}: fed {toks} vs oracle {fed[s]}"
+            err, rel = compare_logits(got, ref_logits[s])
+            assert err <= TIGHT and rel <= REL_L2, (s, err, rel)
+            toks = [int(np.argmax(got[b])) for b in range(rig.B)]
+            lens = [x + 1 for x in lens]
+    finally:
+        rig.close()
+
+
+def test_schedule_outgrown_is_reported():
+    """A step at a length beyond the schedule's attention plan must latch
+    MK_ERR_STATE on the device (no hang, context still usable)."""
+    rig = TinyRig(configs.TINY, [100], shuffled=False, growth=256)
+    try:
+        rig.dec.build_schedule([100], rig.table.shape[1], plan_len=[100])
+        rig.dec.step(rig.i32(rig.tokens), rig.i32([300]), rig.table.to(rig.dev),
+                     rig.i32([300]), rig.logits)
+        rc, detail = rig.dec.check()
+        assert rc == mk.MK_ERR_STATE, (rc, detail)
+        # the context recovers: a valid step right after passes
+        rig.dec.build_schedule([100], rig.table.shape[1])
+        got = rig.step(lens=[100])
+        ref = rig.oracle_step(lens=[100])
+        assert compare_logits(got, ref)[0] <= TIGHT
+    finally:
+        rig.close()
