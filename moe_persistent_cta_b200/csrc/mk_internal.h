@@ -107,7 +107,7 @@ struct Params {
   int max_chunks, max_pages, n_pages, part_stride;
   float eps;
   // byte sizes of the activation formats
-  int actA_bytes;      // per level: B-fragment hi/lo of gamma*x + ss partials
+  int actA_bytes;      // per level: B-fragment fp32 of gamma*x + ss partials
   int actA_frag_bytes; // per level: the fragment part
   int ofrag_bytes;     // per (layer, group)
   int afrag_bytes;     // per (layer, slot)

@@ -21,8 +21,8 @@
 //                      release add on each of the task's counters.
 //   warps 3..10        compute: mma.sync bf16 tiles (weights as the 16-row A
 //                      operand read from the swizzled TMA tile with ldmatrix,
-//                      activations as the 8-column B operand split into bf16
-//                      hi + lo halves so the product keeps ~16 mantissa bits),
+//                      fp32 activations as the 8-column B operand split into
+//                      three bf16 terms, so the product keeps ~24 bits),
 //                      attention with an online softmax, and the epilogues.
 // Every wait is bounded by a globaltimer deadline; on expiry the CTA latches an
 // error in the status word, raises the abort flag and unwinds, waiting for its
@@ -147,16 +147,24 @@ __device__ __forceinline__ float bf16r(float x) {
 __device__ __forceinline__ float bf16_to_f(uint16_t u) {
   return __uint_as_float(((uint32_t)u) << 16);
 }
-// B-operand fragment entry for 16 consecutive k of one column: hi and lo
-// bf16 halves of the four values this lane of the quad owns.
+// B-operand fragment entry for 16 consecutive k of one column: the four
+// fp32 values the lane of the quad owns, in mma register order.
 __device__ __forceinline__ uint4 frag_entry(float v0, float v1, float v2, float v3) {
-  float h0 = bf16r(v0), h1 = bf16r(v1), h2 = bf16r(v2), h3 = bf16r(v3);
-  uint4 e;
-  e.x = pack_bf16(h0, h1);
-  e.y = pack_bf16(h2, h3);
-  e.z = pack_bf16(v0 - h0, v1 - h1);
-  e.w = pack_bf16(v2 - h2, v3 - h3);
-  return e;
+  return make_uint4(__float_as_uint(v0), __float_as_uint(v1), __float_as_uint(v2),
+                    __float_as_uint(v3));
+}
+// Split a pair of fp32 values into three bf16x2 terms hi + mid + lo that sum
+// to the pair within 2^-27 relative (each difference is exact in fp32).
+__device__ __forceinline__ void split3(float a, float b, uint32_t& h, uint32_t& m, uint32_t& l) {
+  __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(hh);
+  const float ra = a - hf.x, rb = b - hf.y;
+  __nv_bfloat162 mm = __floats2bfloat162_rn(ra, rb);
+  const float2 mf = __bfloat1622float2(mm);
+  __nv_bfloat162 ll = __floats2bfloat162_rn(ra - mf.x, rb - mf.y);
+  h = *reinterpret_cast<uint32_t*>(&hh);
+  m = *reinterpret_cast<uint32_t*>(&mm);
+  l = *reinterpret_cast<uint32_t*>(&ll);
 }
 
 // -------------------------------------------------------------- state -----
@@ -547,7 +555,7 @@ __device__ __forceinline__ float level_rstd(const Params& p, const uint8_t* actA
 }
 
 // Generic skinny GEMV tile: n_mat matrices x R rows x (KCH*64) columns
-// against the <=8 activation columns in `act` ([kstep][B][4][16 B] hi/lo
+// against the <=8 activation columns in `act` ([kstep][B][4][16 B] fp32
 // fragment layout).  Leaves the result in scratch res[m][row][n] (floats).
 __device__ void gemv_tile(CCtx& c, const int32_t* ent, const uint8_t* act, int colsel,
                           float* res) {
@@ -577,11 +585,15 @@ __device__ void gemv_tile(CCtx& c, const int32_t* ent, const uint8_t* act, int c
       const int chunk = 2 * i + achunk_hi;
       ldsm_x4(ubase + arow * 128 + ((chunk ^ (arow & 7)) << 4), a0, a1, a2, a3);
       const int ks = kc * 4 + i;
-      uint4 bf = make_uint4(0u, 0u, 0u, 0u);
+      float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (colsel >= 0)
-        bf = *reinterpret_cast<const uint4*>(act + (((size_t)ks * B + colsel) * 4 + q) * 16);
-      mma16816(acc, a0, a1, a2, a3, bf.x, bf.y);
-      mma16816(acc, a0, a1, a2, a3, bf.z, bf.w);
+        bv = *reinterpret_cast<const float4*>(act + (((size_t)ks * B + colsel) * 4 + q) * 16);
+      uint32_t h0, m0, l0, h1, m1, l1;
+      split3(bv.x, bv.y, h0, m0, l0);
+      split3(bv.z, bv.w, h1, m1, l1);
+      mma16816(acc, a0, a1, a2, a3, h0, h1);
+      mma16816(acc, a0, a1, a2, a3, m0, m1);
+      mma16816(acc, a0, a1, a2, a3, l0, l1);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.empty(slot));

@@ -67,7 +67,6 @@ def make_weights(shape: dict, seed: int = 0, device: str = "cpu", routing: str =
     hd, Hq, Hkv = shape["head_dim"], shape["n_q_heads"], shape["n_kv_heads"]
     E, F = shape["n_experts"], shape["d_ff"]
     gen = torch.Generator(device=device).manual_seed(seed)
-    rstd = router_std(shape, routing)
     W: Dict[str, object] = {}
     W["embed"] = _randn_bf16((V, d), gen, device, WEIGHT_STD)
     W["lm_head"] = _randn_bf16((V, d), gen, device, WEIGHT_STD)
@@ -79,15 +78,26 @@ def make_weights(shape: dict, seed: int = 0, device: str = "cpu", routing: str =
         W["attn_norm"].append(torch.ones(d, dtype=torch.bfloat16, device=device))
         W["w_qkv"].append(_randn_bf16(((Hq + 2 * Hkv) * hd, d), gen, device, WEIGHT_STD))
         W["w_o"].append(_randn_bf16((d, Hq * hd), gen, device, WEIGHT_STD))
-        W["w_router"].append(_randn_bf16((E, d), gen, device, rstd))
         W["w_gate"].append(_randn_bf16((E, F, d), gen, device, WEIGHT_STD))
         W["w_up"].append(_randn_bf16((E, F, d), gen, device, WEIGHT_STD))
         W["w_down"].append(_randn_bf16((E, d, F), gen, device, WEIGHT_STD))
-    if routing == "zipf":
-        W["router_bias"] = [b.to(device) for b in zipf_bias(shape, zipf_s, seed + 1000)]
-    else:
-        W["router_bias"] = None
+    W["w_router"], W["router_bias"] = make_router(shape, seed, device, routing, zipf_s)
     return W
+
+
+def make_router(shape: dict, seed: int = 0, device: str = "cpu", routing: str = "uniform",
+                zipf_s: float = 1.1):
+    """Router weights (their own seeded stream, so models that differ only in
+    routing share every other tensor) and the per-layer bias (None for
+    uniform routing)."""
+    gen = torch.Generator(device=device).manual_seed(seed + 500)
+    rstd = router_std(shape, routing)
+    w = [_randn_bf16((shape["n_experts"], shape["d_model"]), gen, device, rstd)
+         for _ in range(shape["n_layers"])]
+    bias = None
+    if routing == "zipf":
+        bias = [b.to(device) for b in zipf_bias(shape, zipf_s, seed + 1000)]
+    return w, bias
 
 
 def seq_lengths(spec, batch: int) -> List[int]:
