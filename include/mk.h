@@ -161,6 +161,11 @@ mk_status mk_decode_step_unfused(mk_ctx* ctx, const int32_t* tokens,
  * the device status.  Clears the latched status.                           */
 mk_status mk_check(mk_ctx* ctx, int32_t* device_status, int32_t* detail);
 
+/* Record per-task timestamps in every following fused step (enable != 0),
+ * readable with mk_debug_read(MK_BUF_TRACE).  Costs a few global stores per
+ * task.  Default off.                                                       */
+mk_status mk_set_trace(mk_ctx* ctx, int32_t enable);
+
 /* Per-wait deadline in milliseconds for device-side spins (default 2000). */
 mk_status mk_set_timeout_ms(mk_ctx* ctx, int32_t ms);
 
@@ -176,6 +181,13 @@ mk_status mk_set_timeout_ms(mk_ctx* ctx, int32_t ms);
  *   MK_BUF_EXPERT_A float [L][S][B][F]       SwiGLU activation per slot
  *   MK_BUF_MOE      float [L][k][B][d]       weighted expert outputs by rank
  *   MK_BUF_OPART    float [L][Hkv][B][d]     O-proj output per KV group
+ *   MK_BUF_TRACE    uint32 [n_tasks][9] per task of the last traced step (see
+ *                   mk_set_trace): globaltimer stamps (ns, low 32 bits) of
+ *                   producer resolved, producer issued last stage, loader
+ *                   deps met, loader activation issued, consumer picked up,
+ *                   consumer has activation, consumer math done, consumer
+ *                   epilogue done; then the CTA that ran it, plus one
+ *   MK_BUF_PLAN     int32 [n_tasks][32] descriptors of the schedule
  * `bytes` must equal the buffer's size for the current schedule.            */
 enum {
   MK_BUF_X = 0,
@@ -186,24 +198,27 @@ enum {
   MK_BUF_NSLOTS = 5,
   MK_BUF_EXPERT_A = 6,
   MK_BUF_MOE = 7,
-  MK_BUF_OPART = 8
+  MK_BUF_OPART = 8,
+  MK_BUF_TRACE = 9,
+  MK_BUF_PLAN = 10
 };
 mk_status mk_debug_read(mk_ctx* ctx, int which, void* host_dst, size_t bytes);
 size_t mk_debug_size(mk_ctx* ctx, int which);
 
-/* Host-only schedule planner (no GPU needed): the exact descriptor lists
- * mk_build_schedule would upload for `n_ctas` CTAs.
- *   meta (HOST int32[16]) receives {n_ctas, max_tasks, total_tasks,
- *   n_counters, n_slots, max_chunks, desc_words, n_phases, ...}.
- *   counts (HOST int32[n_ctas] or NULL) receives tasks per CTA.
- *   desc (HOST int32[n_ctas][max_tasks][desc_words] or NULL) receives the
- *   descriptors; pass NULL first to learn max_tasks from meta.
+/* Host-only schedule planner (no GPU needed): the task list mk_build_schedule
+ * would upload, sized for `n_ctas` CTAs (attention chunks are cut so the KV
+ * stream spreads over them).  The list is in topological priority order; at
+ * run time every CTA takes the next task with an atomic add.
+ *   meta (HOST int32[16]) receives {n_tasks, n_counters, n_slots, max_chunks,
+ *   desc_words, n_phases, qkv_rows_per_tile, pages_per_chunk, dispenser
+ *   counter, first phase dispenser counter, 0...}.
+ *   desc (HOST int32[n_tasks][desc_words] or NULL) receives the descriptors;
+ *   pass NULL first to learn n_tasks from meta.
  *   targets (HOST int32[n_counters] or NULL) receives each counter's
  *   per-step arrival count.                                                 */
 mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batch,
                            const int32_t* seq_lens, const int32_t* plan_len,
-                           int32_t* meta, int32_t* counts, int32_t* desc,
-                           int32_t* targets);
+                           int32_t* meta, int32_t* desc, int32_t* targets);
 
 const char* mk_strerror(mk_status s);
 

@@ -49,15 +49,16 @@ struct mk_ctx {
   int32_t* d_status = nullptr;
   uint32_t* d_counters = nullptr;
   int counters_cap = 0;
-  DevBuf desc, ntasks, phase_desc, phase_counts;
+  DevBuf desc, phase_desc;
   DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, route, expert_a, afrag,
-      moe_part;
+      moe_part, trace;
+  bool tracing = false;
   // schedule
   bool have_schedule = false;
   Plan plan;
   SmemLayout sl{};
   int B = 0, S = 0, max_chunks = 1, max_pages = 0;
-  std::vector<int> phase_tasks;  // tasks per phase (0: skip the launch)
+
   uint32_t epoch = 0;
   unsigned long long timeout_ns = 2000ull * 1000ull * 1000ull;
   cudaStream_t last_stream = nullptr;
@@ -161,9 +162,10 @@ void mk_destroy(mk_ctx* c) {
   cudaFree(c->d_inv_freq);
   cudaFree(c->d_status);
   cudaFree(c->d_counters);
-  for (DevBuf* b : {&c->desc, &c->ntasks, &c->phase_desc, &c->phase_counts, &c->x, &c->actA,
+  for (DevBuf* b : {&c->desc, &c->phase_desc, &c->x, &c->actA,
                     &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
-                    &c->rlogits, &c->route, &c->expert_a, &c->afrag, &c->moe_part})
+                    &c->rlogits, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
+                    &c->trace})
     release(*b);
   c->plan.release();
   delete c;
@@ -283,6 +285,12 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
   return MK_OK;
 }
 
+mk_status mk_set_trace(mk_ctx* c, int32_t enable) {
+  if (!c) return MK_ERR_INVALID;
+  c->tracing = enable != 0;
+  return MK_OK;
+}
+
 mk_status mk_set_timeout_ms(mk_ctx* c, int32_t ms) {
   if (!c || ms <= 0) return MK_ERR_INVALID;
   c->timeout_ns = (unsigned long long)ms * 1000000ull;
@@ -347,10 +355,8 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   ENSURE(expert_a, (size_t)L * S * B * s.F * 4);
   ENSURE(afrag, (size_t)L * S * afrag_bytes);
   ENSURE(moe_part, (size_t)L * s.k * B * d * 4);
-  ENSURE(desc, (size_t)plan.n_ctas * plan.max_tasks * mk::kDescWords * 4);
-  ENSURE(ntasks, (size_t)plan.n_ctas * 4);
-  ENSURE(phase_desc, (size_t)plan.n_phases * plan.n_ctas * plan.phase_max_tasks * mk::kDescWords * 4);
-  ENSURE(phase_counts, (size_t)plan.n_phases * plan.n_ctas * 4);
+  ENSURE(desc, (size_t)plan.n_tasks * mk::kDescWords * 4);
+  ENSURE(phase_desc, (size_t)plan.n_tasks * mk::kDescWords * 4);
 #undef ENSURE
   if (plan.n_counters > c->counters_cap) {
     cudaFree(c->d_counters);
@@ -363,21 +369,11 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   if (cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap) != cudaSuccess)
     return fail(MK_ERR_CUDA);
   if (cudaMemset(c->route.ptr, 0, c->route.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
-  if (cudaMemcpy(c->desc.ptr, plan.desc,
-                 (size_t)plan.n_ctas * plan.max_tasks * mk::kDescWords * 4,
+  if (cudaMemcpy(c->desc.ptr, plan.desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
                  cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(c->ntasks.ptr, plan.counts, (size_t)plan.n_ctas * 4, cudaMemcpyHostToDevice) !=
-          cudaSuccess ||
-      cudaMemcpy(c->phase_desc.ptr, plan.phase_desc,
-                 (size_t)plan.n_phases * plan.n_ctas * plan.phase_max_tasks * mk::kDescWords * 4,
-                 cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(c->phase_counts.ptr, plan.phase_counts, (size_t)plan.n_phases * plan.n_ctas * 4,
+      cudaMemcpy(c->phase_desc.ptr, plan.phase_desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
                  cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(MK_ERR_CUDA);
-  c->phase_tasks.assign(plan.n_phases, 0);
-  for (int ph = 0; ph < plan.n_phases; ++ph)
-    for (int cc = 0; cc < plan.n_ctas; ++cc)
-      c->phase_tasks[ph] += plan.phase_counts[(size_t)ph * plan.n_ctas + cc];
 
   Params& p = c->base;
   std::memset(&p, 0, sizeof(p));
@@ -458,18 +454,26 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
   p.timeout_ns = c->timeout_ns;
   p.epoch = c->epoch + 1;
   cudaError_t e = cudaSuccess;
+  p.n_ctas = c->plan.n_ctas;
   if (!unfused) {
+    if (c->tracing) {
+      const size_t tb = (size_t)c->plan.n_tasks * mk::kTraceWords * 4;
+      MK_TRY(ensure(c->trace, tb));
+      MK_CUDA(cudaMemsetAsync(c->trace.ptr, 0, tb, st));
+      p.trace = static_cast<uint32_t*>(c->trace.ptr);
+    }
     p.desc = static_cast<const int32_t*>(c->desc.ptr);
-    p.ntasks = static_cast<const int32_t*>(c->ntasks.ptr);
-    p.max_tasks = c->plan.max_tasks;
+    p.n_tasks = c->plan.n_tasks;
+    p.grab = c->plan.grab;
     e = mk::launch_interp(p, c->plan.n_ctas, st);
   } else {
-    const size_t stride = (size_t)c->plan.n_ctas * c->plan.phase_max_tasks * mk::kDescWords;
     for (int ph = 0; ph < c->plan.n_phases && e == cudaSuccess; ++ph) {
-      if (c->phase_tasks[ph] == 0) continue;
-      p.desc = static_cast<const int32_t*>(c->phase_desc.ptr) + stride * ph;
-      p.ntasks = static_cast<const int32_t*>(c->phase_counts.ptr) + (size_t)ph * c->plan.n_ctas;
-      p.max_tasks = c->plan.phase_max_tasks;
+      const int n = c->plan.phase_off[ph + 1] - c->plan.phase_off[ph];
+      if (n == 0) continue;
+      p.desc = static_cast<const int32_t*>(c->phase_desc.ptr) +
+               (size_t)c->plan.phase_off[ph] * mk::kDescWords;
+      p.n_tasks = n;
+      p.grab = c->plan.grab_phase0 + ph;
       e = mk::launch_interp(p, c->plan.n_ctas, st);
     }
   }
@@ -526,6 +530,8 @@ size_t mk_debug_size(mk_ctx* c, int which) {
     case MK_BUF_EXPERT_A: return L * S * B * s.F * 4;
     case MK_BUF_MOE: return L * s.k * B * s.d * 4;
     case MK_BUF_OPART: return L * s.Hkv * B * s.d * 4;
+    case MK_BUF_TRACE: return (size_t)c->plan.n_tasks * mk::kTraceWords * 4;
+    case MK_BUF_PLAN: return (size_t)c->plan.n_tasks * mk::kDescWords * 4;
   }
   return 0;
 }
@@ -549,6 +555,14 @@ mk_status mk_debug_read(mk_ctx* c, int which, void* dst, size_t bytes) {
     case MK_BUF_MOE: src = c->moe_part.ptr; break;
     case MK_BUF_OPART: src = c->o_part.ptr; break;
     default: break;
+  }
+  if (which == MK_BUF_TRACE) {
+    if (!c->trace.ptr) return MK_ERR_STATE;
+    src = c->trace.ptr;
+  }
+  if (which == MK_BUF_PLAN) {
+    std::memcpy(dst, c->plan.desc, sizeof(int32_t) * (size_t)c->plan.n_tasks * mk::kDescWords);
+    return MK_OK;
   }
   if (src) {
     MK_CUDA(cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost));

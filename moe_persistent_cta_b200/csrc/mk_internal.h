@@ -34,6 +34,21 @@ constexpr int kThreads = (kFirstConsumerWarp + kConsumerWarps) * 32;   // 352
 constexpr int kFifo = 16;            // task entries in flight per CTA
 constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words
 constexpr int kMapsPerLayer = 8;     // qkv, o, router, gate, up, down, kpool, vpool
+constexpr int kTraceWords = 9;       // per task: see TraceField
+
+// Per-task trace words: globaltimer stamps (low 32 bits, ns) and the CTA
+// that ran the task.
+enum TraceField : int {
+  T_P_RESOLVED = 0,   // producer wrote the task's entry
+  T_P_ISSUED = 1,     // producer issued the task's last stage
+  T_L_DEPS = 2,       // loader saw the task's counters satisfied
+  T_L_ACT = 3,        // loader issued the task's activation copy
+  T_C_READY = 4,      // consumers picked the task up
+  T_C_ACT = 5,        // consumers have the activation
+  T_C_MATH = 6,       // consumers finished the streamed stages
+  T_C_END = 7,        // consumers finished the epilogue
+  T_CTA = 8           // CTA index + 1
+};
 
 // ---------------------------------------------------------------- opcodes --
 enum Op : int32_t {
@@ -71,17 +86,16 @@ enum DescField : int {
   D_R = 21,         // GEMV: rows per tile (TMA box height)
   D_NMAT = 22,      // GEMV: matrices per tile (2 = gate+up)
   D_MAP0 = 23, D_MAP1 = 24,                     // tensor-map indices
-  D_BSLOT = 25,     // small-activation buffer (0/1)
-  D_SEQ = 26,       // position of this task in its CTA list
+  D_ACT = 25,       // activation: 0 none, 1 normalized input of level D_LAYER
+                    // (slot A, reused while the level repeats), 2 small (slot B)
   D_PPC = 27,       // attention: pages per chunk
   D_PHASE = 28,     // operation phase (for the unfused launcher)
   D_X0 = 29, D_X1 = 30, D_X2 = 31
 };
 
+enum ActKind : int32_t { ACT_NONE = 0, ACT_A = 1, ACT_B = 2 };
+
 enum Flags : int32_t {
-  F_LOAD_A = 1,      // loader fetches the normalized-input activation (slot A)
-  F_REL_A = 2,       // consumer releases slot A after this task
-  F_LOAD_B = 4,      // loader fetches this task's small activation (slot B[D_BSLOT])
   F_LAST_CHUNK = 8,  // attention chunk that owns the new token (and appends it)
   F_SINGLE = 16      // attention of (b, g) in one chunk: write the final output
 };
@@ -95,6 +109,7 @@ enum ResolvedField : int {
   R_P0 = 3,         // attention: first logical page of the chunk
   R_SEQLEN = 4,     // attention: cached tokens of the sequence
   R_PHYS_NEW = 5,   // attention: physical page receiving the new token
+  R_TASK = 6,       // index of the task in the step's list (-1: no more tasks)
   R_TOK = 8,        // [8] slot token ids
   R_RANK = 16,      // [8] rank of the expert in each token's top-k
   R_W = 24          // [8] routing weight (float bits)
@@ -112,10 +127,12 @@ struct Params {
   int ofrag_bytes;     // per (layer, group)
   int afrag_bytes;     // per (layer, slot)
   int route_words;     // per layer
-  // schedule
-  const int32_t* desc;     // [n_ctas][max_tasks][kDescWords]
-  const int32_t* ntasks;   // [n_ctas]
-  int max_tasks;
+  // schedule: one list in topological priority order; CTAs take the next
+  // task with an atomic add on counters[grab]
+  const int32_t* desc;     // [n_tasks][kDescWords]
+  int n_tasks;
+  int n_ctas;
+  int grab;                // counter index of the task dispenser
   uint32_t* counters;
   uint32_t epoch;
   // tensors
@@ -148,6 +165,7 @@ struct Params {
   uint8_t* afrag;    // [L][S][afrag_bytes]
   float* moe_part;   // [L][k][B][d]
   int32_t* status;   // [16]
+  uint32_t* trace;   // null, or [n_tasks][kTraceWords]
   unsigned long long timeout_ns;
   // shared-memory layout (byte offsets from the 1024-aligned base)
   int n_stages, nA, actA_stride;
@@ -181,18 +199,17 @@ struct Shape {
 };
 
 struct Plan {
-  int n_ctas = 0, B = 0, S = 0, max_chunks = 1, n_counters = 0, max_tasks = 0;
+  int n_ctas = 0, B = 0, S = 0, max_chunks = 1, n_counters = 0, n_tasks = 0;
   int n_phases = 0;
   int r_qkv = 16, r_router = 16;
-  size_t total_tasks = 0;
-  // flat storage: CTA c has counts[c] descriptors
-  int32_t* desc = nullptr;           // [n_ctas][max_tasks][kDescWords]
-  int32_t* counts = nullptr;         // [n_ctas]
-  int32_t* targets = nullptr;        // [n_counters]
-  // per-phase lists for the unfused launcher: [n_phases][n_ctas][max_tasks_phase][32]
+  int grab = 0;                      // dispenser counter of the fused list
+  int grab_phase0 = 0;               // dispenser counters of the phase lists
+  int32_t* desc = nullptr;           // [n_tasks][kDescWords], fused priority order
+  int32_t* targets = nullptr;        // [n_counters] arrivals per step
+  // unfused launcher: the same tasks grouped by phase, phase ph being
+  // phase_desc[phase_off[ph] .. phase_off[ph+1])
   int32_t* phase_desc = nullptr;
-  int32_t* phase_counts = nullptr;   // [n_phases][n_ctas]
-  int phase_max_tasks = 0;
+  int32_t* phase_off = nullptr;      // [n_phases + 1]
   int nc[kMaxBatch] = {0};           // attention chunks per sequence
   int ppc[kMaxBatch] = {0};          // pages per chunk per sequence
   void release();

@@ -70,11 +70,19 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
+// L2 policy for streamed tensors (weights, cached K/V): evict first, so the
+// once-per-step stream does not push code, activations and counters out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar,
+                                       uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar)
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
@@ -144,9 +152,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16r(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
 }
-__device__ __forceinline__ float bf16_to_f(uint16_t u) {
-  return __uint_as_float(((uint32_t)u) << 16);
-}
 // B-operand fragment entry for 16 consecutive k of one column: the four
 // fp32 values the lane of the quad owns, in mma register order.
 __device__ __forceinline__ uint4 frag_entry(float v0, float v1, float v2, float v3) {
@@ -168,29 +173,51 @@ __device__ __forceinline__ void split3(float a, float b, uint32_t& h, uint32_t& 
 }
 
 // -------------------------------------------------------------- state -----
+extern __shared__ uint8_t g_smem[];
+__shared__ int g_abort;   // this CTA's abort flag
+
+// View of the CTA's shared-memory carve-out, rebuilt from the launch
+// parameters inside each role function so that it lives in registers.
 struct Smem {
-  uint8_t* base;
   uint8_t* ring;
-  uint64_t* bars;
-  int32_t* fifo;
   uint8_t* scratch;
   uint8_t* actA;
   uint8_t* actB;
+  int32_t* fifo;
+  uint32_t bars;  // shared-window address of barrier 0
   int NS;
-  int* abort_flag;
-  // barrier indices
-  __device__ uint32_t full(int s) const { return saddr(bars + s); }
-  __device__ uint32_t empty(int s) const { return saddr(bars + NS + s); }
-  __device__ uint32_t ready(int e) const { return saddr(bars + 2 * NS + e); }
-  __device__ uint32_t done(int e) const { return saddr(bars + 2 * NS + kFifo + e); }
-  __device__ uint32_t fempty(int e) const { return saddr(bars + 2 * NS + 2 * kFifo + e); }
-  __device__ uint32_t afullA(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + i); }
-  __device__ uint32_t aemptyA(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 2 + i); }
-  __device__ uint32_t afullB(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 4 + i); }
-  __device__ uint32_t aemptyB(int i) const { return saddr(bars + 2 * NS + 3 * kFifo + 6 + i); }
+  __device__ uint32_t bar(int i) const { return bars + 8u * (uint32_t)i; }
+  __device__ uint32_t full(int s) const { return bar(s); }
+  __device__ uint32_t empty(int s) const { return bar(NS + s); }
+  __device__ uint32_t ready(int e) const { return bar(2 * NS + e); }
+  __device__ uint32_t done(int e) const { return bar(2 * NS + kFifo + e); }
+  __device__ uint32_t fempty(int e) const { return bar(2 * NS + 2 * kFifo + e); }
+  __device__ uint32_t posted(int e) const { return bar(2 * NS + 3 * kFifo + e); }
+  __device__ uint32_t afullA(int i) const { return bar(2 * NS + 4 * kFifo + i); }
+  __device__ uint32_t aemptyA(int i) const { return bar(2 * NS + 4 * kFifo + 2 + i); }
+  __device__ uint32_t afullB(int i) const { return bar(2 * NS + 4 * kFifo + 4 + i); }
+  __device__ uint32_t aemptyB(int i) const { return bar(2 * NS + 4 * kFifo + 6 + i); }
 };
 
-__device__ void raise_error(const Params& p, int code, int task, int op, int ctr, uint32_t obs,
+__device__ __forceinline__ Smem smem_view(const Params& p) {
+  Smem s;
+  const uint32_t raw = saddr(g_smem);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  uint8_t* base = g_smem + pad;
+  s.ring = base + p.off_ring;
+  s.scratch = base + p.off_scratch;
+  s.actA = base + p.off_actA;
+  s.actB = base + p.off_actB;
+  s.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
+  s.bars = raw + pad + (uint32_t)p.off_bars;
+  s.NS = p.n_stages;
+  return s;
+}
+
+__device__ __forceinline__ bool aborted() { return *(volatile int*)&g_abort != 0; }
+__device__ __forceinline__ void set_abort() { *(volatile int*)&g_abort = 1; }
+
+__device__ __noinline__ void raise_error(const Params& p, int code, int task, int op, int ctr, uint32_t obs,
                             uint32_t tgt, int aux) {
   if (atomicCAS(&p.status[ST_CODE], 0, code) == 0) {
     p.status[ST_CTA] = blockIdx.x;
@@ -205,13 +232,9 @@ __device__ void raise_error(const Params& p, int code, int task, int op, int ctr
   atomicExch(&p.status[ST_ABORT], 1);
 }
 
-__device__ __forceinline__ bool aborted(const Smem& sm) {
-  return *(volatile int*)sm.abort_flag != 0;
-}
-
 // Bounded spin on a global counter (one lane).
-__device__ bool wait_counter(const Params& p, const Smem& sm, int ctr, uint32_t target, int task,
-                             int op) {
+__device__ __noinline__ bool wait_counter(const Params& p, int ctr, uint32_t target, int task,
+                                          int op) {
   const uint32_t* c = p.counters + ctr;
   uint32_t v = ld_acquire(c);
   if (v >= target) return true;
@@ -220,69 +243,93 @@ __device__ bool wait_counter(const Params& p, const Smem& sm, int ctr, uint32_t 
     v = ld_acquire(c);
     if (v >= target) return true;
     if ((it & 7u) == 0) {
-      if (aborted(sm)) return false;
+      if (aborted()) return false;
       if (*(volatile int*)(p.status + ST_ABORT)) {
-        *(volatile int*)sm.abort_flag = 1;
+        set_abort();
         return false;
       }
       if (gtimer() - t0 > p.timeout_ns) {
         raise_error(p, MK_ERR_TIMEOUT, task, op, ctr, v, target, 0);
-        *(volatile int*)sm.abort_flag = 1;
+        set_abort();
         return false;
       }
     }
   }
 }
 
-// Bounded wait on a shared-memory mbarrier phase (every calling lane).
-__device__ bool wait_bar(const Params& p, const Smem& sm, uint32_t bar, uint32_t parity, int aux) {
-  if (mbar_test(bar, parity)) return true;
+// Bounded wait on a shared-memory mbarrier phase (every calling lane): the
+// common already-complete case inline, the spin out of line.
+__device__ __noinline__ bool wait_bar_slow(const Params& p, uint32_t bar, uint32_t parity,
+                                           int aux) {
   const uint64_t t0 = gtimer();
   for (;;) {
     for (int i = 0; i < 8; ++i)
       if (mbar_test(bar, parity)) return true;
-    if (aborted(sm)) return false;
+    if (aborted()) return false;
     if (gtimer() - t0 > p.timeout_ns) {
       raise_error(p, MK_ERR_TIMEOUT, -1, -1, -1, 0, 0, aux);
-      *(volatile int*)sm.abort_flag = 1;
+      set_abort();
       return false;
     }
   }
 }
+__device__ __forceinline__ bool wait_bar(const Params& p, uint32_t bar, uint32_t parity, int aux) {
+  if (mbar_test(bar, parity)) return true;
+  return wait_bar_slow(p, bar, parity, aux);
+}
 
 // Warp-uniform bounded wait: lane 0 waits, the outcome is broadcast.
-__device__ bool warp_wait(const Params& p, const Smem& sm, uint32_t bar, uint32_t parity,
-                          int aux) {
+__device__ __forceinline__ bool warp_wait(const Params& p, uint32_t bar, uint32_t parity,
+                                          int aux) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = wait_bar(p, sm, bar, parity, aux) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(p, bar, parity, aux) ? 1 : 0;
   ok = __shfl_sync(FULL, ok, 0);
   return ok != 0;
 }
 
 // Wait for a phase that is known to complete (copies in flight), bounded.
-__device__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
+__device__ __noinline__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
   const uint64_t t0 = gtimer();
   while (!mbar_test(bar, parity)) {
     if (gtimer() - t0 > p.timeout_ns) break;
   }
 }
 
+__device__ __forceinline__ void stamp(const Params& p, int task, int field) {
+  if (p.trace) p.trace[(size_t)task * kTraceWords + field] = (uint32_t)gtimer();
+}
+
+
 __device__ __forceinline__ const void* tmap(const Params& p, int idx) {
   return static_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
 }
 
 // ============================================================== producer ==
-__device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my, int ntasks) {
+// The producer takes the next task of the step's list from the dispenser
+// (an atomic add on a counter that advances by n_tasks + n_ctas per step),
+// posts it in the CTA's task FIFO, and streams its tiles.  A taken index past
+// the end posts a stop entry.
+__device__ __noinline__ void producer_loop(const Params& p) {
+  const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
   uint32_t stage_ctr = 0;
-  int fills[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) fills[i] = 0;
   const int NS = sm.NS;
-  for (int i = 0; i < ntasks; ++i) {
+  const uint32_t base = (p.epoch - 1u) * (uint32_t)(p.n_tasks + p.n_ctas);
+  const uint64_t pol = l2_evict_first();
+  for (int i = 0;; ++i) {
     const int e = i % kFifo;
-    if (!warp_wait(p, sm, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 100)) break;
-    const int32_t dw = my[(size_t)i * kDescWords + lane];
+    if (!warp_wait(p, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 100)) break;
+    int t = 0;
+    if (lane == 0) t = (int)(atomicAdd(p.counters + p.grab, 1u) - base);
+    t = __shfl_sync(FULL, t, 0);
+    int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    if (t < 0 || t >= p.n_tasks) {
+      ent[D_OP] = OP_NONE;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.posted(e));
+      break;
+    }
+    const int32_t dw = __ldg(p.desc + (size_t)t * kDescWords + lane);
     const int op = __shfl_sync(FULL, dw, D_OP);
     const int layer = __shfl_sync(FULL, dw, D_LAYER);
     int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
@@ -293,7 +340,7 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
       const int ctr = __shfl_sync(FULL, dw, D_PW);
       const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
       int ok = 1;
-      if (lane == 0) ok = wait_counter(p, sm, ctr, tgt, i, op) ? 1 : 0;
+      if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
       ok = __shfl_sync(FULL, ok, 0);
       if (!ok) break;
       __syncwarp();
@@ -304,8 +351,8 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
       ntok = __ldcg(rt + route_slot_ntok(B, K, S) + j);
       if (expert < 0 || expert >= p.E || ntok < 0 || ntok > B) {
         if (expert >= p.E || ntok < 0 || ntok > B) {
-          if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, expert, ntok, 1);
-          *(volatile int*)sm.abort_flag = 1;
+          if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, expert, ntok, 1);
+          set_abort();
           break;
         }
         expert = -1;
@@ -334,15 +381,15 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
       if (np < 0) np = 0;
       const bool last = (c == nc - 1);
       if (seqlen < 0 || (last && p0 + ppc < pages_now) || (seqlen / kPage) >= p.max_pages) {
-        if (lane == 0) raise_error(p, MK_ERR_STATE, i, op, -1, seqlen, pages_now, b);
-        *(volatile int*)sm.abort_flag = 1;
+        if (lane == 0) raise_error(p, MK_ERR_STATE, t, op, -1, seqlen, pages_now, b);
+        set_abort();
         fail = true;
       }
       if (!fail && last) {
         phys_new = __ldg(p.page_table + (size_t)b * p.max_pages + seqlen / kPage);
         if (phys_new < 0 || phys_new >= p.n_pages) {
-          if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, phys_new, p.n_pages, 2);
-          *(volatile int*)sm.abort_flag = 1;
+          if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, phys_new, p.n_pages, 2);
+          set_abort();
           fail = true;
         }
       }
@@ -356,11 +403,15 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
     if (lane == R_P0) rw = p0;
     if (lane == R_SEQLEN) rw = seqlen;
     if (lane == R_PHYS_NEW) rw = phys_new;
-    int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    if (lane == R_TASK) rw = t;
     ent[lane] = dw;
     ent[32 + lane] = rw;
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.ready(e));
+    if (lane == 0) {
+      stamp(p, t, T_P_RESOLVED);
+      if (p.trace) p.trace[(size_t)t * kTraceWords + T_CTA] = blockIdx.x + 1;
+      mbar_arrive(sm.posted(e));
+    }
 
     // ---- stream the task's tiles
     if (op == OP_ATTN) {
@@ -378,8 +429,8 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
           pg = (pi + lane < np) ? __ldg(pt + idx) : 0;
           int bad = (pi + lane < np) && (pg < 0 || pg >= p.n_pages);
           if (__any_sync(FULL, bad)) {
-            if (lane == 0) raise_error(p, MK_ERR_DEVICE, i, op, -1, 0, 0, 3);
-            *(volatile int*)sm.abort_flag = 1;
+            if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, 0, 0, 3);
+            set_abort();
             fail = true;
           }
         }
@@ -387,7 +438,7 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
         const int phys = __shfl_sync(FULL, pg, pi & 31);
         const uint32_t slot = stage_ctr % NS;
         const uint32_t ph = (stage_ctr / NS) & 1;
-        if (!warp_wait(p, sm, sm.empty(slot), ph ^ 1, 101)) {
+        if (!warp_wait(p, sm.empty(slot), ph ^ 1, 101)) {
           fail = true;
           break;
         }
@@ -398,9 +449,8 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
           const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
           const int y = (phys * p.Hkv + g) * kPage;
           const void* m = (s & 1) ? mv_ : mk_;
-          for (int xb = 0; xb < p.hd / 64; ++xb) tma_2d(dst + xb * 8192, m, xb * 64, y, fb);
+          for (int xb = 0; xb < p.hd / 64; ++xb) tma_2d(dst + xb * 8192, m, xb * 64, y, fb, pol);
         }
-        fills[slot] += 1;
         __syncwarp();
         ++stage_ctr;
       }
@@ -418,7 +468,7 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
       for (int s = 0; s < nstage; ++s) {
         const uint32_t slot = stage_ctr % NS;
         const uint32_t ph = (stage_ctr / NS) & 1;
-        if (!warp_wait(p, sm, sm.empty(slot), ph ^ 1, 102)) {
+        if (!warp_wait(p, sm.empty(slot), ph ^ 1, 102)) {
           fail = true;
           break;
         }
@@ -428,46 +478,63 @@ __device__ void producer_loop(const Params& p, const Smem& sm, const int32_t* my
           const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
           for (int kl = 0; kl < kcps; ++kl) {
             const int x = k0 + (s * kcps + kl) * 64;
-            tma_2d(dst + (kl * nm + 0) * MT * kUnitBytes, m0, x, row0, fb);
-            if (nm > 1) tma_2d(dst + (kl * nm + 1) * MT * kUnitBytes, m1, x, row0, fb);
+            tma_2d(dst + (kl * nm + 0) * MT * kUnitBytes, m0, x, row0, fb, pol);
+            if (nm > 1) tma_2d(dst + (kl * nm + 1) * MT * kUnitBytes, m1, x, row0, fb, pol);
           }
         }
-        fills[slot] += 1;
         __syncwarp();
         ++stage_ctr;
       }
       if (fail) break;
     }
+    if (lane == 0) stamp(p, t, T_P_ISSUED);
   }
-  // drain: every fill issued must land before the CTA may exit
-  for (int s = 0; s < NS && s < 16; ++s)
-    if (fills[s] > 0) drain_bar(p, sm.full(s), (uint32_t)((fills[s] - 1) & 1));
+  // drain: every fill issued must land before the CTA may exit (stage s was
+  // filled (stage_ctr - 1 - s) / NS + 1 times; wait for the last fill's phase)
+  for (int s = 0; s < NS; ++s)
+    if ((int)stage_ctr > s)
+      drain_bar(p, sm.full(s), (uint32_t)((((int)stage_ctr - 1 - s) / NS) & 1));
 }
 
 // ================================================================ loader ==
-__device__ void loader_loop(const Params& p, const Smem& sm, const int32_t* my, int ntasks) {
+// The loader follows the FIFO: it waits for the producer to post a task,
+// spins on the task's counters, and bulk-copies the task's activation into
+// shared memory: the normalized input of a level into slot A (reused while
+// consecutive A-tasks read the same level; two buffers when they fit), a
+// small activation into the next of the two B buffers.
+__device__ __noinline__ void loader_loop(const Params& p) {
+  const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
-  int nloadA[2] = {0, 0}, nloadB[2] = {0, 0};
-  for (int i = 0; i < ntasks; ++i) {
+  int curA = -1, nloadA = 0, nloadB = 0;
+  const int nA = p.nA;
+  for (int i = 0;; ++i) {
     const int e = i % kFifo;
-    if (!warp_wait(p, sm, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 200)) break;
-    const int32_t dw = my[(size_t)i * kDescWords + lane];
+    if (!warp_wait(p, sm.posted(e), (i / kFifo) & 1, 200)) break;
+    const int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    const int32_t dw = ent[lane];
     const int op = __shfl_sync(FULL, dw, D_OP);
+    if (op == OP_NONE) {
+      if (lane == 0) mbar_arrive(sm.ready(e));
+      break;
+    }
+    const int t = ent[32 + R_TASK];
     const int layer = __shfl_sync(FULL, dw, D_LAYER);
-    const int flags = __shfl_sync(FULL, dw, D_FLAGS);
+    const int act = __shfl_sync(FULL, dw, D_ACT);
     const int nwait = __shfl_sync(FULL, dw, D_NWAIT);
     int ok = 1;
     for (int w = 0; w < nwait && ok; ++w) {
       const int ctr = __shfl_sync(FULL, dw, D_W0 + 2 * w);
       const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_W0N + 2 * w);
-      if (lane == 0) ok = wait_counter(p, sm, ctr, tgt, i, op) ? 1 : 0;
+      if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
       ok = __shfl_sync(FULL, ok, 0);
     }
     if (!ok) break;
-    if (flags & F_LOAD_A) {
-      const int buf = __shfl_sync(FULL, dw, D_X0);
-      if (!warp_wait(p, sm, sm.aemptyA(buf), (uint32_t)((nloadA[buf] & 1) ^ 1), 201)) break;
-      nloadA[buf]++;
+    if (lane == 0) stamp(p, t, T_L_DEPS);
+    if (act == ACT_A && layer != curA) {
+      const int buf = nloadA % nA;
+      if (!warp_wait(p, sm.aemptyA(buf), (uint32_t)(((nloadA / nA) & 1) ^ 1), 201)) break;
+      ++nloadA;
+      curA = layer;
       if (lane == 0) {
         fence_proxy_async_global();
         const uint32_t fb = sm.afullA(buf);
@@ -477,16 +544,16 @@ __device__ void loader_loop(const Params& p, const Smem& sm, const int32_t* my, 
       }
       __syncwarp();
     }
-    if (flags & F_LOAD_B) {
-      const int buf = __shfl_sync(FULL, dw, D_BSLOT);
-      if (!warp_wait(p, sm, sm.aemptyB(buf), (uint32_t)((nloadB[buf] & 1) ^ 1), 202)) break;
-      nloadB[buf]++;
+    if (act == ACT_B) {
+      const int buf = nloadB & 1;
+      if (!warp_wait(p, sm.aemptyB(buf), (uint32_t)(((nloadB >> 1) & 1) ^ 1), 202)) break;
+      ++nloadB;
       if (lane == 0) {
         fence_proxy_async_global();
         const uint32_t fb = sm.afullB(buf);
         const uint32_t dst = saddr(sm.actB + (size_t)buf * p.actB_bytes);
-        const int a = __ldg(my + (size_t)i * kDescWords + D_A);
-        const int bb = __ldg(my + (size_t)i * kDescWords + D_B);
+        const int a = ent[D_A];
+        const int bb = ent[D_B];
         if (op == OP_ATTN) {
           const int b = a, g = bb, G = p.G, hd = p.hd;
           const float* row = p.qkv + ((size_t)layer * p.B + b) * p.qkvR;
@@ -510,24 +577,29 @@ __device__ void loader_loop(const Params& p, const Smem& sm, const int32_t* my, 
       }
       __syncwarp();
     }
-    if (lane == 0) mbar_arrive(sm.ready(e));
+    if (lane == 0) {
+      stamp(p, t, T_L_ACT);
+      mbar_arrive(sm.ready(e));
+    }
     __syncwarp();
   }
-  // drain activation copies in flight
-  for (int b = 0; b < 2; ++b) {
-    if (nloadA[b] > 0 && b < p.nA) drain_bar(p, sm.afullA(b), (uint32_t)((nloadA[b] - 1) & 1));
-    if (nloadB[b] > 0) drain_bar(p, sm.afullB(b), (uint32_t)((nloadB[b] - 1) & 1));
-  }
+  // drain activation copies in flight (the last load of each buffer)
+  for (int b = 0; b < nA; ++b)
+    if (nloadA > b) drain_bar(p, sm.afullA(b), (uint32_t)((((nloadA - 1 - b) / nA)) & 1));
+  for (int b = 0; b < 2; ++b)
+    if (nloadB > b) drain_bar(p, sm.afullB(b), (uint32_t)(((nloadB - 1 - b) / 2) & 1));
 }
 
 // ============================================================== signaler ==
-__device__ void signal_loop(const Params& p, const Smem& sm, int ntasks) {
+__device__ __noinline__ void signal_loop(const Params& p) {
+  const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
-  for (int i = 0; i < ntasks; ++i) {
+  for (int i = 0;; ++i) {
     const int e = i % kFifo;
-    if (!warp_wait(p, sm, sm.done(e), (i / kFifo) & 1, 300)) break;
+    if (!warp_wait(p, sm.done(e), (i / kFifo) & 1, 300)) break;
+    const int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    if (ent[D_OP] == OP_NONE) break;
     if (lane == 0) {
-      const int32_t* ent = sm.fifo + e * kFifoEntryWords;
       const int nsig = ent[D_NSIG];
       for (int s = 0; s < nsig; ++s) red_release_add(p.counters + ent[D_S0 + s], 1u);
       mbar_arrive(sm.fempty(e));
@@ -537,78 +609,93 @@ __device__ void signal_loop(const Params& p, const Smem& sm, int ntasks) {
 }
 
 // ============================================================= consumers ==
-struct CCtx {
-  const Params* p;
-  const Smem* sm;
-  int ct;     // consumer thread 0..255
-  int cw;     // consumer warp 0..7
-  int lane;
-  uint32_t stage_ctr;
-};
+// consumer thread / warp / lane indices
+#define MK_CONSUMER_IDS                                        \
+  const int ct = (int)threadIdx.x - kFirstConsumerWarp * 32;   \
+  const int cw = ct >> 5;                                      \
+  const int lane = (int)threadIdx.x & 31;                      \
+  (void)ct;                                                    \
+  (void)cw;                                                    \
+  (void)lane
 
-// rstd of each token from the level's sum-of-squares partials (slot A tail)
-__device__ __forceinline__ float level_rstd(const Params& p, const uint8_t* actA, int b) {
-  const float* ss = reinterpret_cast<const float*>(actA + p.actA_frag_bytes);
-  float acc = 0.f;
-  for (int r = 0; r < p.NR; ++r) acc += ss[r * p.B + b];
-  return 1.0f / sqrtf(acc / (float)p.d + p.eps);
+// rstd of each token from the level's sum-of-squares partials (slot A tail):
+// warp b reduces token b's partials into rstd_out[b].  Read after a barrier.
+__device__ __forceinline__ void level_rstd(const Params& p, const uint8_t* actA, float* rstd_out) {
+  MK_CONSUMER_IDS;
+  if (cw < p.B) {
+    const float* ss = reinterpret_cast<const float*>(actA + p.actA_frag_bytes);
+    float acc = 0.f;
+    for (int r = lane; r < p.NR; r += 32) acc += ss[r * p.B + cw];
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+    if (lane == 0) rstd_out[cw] = 1.0f / sqrtf(acc / (float)p.d + p.eps);
+  }
 }
 
 // Generic skinny GEMV tile: n_mat matrices x R rows x (KCH*64) columns
 // against the <=8 activation columns in `act` ([kstep][B][4][16 B] fp32
 // fragment layout).  Leaves the result in scratch res[m][row][n] (floats).
-__device__ void gemv_tile(CCtx& c, const int32_t* ent, const uint8_t* act, int colsel,
-                          float* res) {
-  const Params& p = *c.p;
-  const Smem& sm = *c.sm;
+__device__ __noinline__ uint32_t gemv_tile(const Params& p, const int32_t* ent, const uint8_t* act,
+                                           int colsel, float* res, uint32_t stage_ctr) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
   const int nstage = ent[32 + R_NSTAGE];
   const int nm = ent[D_NMAT], R = ent[D_R];
   const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
-  const int kl = c.cw / MTn;
-  const int lane = c.lane;
+  const int kl = cw / MTn;
   const int g8 = lane >> 2, q = lane & 3;
   const int B = p.B;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // three independent accumulators (hi, mid, lo terms) keep the mma chains
+  // short; all smem reads of a stage are issued before the stage is released
+  float ah[4] = {0.f, 0.f, 0.f, 0.f}, am[4] = {0.f, 0.f, 0.f, 0.f},
+        al[4] = {0.f, 0.f, 0.f, 0.f};
   // A-operand row/chunk of this lane inside a 16x64 unit (128B-swizzled)
   const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
   const int achunk_hi = lane >> 4;
+  const uint32_t aoff = arow * 128;
+  const uint8_t* bbase = act + ((size_t)(colsel < 0 ? 0 : colsel) * 4 + q) * 16;
+  const size_t bstride = (size_t)B * 64;   // bytes per k-step
   for (int s = 0; s < nstage; ++s) {
-    const uint32_t slot = c.stage_ctr % sm.NS;
-    const uint32_t ph = (c.stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm, sm.full(slot), ph, 400);
+    const uint32_t slot = stage_ctr % sm.NS;
+    const uint32_t ph = (stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm.full(slot), ph, 400);
     __syncwarp();
-    const uint32_t ubase = saddr(sm.ring + (size_t)slot * kStageBytes + c.cw * kUnitBytes);
+    const uint32_t ubase = saddr(sm.ring + (size_t)slot * kStageBytes + cw * kUnitBytes);
     const int kc = s * kcps + kl;
+    uint32_t a[4][4];
+    float4 bv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint32_t a0, a1, a2, a3;
       const int chunk = 2 * i + achunk_hi;
-      ldsm_x4(ubase + arow * 128 + ((chunk ^ (arow & 7)) << 4), a0, a1, a2, a3);
-      const int ks = kc * 4 + i;
-      float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (colsel >= 0)
-        bv = *reinterpret_cast<const float4*>(act + (((size_t)ks * B + colsel) * 4 + q) * 16);
-      uint32_t h0, m0, l0, h1, m1, l1;
-      split3(bv.x, bv.y, h0, m0, l0);
-      split3(bv.z, bv.w, h1, m1, l1);
-      mma16816(acc, a0, a1, a2, a3, h0, h1);
-      mma16816(acc, a0, a1, a2, a3, m0, m1);
-      mma16816(acc, a0, a1, a2, a3, l0, l1);
+      ldsm_x4(ubase + aoff + ((chunk ^ (arow & 7)) << 4), a[i][0], a[i][1], a[i][2], a[i][3]);
+      bv[i] = colsel >= 0 ? *reinterpret_cast<const float4*>(bbase + (size_t)(kc * 4 + i) * bstride)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.empty(slot));
-    ++c.stage_ctr;
+    ++stage_ctr;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t h0, m0, l0, h1, m1, l1;
+      split3(bv[i].x, bv[i].y, h0, m0, l0);
+      split3(bv[i].z, bv[i].w, h1, m1, l1);
+      mma16816(ah, a[i][0], a[i][1], a[i][2], a[i][3], h0, h1);
+      mma16816(am, a[i][0], a[i][1], a[i][2], a[i][3], m0, m1);
+      mma16816(al, a[i][0], a[i][1], a[i][2], a[i][3], l0, l1);
+    }
   }
+  float acc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = ah[j] + (am[j] + al[j]);
   // cross-warp reduction over the column chunks that shared a row tile
   float* part = reinterpret_cast<float*>(sm.scratch);  // [8][16][8]
-  float* pw = part + c.cw * 128;
+  float* pw = part + cw * 128;
   pw[g8 * 8 + 2 * q] = acc[0];
   pw[g8 * 8 + 2 * q + 1] = acc[1];
   pw[(g8 + 8) * 8 + 2 * q] = acc[2];
   pw[(g8 + 8) * 8 + 2 * q + 1] = acc[3];
   cbar();
   const int nout = nm * R * 8;
-  for (int idx = c.ct; idx < nout; idx += 256) {
+  for (int idx = ct; idx < nout; idx += 256) {
     const int n = idx & 7;
     const int row = (idx >> 3) % R;
     const int m = (idx >> 3) / R;
@@ -618,18 +705,21 @@ __device__ void gemv_tile(CCtx& c, const int32_t* ent, const uint8_t* act, int c
     res[idx] = v;  // res[(m*R + row)*8 + n]
   }
   cbar();
+  if (ct == 0) stamp(p, ent[32 + R_TASK], T_C_MATH);
+  return stage_ctr;
 }
 
 // Write the normalized attention output o[G][hd] (smem) of token b, group g:
 // fp32 copy and the O-proj B-operand fragments.
-__device__ void write_attn_out(CCtx& c, int layer, int b, int g, const float* o) {
-  const Params& p = *c.p;
+__device__ __noinline__ void write_attn_out(const Params& p, int layer, int b, int g,
+                                           const float* o) {
+  MK_CONSUMER_IDS;
   const int G = p.G, hd = p.hd, B = p.B;
   float* dst = p.attn_o + ((size_t)layer * B + b) * (size_t)p.Hq * hd + (size_t)g * G * hd;
-  for (int idx = c.ct; idx < G * hd; idx += 256) dst[idx] = o[idx];
+  for (int idx = ct; idx < G * hd; idx += 256) dst[idx] = o[idx];
   uint8_t* fr = p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes;
   const int nent = (G * hd / 16) * 4;
-  for (int t = c.ct; t < nent; t += 256) {
+  for (int t = ct; t < nent; t += 256) {
     const int ks = t >> 2, q = t & 3;
     const float* v = o + ks * 16 + 2 * q;
     *reinterpret_cast<uint4*>(fr + (((size_t)ks * B + b) * 4 + q) * 16) =
@@ -638,15 +728,16 @@ __device__ void write_attn_out(CCtx& c, int layer, int b, int g, const float* o)
 }
 
 template <int HD>
-__device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
-  const Params& p = *c.p;
-  const Smem& sm = *c.sm;
+__device__ __noinline__ uint32_t attn_task(const Params& p, const int32_t* ent, const uint8_t* act,
+                                           uint32_t stage_ctr) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
   const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], chunk = ent[D_C];
   const int flags = ent[D_FLAGS];
   const int np = ent[32 + R_NTOK], p0 = ent[32 + R_P0], seqlen = ent[32 + R_SEQLEN];
   const int phys_new = ent[32 + R_PHYS_NEW];
   const int G = p.G;
-  const int lane = c.lane, g8 = lane >> 2, q = lane & 3;
+  const int g8 = lane >> 2, q = lane & 3;
   constexpr int HALF = HD / 2;
   const float* q_raw = reinterpret_cast<const float*>(act);
   const float* k_raw = q_raw + G * HD;
@@ -657,7 +748,7 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
   float* kn = qs + G * HD;                                 // [HD]
   float* vn = kn + HD;                                     // [HD]
   const float qscale = 1.4426950408889634f / sqrtf((float)HD);
-  for (int idx = c.ct; idx < G * HD; idx += 256) {
+  for (int idx = ct; idx < G * HD; idx += 256) {
     const int h = idx / HD, i = idx % HD, i1 = i % HALF;
     const float co = csv[i1], si = csv[HALF + i1];
     const float x = q_raw[h * HD + i];
@@ -665,7 +756,7 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
     const float r = (i < HALF) ? (x * co - y * si) : (x * co + y * si);
     qs[idx] = r * qscale;
   }
-  for (int i = c.ct; i < HD; i += 256) {
+  for (int i = ct; i < HD; i += 256) {
     const int i1 = i % HALF;
     const float co = csv[i1], si = csv[HALF + i1];
     const float x = k_raw[i];
@@ -710,7 +801,7 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
 #pragma unroll
   for (int j = 0; j < HD / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   // the new token joins the softmax of the chunk that owns it (warp 0)
-  if ((flags & F_LAST_CHUNK) && c.cw == 0) {
+  if ((flags & F_LAST_CHUNK) && cw == 0) {
     float sn[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i = lane; i < HD; i += 32)
       for (int h = 0; h < G; ++h) sn[h] += qs[h * HD + i] * kn[i];
@@ -727,29 +818,35 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
       }
     }
   }
-  const int key8 = 8 * c.cw;
+  const int key8 = 8 * cw;
   const int krow = key8 + (lane & 7);
   for (int pi = 0; pi < np; ++pi) {
     // ---- K page: scores of this warp's 8 keys for the G heads
-    uint32_t slot = c.stage_ctr % sm.NS;
-    uint32_t ph = (c.stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm, sm.full(slot), ph, 401);
+    uint32_t slot = stage_ctr % sm.NS;
+    uint32_t ph = (stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm.full(slot), ph, 401);
     __syncwarp();
     uint32_t kb = saddr(sm.ring + (size_t)slot * kStageBytes);
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t kr[HD / 32][4];
 #pragma unroll
     for (int k2 = 0; k2 < HD / 32; ++k2) {
       const int hd0 = k2 * 32;
       const int box = hd0 / 64;
       const int chunk = ((hd0 % 64) >> 3) + (lane >> 3);
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4(kb + box * 8192 + krow * 128 + ((chunk ^ (krow & 7)) << 4), r0, r1, r2, r3);
-      mma16816(sc, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, r0, r1);
-      mma16816(sc, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, r2, r3);
+      ldsm_x4(kb + box * 8192 + krow * 128 + ((chunk ^ (krow & 7)) << 4), kr[k2][0], kr[k2][1],
+              kr[k2][2], kr[k2][3]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.empty(slot));
-    ++c.stage_ctr;
+    ++stage_ctr;
+#pragma unroll
+    for (int k2 = 0; k2 < HD / 32; ++k2) {
+      mma16816(sc, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, kr[k2][0], kr[k2][1]);
+      mma16816(sd, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, kr[k2][2], kr[k2][3]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sc[j] += sd[j];
     float s0 = sc[0] + __shfl_down_sync(FULL, sc[0], 4 * G);
     float s1 = sc[1] + __shfl_down_sync(FULL, sc[1], 4 * G);
     const int kidx = (p0 + pi) * kPage + key8 + 2 * q;
@@ -785,9 +882,9 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
       acc[j][1] *= my_alpha;
     }
     // ---- V page: acc += P V
-    slot = c.stage_ctr % sm.NS;
-    ph = (c.stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm, sm.full(slot), ph, 402);
+    slot = stage_ctr % sm.NS;
+    ph = (stage_ctr / sm.NS) & 1;
+    wait_bar(p, sm.full(slot), ph, 402);
     __syncwarp();
     const uint32_t vb = saddr(sm.ring + (size_t)slot * kStageBytes);
 #pragma unroll
@@ -804,10 +901,11 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.empty(slot));
-    ++c.stage_ctr;
+    ++stage_ctr;
   }
+  if (ct == 0) stamp(p, ent[32 + R_TASK], T_C_MATH);
   // ---- per-warp state -> shared memory: O = hi rows + lo rows
-  float* mw = mrg + c.cw * G * (HD + 4);
+  float* mw = mrg + cw * G * (HD + 4);
 #pragma unroll
   for (int j = 0; j < HD / 8; ++j) {
     const float o0 = acc[j][0] + __shfl_down_sync(FULL, acc[j][0], 4 * G);
@@ -827,7 +925,7 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
   const bool single = (flags & F_SINGLE) != 0;
   float* part = p.attn_part +
                 ((((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks + chunk) * p.part_stride;
-  for (int idx = c.ct; idx < G * HD; idx += 256) {
+  for (int idx = ct; idx < G * HD; idx += 256) {
     const int h = idx / HD, i = idx % HD;
     float M = -1e30f;
     for (int w = 0; w < 8; ++w) M = fmaxf(M, mrg[(w * G + h) * (HD + 4) + HD]);
@@ -850,101 +948,131 @@ __device__ void attn_task(CCtx& c, const int32_t* ent, const uint8_t* act) {
   }
   if (single) {
     cbar();
-    write_attn_out(c, layer, b, g, osm);
+    write_attn_out(p, layer, b, g, osm);
   }
+  return stage_ctr;
 }
 
-__device__ void combine_task(CCtx& c, const int32_t* ent) {
-  const Params& p = *c.p;
-  const Smem& sm = *c.sm;
+// Log-sum-exp merge of the chunk partials of (token b, KV group g).  Every
+// load is issued in parallel across the CTA (no per-chunk dependency chain).
+__device__ __noinline__ void combine_task(const Params& p, const int32_t* ent) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
   const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], nc = ent[D_D];
-  const int G = p.G, hd = p.hd;
+  const int G = p.G, hd = p.hd, PS = p.part_stride;
   const float* parts =
-      p.attn_part + (((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks * (size_t)p.part_stride;
-  float* wsm = reinterpret_cast<float*>(sm.scratch);  // [nc][G]
+      p.attn_part + (((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks * (size_t)PS;
+  float* msm = reinterpret_cast<float*>(sm.scratch);  // [nc][G] chunk maxima
+  float* lsm = msm + p.max_chunks * G;                // [nc][G] chunk sums
+  float* wsm = lsm + p.max_chunks * G;                // [nc][G] merge weights
   float* ML = wsm + p.max_chunks * G;                 // [2][G]
   float* osm = ML + 2 * G;                            // [G][hd]
-  if (c.ct < G) {
-    const int h = c.ct;
+  for (int t = ct; t < nc * G; t += 256) {
+    const float* pp = parts + (size_t)(t / G) * PS;
+    msm[t] = __ldcg(pp + t % G);
+    lsm[t] = __ldcg(pp + G + t % G);
+  }
+  cbar();
+  if (cw < G) {
+    const int h = cw;
     float M = -1e30f;
-    for (int ch = 0; ch < nc; ++ch) M = fmaxf(M, __ldcg(parts + (size_t)ch * p.part_stride + h));
+    for (int ch = lane; ch < nc; ch += 32) M = fmaxf(M, msm[ch * G + h]);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
     float Ls = 0.f;
-    for (int ch = 0; ch < nc; ++ch) {
-      const float* pp = parts + (size_t)ch * p.part_stride;
-      Ls += exp2f(__ldcg(pp + h) - M) * __ldcg(pp + G + h);
+    for (int ch = lane; ch < nc; ch += 32) Ls += exp2f(msm[ch * G + h] - M) * lsm[ch * G + h];
+    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(FULL, Ls, o);
+    if (lane == 0) {
+      ML[h] = M;
+      ML[G + h] = 1.0f / Ls;
     }
-    ML[h] = M;
-    ML[G + h] = 1.0f / Ls;
   }
   cbar();
-  for (int t = c.ct; t < nc * G; t += 256) {
-    const int ch = t / G, h = t % G;
-    wsm[t] = exp2f(__ldcg(parts + (size_t)ch * p.part_stride + h) - ML[h]) * ML[G + h];
-  }
+  for (int t = ct; t < nc * G; t += 256) wsm[t] = exp2f(msm[t] - ML[t % G]) * ML[G + t % G];
   cbar();
-  for (int idx = c.ct; idx < G * hd; idx += 256) {
+  for (int idx = ct; idx < G * hd; idx += 256) {
     const int h = idx / hd;
-    float o = 0.f;
-    for (int ch = 0; ch < nc; ++ch)
-      o += wsm[ch * G + h] * __ldcg(parts + (size_t)ch * p.part_stride + 2 * G + idx);
-    osm[idx] = o;
+    const float* pp = parts + 2 * G + idx;
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    int ch = 0;
+    for (; ch + 4 <= nc; ch += 4) {
+      const float v0 = __ldcg(pp + (size_t)ch * PS), v1 = __ldcg(pp + (size_t)(ch + 1) * PS);
+      const float v2 = __ldcg(pp + (size_t)(ch + 2) * PS), v3 = __ldcg(pp + (size_t)(ch + 3) * PS);
+      o0 += wsm[ch * G + h] * v0;
+      o1 += wsm[(ch + 1) * G + h] * v1;
+      o2 += wsm[(ch + 2) * G + h] * v2;
+      o3 += wsm[(ch + 3) * G + h] * v3;
+    }
+    for (; ch < nc; ++ch) o0 += wsm[ch * G + h] * __ldcg(pp + (size_t)ch * PS);
+    osm[idx] = (o0 + o1) + (o2 + o3);
   }
   cbar();
-  write_attn_out(c, layer, b, g, osm);
+  write_attn_out(p, layer, b, g, osm);
 }
 
-// fused residual add + RMSNorm statistics for one 64-row tile of level l
-__device__ void rn_task(CCtx& c, const int32_t* ent) {
-  const Params& p = *c.p;
-  const Smem& sm = *c.sm;
+// fused residual add + RMSNorm statistics for one 64-row tile of level l:
+// x_l = x_{l-1} + sum_g o_part[g] + sum_j moe_part[j] (fixed order), the
+// gamma-scaled fragments the next projections read, and the tile's sum of
+// squares (the norm's 1/rms is applied in the consumers' epilogues).
+__device__ __noinline__ void rn_task(const Params& p, const int32_t* ent) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
   const int l = ent[D_LAYER], r = ent[D_A];
   const int B = p.B, d = p.d;
   float* xs = reinterpret_cast<float*>(sm.scratch);  // [B][64] gamma * x
-  const int b = c.cw;
-  const int col = r * 64 + 2 * c.lane;
+  const int b = cw;
+  const int col = r * 64 + 2 * lane;
   if (b < B) {
-    float x0, x1;
+    float2 x;
     if (l == 0) {
       int tok = __ldg(p.tokens + b);
       if (tok < 0 || tok >= p.V) {
-        if (c.lane == 0) raise_error(p, MK_ERR_DEVICE, ent[D_SEQ], OP_RN, -1, tok, p.V, 4);
+        if (lane == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
         tok = 0;
       }
-      const uint16_t* er = p.embed + (size_t)tok * d + col;
-      x0 = bf16_to_f(__ldg(er));
-      x1 = bf16_to_f(__ldg(er + 1));
+      const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d + col));
+      x = make_float2(__uint_as_float(pr << 16), __uint_as_float(pr & 0xffff0000u));
     } else {
+      // all partial loads in flight at once, then a fixed-order sum
+      constexpr int kMaxParts = 1 + 16 + kMaxTopK;
+      const int nparts = 1 + p.Hkv + p.k;
       const size_t o = (size_t)b * d + col;
-      const float* xp = p.x + (size_t)(l - 1) * B * d;
-      x0 = __ldcg(xp + o);
-      x1 = __ldcg(xp + o + 1);
-      for (int g = 0; g < p.Hkv; ++g) {
-        const float* op = p.o_part + ((size_t)(l - 1) * p.Hkv + g) * B * d;
-        x0 += __ldcg(op + o);
-        x1 += __ldcg(op + o + 1);
+      float2 v[kMaxParts];
+#pragma unroll
+      for (int t = 0; t < kMaxParts; ++t) {
+        const float* src;
+        if (t == 0)
+          src = p.x + (size_t)(l - 1) * B * d;
+        else if (t <= p.Hkv)
+          src = p.o_part + ((size_t)(l - 1) * p.Hkv + (t - 1)) * B * d;
+        else
+          src = p.moe_part + ((size_t)(l - 1) * p.k + (t - 1 - p.Hkv)) * B * d;
+        v[t] = t < nparts ? __ldcg(reinterpret_cast<const float2*>(src + o))
+                          : make_float2(0.f, 0.f);
       }
-      for (int j = 0; j < p.k; ++j) {
-        const float* mp = p.moe_part + ((size_t)(l - 1) * p.k + j) * B * d;
-        x0 += __ldcg(mp + o);
-        x1 += __ldcg(mp + o + 1);
+      x = v[0];
+#pragma unroll
+      for (int t = 1; t < kMaxParts; ++t) {
+        if (t < nparts) {
+          x.x += v[t].x;
+          x.y += v[t].y;
+        }
       }
     }
-    float* xo = p.x + ((size_t)l * B + b) * d + col;
-    xo[0] = x0;
-    xo[1] = x1;
+    *reinterpret_cast<float2*>(p.x + ((size_t)l * B + b) * d + col) = x;
     const uint16_t* gam = (l < p.L) ? p.attn_norm[l] : p.final_norm;
-    xs[b * 64 + 2 * c.lane] = x0 * bf16_to_f(__ldg(gam + col));
-    xs[b * 64 + 2 * c.lane + 1] = x1 * bf16_to_f(__ldg(gam + col + 1));
-    float ss = x0 * x0 + x1 * x1;
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-    if (c.lane == 0) {
+    const uint32_t gp = __ldg(reinterpret_cast<const uint32_t*>(gam + col));
+    xs[b * 64 + 2 * lane] = x.x * __uint_as_float(gp << 16);
+    xs[b * 64 + 2 * lane + 1] = x.y * __uint_as_float(gp & 0xffff0000u);
+    float ss = x.x * x.x + x.y * x.y;
+    for (int o2 = 16; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(FULL, ss, o2);
+    if (lane == 0) {
       float* ssd = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_frag_bytes);
       ssd[r * B + b] = ss;
     }
   }
   cbar();
   uint8_t* fr = p.actA + (size_t)l * p.actA_bytes;
-  for (int t = c.ct; t < 16 * B; t += 256) {
+  for (int t = ct; t < 16 * B; t += 256) {
     const int ksl = t / (4 * B), n = (t >> 2) % B, q = t & 3;
     const float* v = xs + n * 64 + ksl * 16 + 2 * q;
     *reinterpret_cast<uint4*>(fr + (((size_t)(4 * r + ksl) * B + n) * 4 + q) * 16) =
@@ -952,11 +1080,11 @@ __device__ void rn_task(CCtx& c, const int32_t* ent) {
   }
   if (l == 0 && r == 0) {
     const int half = p.hd / 2;
-    for (int t = c.ct; t < B * half; t += 256) {
+    for (int t = ct; t < B * half; t += 256) {
       const int bb = t / half, i = t % half;
       const int pos = __ldg(p.positions + bb);
       const int sl = __ldg(p.seq_lens + bb);
-      if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, ent[D_SEQ], OP_RN, -1, pos, sl, 5);
+      if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, pos, sl, 5);
       double sv, cv;
       sincos((double)pos * p.inv_freq[i], &sv, &cv);
       p.cs[(size_t)bb * p.hd + i] = (float)cv;
@@ -966,9 +1094,9 @@ __device__ void rn_task(CCtx& c, const int32_t* ent) {
 }
 
 // top-k (logit desc, index asc) + softmax over the selected + slot compaction
-__device__ void topk_task(CCtx& c, const int32_t* ent) {
-  const Params& p = *c.p;
-  const Smem& sm = *c.sm;
+__device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
   const int l = ent[D_LAYER];
   const int B = p.B, E = p.E, K = p.k, S = p.S;
   int32_t* rt = p.route + (size_t)l * p.route_words;
@@ -976,44 +1104,44 @@ __device__ void topk_task(CCtx& c, const int32_t* ent) {
   float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [B][8]
   int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8); // [E]
   uint32_t* used = reinterpret_cast<uint32_t*>(slot_of + 256); // [8]
-  if (c.ct < 8) used[c.ct] = 0u;
+  if (ct < 8) used[ct] = 0u;
   cbar();
-  const int b = c.cw;
+  const int b = cw;
   if (b < B) {
     const float* lg = p.rlogits + ((size_t)l * B + b) * E;
-    float v[8];
+    // order-preserving unsigned keys of the logits; 0 marks taken / absent
+    uint32_t key[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      const int e = c.lane + 32 * t;
-      v[t] = (e < E) ? __ldcg(lg + e) : -INFINITY;
+      const int e = lane + 32 * t;
+      uint32_t k = 0u;
+      if (e < E) {
+        const uint32_t u = __float_as_uint(__ldcg(lg + e));
+        k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      }
+      key[t] = k;
     }
     float selv[8];
     for (int j = 0; j < K; ++j) {
-      float bv = -INFINITY;
+      uint32_t bk = 0u;
       int bi = 0x7fffffff;
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const int e = c.lane + 32 * t;
-        if (e < E && (v[t] > bv || (v[t] == bv && e < bi))) {
-          bv = v[t];
-          bi = e;
+        if (key[t] > bk) {   // ascending e within a lane: first max has the smallest e
+          bk = key[t];
+          bi = lane + 32 * t;
         }
       }
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(FULL, bv, o);
-        const int oi = __shfl_xor_sync(FULL, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      selv[j] = bv;
-      if (c.lane == 0) sel[b * 8 + j] = bi;
+      const uint32_t mk = __reduce_max_sync(FULL, bk);
+      const int wi = __reduce_min_sync(FULL, bk == mk ? bi : 0x7fffffff);
 #pragma unroll
       for (int t = 0; t < 8; ++t)
-        if (c.lane + 32 * t == bi) v[t] = -INFINITY;
+        if (lane + 32 * t == wi) key[t] = 0u;
+      const uint32_t u = (mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk;
+      selv[j] = __uint_as_float(u);
+      if (lane == 0) sel[b * 8 + j] = wi;
     }
-    if (c.lane == 0) {
+    if (lane == 0) {
       float ws[8], sum = 0.f;
       for (int j = 0; j < K; ++j) {
         ws[j] = expf(selv[j] - selv[0]);
@@ -1030,7 +1158,7 @@ __device__ void topk_task(CCtx& c, const int32_t* ent) {
   }
   cbar();
   // slot of each used expert = number of used experts below it
-  for (int e = c.ct; e < E; e += 256) {
+  for (int e = ct; e < E; e += 256) {
     int cnt = 0;
     for (int w = 0; w < (e >> 5); ++w) cnt += __popc(used[w]);
     cnt += __popc(used[e >> 5] & ((1u << (e & 31)) - 1u));
@@ -1039,16 +1167,16 @@ __device__ void topk_task(CCtx& c, const int32_t* ent) {
   cbar();
   int n_used = 0;
   for (int w = 0; w < 8; ++w) n_used += __popc(used[w]);
-  for (int s = c.ct; s < S; s += 256) {
+  for (int s = ct; s < S; s += 256) {
     if (s >= n_used) {
       rt[route_slot_expert(B, K) + s] = -1;
       rt[route_slot_ntok(B, K, S) + s] = 0;
     }
   }
-  if (c.ct == 0) rt[0] = n_used;
+  if (ct == 0) rt[0] = n_used;
   // one thread per (token, rank): its position in the slot's token list
-  if (c.ct < B * K) {
-    const int bb = c.ct / K, j = c.ct % K;
+  if (ct < B * K) {
+    const int bb = ct / K, j = ct % K;
     const int e = sel[bb * 8 + j];
     const int s = slot_of[e];
     int pos = 0;
@@ -1067,61 +1195,71 @@ __device__ void topk_task(CCtx& c, const int32_t* ent) {
   }
 }
 
-__device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
-  CCtx c;
-  c.p = &p;
-  c.sm = &sm;
-  c.ct = threadIdx.x - kFirstConsumerWarp * 32;
-  c.cw = c.ct >> 5;
-  c.lane = threadIdx.x & 31;
-  c.stage_ctr = 0;
-  int nA[2] = {0, 0}, nB[2] = {0, 0};
+__device__ __noinline__ void consumer_loop(const Params& p) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
+  uint32_t stage_ctr = 0;
+  int curA = -1, nloadA = 0, nloadB = 0, bufA = 0;
+  const int nA = p.nA;
   float* res = reinterpret_cast<float*>(sm.scratch) + 8 * 128;  // after the partials
-  for (int i = 0; i < ntasks; ++i) {
+  float* rstd = res + 1024;                                       // [8] per-token 1/rms
+  for (int i = 0;; ++i) {
     const int e = i % kFifo;
-    const bool ok = wait_bar(p, sm, sm.ready(e), (i / kFifo) & 1, 500);
-    if (cbar_or(!ok || aborted(sm))) break;
+    const bool ok = wait_bar(p, sm.ready(e), (i / kFifo) & 1, 500);
+    if (cbar_or(!ok || aborted())) break;
     const int32_t* ent = sm.fifo + e * kFifoEntryWords;
     const int op = ent[D_OP];
-    const int flags = ent[D_FLAGS];
-    const int bufA = ent[D_X0], bufB = ent[D_BSLOT];
-    if (flags & F_LOAD_A) {
-      wait_bar(p, sm, sm.afullA(bufA), (uint32_t)(nA[bufA] & 1), 501);
-      nA[bufA]++;
+    if (op == OP_NONE) {
+      if (ct == 0) mbar_arrive(sm.done(e));
+      break;
     }
-    if (flags & F_LOAD_B) {
-      wait_bar(p, sm, sm.afullB(bufB), (uint32_t)(nB[bufB] & 1), 502);
-      nB[bufB]++;
+    const int t = ent[32 + R_TASK];
+    if (ct == 0) stamp(p, t, T_C_READY);
+    const int act = ent[D_ACT];
+    if (act == ACT_A && ent[D_LAYER] != curA) {
+      // a new level: the previous level's buffer is free (its tasks are done)
+      if (curA >= 0 && ct == 0) mbar_arrive(sm.aemptyA(bufA));
+      bufA = nloadA % nA;
+      wait_bar(p, sm.afullA(bufA), (uint32_t)((nloadA / nA) & 1), 501);
+      ++nloadA;
+      curA = ent[D_LAYER];
     }
+    const int bufB = nloadB & 1;
+    if (act == ACT_B) {
+      wait_bar(p, sm.afullB(bufB), (uint32_t)((nloadB >> 1) & 1), 502);
+      ++nloadB;
+    }
+    if (ct == 0) stamp(p, t, T_C_ACT);
     const uint8_t* actA = sm.actA + (size_t)bufA * p.actA_stride;
     const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
     const int layer = ent[D_LAYER];
-    const int n = c.lane >> 2;
+    const int n = lane >> 2;
     switch (op) {
       case OP_RN:
-        rn_task(c, ent);
+        rn_task(p, ent);
         break;
       case OP_TOPK:
-        topk_task(c, ent);
+        topk_task(p, ent);
         break;
       case OP_COMBINE:
-        combine_task(c, ent);
+        combine_task(p, ent);
         break;
       case OP_ATTN:
         if (p.hd == 128)
-          attn_task<128>(c, ent, actB);
+          stage_ctr = attn_task<128>(p, ent, actB, stage_ctr);
         else
-          attn_task<64>(c, ent, actB);
+          stage_ctr = attn_task<64>(p, ent, actB, stage_ctr);
         break;
       case OP_QKV:
       case OP_ROUTER:
       case OP_LMHEAD: {
-        gemv_tile(c, ent, actA, n < p.B ? n : -1, res);
+        level_rstd(p, actA, rstd);
+        stage_ctr = gemv_tile(p, ent, actA, n < p.B ? n : -1, res, stage_ctr);
         const int R = ent[D_R], row0 = ent[D_ROW0];
-        for (int idx = c.ct; idx < R * 8; idx += 256) {
+        for (int idx = ct; idx < R * 8; idx += 256) {
           const int nn = idx / R, r = idx % R;  // r fastest: coalesced rows
           if (nn >= p.B) continue;
-          const float v = res[r * 8 + nn] * level_rstd(p, actA, nn);
+          const float v = res[r * 8 + nn] * rstd[nn];
           const int row = row0 + r;
           if (op == OP_QKV) {
             p.qkv[((size_t)layer * p.B + nn) * p.qkvR + row] = v;
@@ -1137,9 +1275,9 @@ __device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
         break;
       }
       case OP_OPROJ: {
-        gemv_tile(c, ent, actB, n < p.B ? n : -1, res);
+        stage_ctr = gemv_tile(p, ent, actB, n < p.B ? n : -1, res, stage_ctr);
         const int g = ent[D_B], row0 = ent[D_ROW0];
-        for (int idx = c.ct; idx < 64 * 8; idx += 256) {
+        for (int idx = ct; idx < 64 * 8; idx += 256) {
           const int nn = idx / 64, r = idx % 64;
           if (nn >= p.B) continue;
           p.o_part[(((size_t)layer * p.Hkv + g) * p.B + nn) * p.d + row0 + r] = res[r * 8 + nn];
@@ -1150,14 +1288,15 @@ __device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
         const int ntok = ent[32 + R_NTOK];
         if (ent[32 + R_EXPERT] < 0) break;
         const int col = n < ntok ? ent[32 + R_TOK + n] : -1;
-        gemv_tile(c, ent, actA, col, res);
+        level_rstd(p, actA, rstd);
+        stage_ctr = gemv_tile(p, ent, actA, col, res, stage_ctr);
         const int R = ent[D_R], f = ent[D_B], j = ent[D_A];
         float* asm_ = res + 2 * R * 8;  // [R][8] activations
-        for (int idx = c.ct; idx < R * 8; idx += 256) {
+        for (int idx = ct; idx < R * 8; idx += 256) {
           const int nn = idx / R, r = idx % R;
           float a = 0.f;
           if (nn < ntok) {
-            const float rs = level_rstd(p, actA, ent[32 + R_TOK + nn]);
+            const float rs = rstd[ent[32 + R_TOK + nn]];
             const float gt = res[r * 8 + nn] * rs;
             const float ut = res[(R + r) * 8 + nn] * rs;
             a = gt / (1.0f + expf(-gt)) * ut;
@@ -1168,7 +1307,7 @@ __device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
         cbar();
         uint8_t* fr = p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes;
         const int nent = (R / 16) * ntok * 4;
-        for (int t = c.ct; t < nent; t += 256) {
+        for (int t = ct; t < nent; t += 256) {
           const int ksl = t / (4 * ntok), nn = (t >> 2) % ntok, q = t & 3;
           const int r0 = ksl * 16 + 2 * q;
           const uint4 fe = frag_entry(asm_[r0 * 8 + nn], asm_[(r0 + 1) * 8 + nn],
@@ -1181,9 +1320,9 @@ __device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
       case OP_DOWN: {
         const int ntok = ent[32 + R_NTOK];
         if (ent[32 + R_EXPERT] < 0) break;
-        gemv_tile(c, ent, actB, n < ntok ? n : -1, res);
+        stage_ctr = gemv_tile(p, ent, actB, n < ntok ? n : -1, res, stage_ctr);
         const int row0 = ent[D_ROW0];
-        for (int idx = c.ct; idx < 64 * 8; idx += 256) {
+        for (int idx = ct; idx < 64 * 8; idx += 256) {
           const int nn = idx / 64, r = idx % 64;
           if (nn >= ntok) continue;
           const int tok = ent[32 + R_TOK + nn];
@@ -1198,42 +1337,27 @@ __device__ void consumer_loop(const Params& p, const Smem& sm, int ntasks) {
         break;
     }
     cbar();
-    if (c.ct == 0) {
-      if (flags & F_REL_A) mbar_arrive(sm.aemptyA(bufA));
-      if (flags & F_LOAD_B) mbar_arrive(sm.aemptyB(bufB));
+    if (ct == 0) {
+      stamp(p, t, T_C_END);
+      if (act == ACT_B) mbar_arrive(sm.aemptyB(bufB));
       mbar_arrive(sm.done(e));
     }
-    if (cbar_or(aborted(sm))) break;
+    if (cbar_or(aborted())) break;
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ int s_abort;
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Smem sm;
-  sm.base = base;
-  sm.ring = base + p.off_ring;
-  sm.bars = reinterpret_cast<uint64_t*>(base + p.off_bars);
-  sm.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
-  sm.scratch = base + p.off_scratch;
-  sm.actA = base + p.off_actA;
-  sm.actB = base + p.off_actB;
-  sm.NS = p.n_stages;
-  sm.abort_flag = &s_abort;
   const int warp = threadIdx.x >> 5;
-  const int cta = blockIdx.x;
-  const int ntasks = p.ntasks[cta];
-  const int32_t* my = p.desc + (size_t)cta * p.max_tasks * kDescWords;
   if (threadIdx.x == 0) {
-    s_abort = 0;
+    const Smem sm = smem_view(p);
+    g_abort = 0;
     for (int s = 0; s < sm.NS; ++s) {
       mbar_init(sm.full(s), 1);
       mbar_init(sm.empty(s), kConsumerWarps);
     }
     for (int e = 0; e < kFifo; ++e) {
-      mbar_init(sm.ready(e), 2);
+      mbar_init(sm.posted(e), 1);
+      mbar_init(sm.ready(e), 1);
       mbar_init(sm.done(e), 1);
       mbar_init(sm.fempty(e), 1);
     }
@@ -1248,13 +1372,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
   }
   __syncthreads();
   if (warp == kProducerWarp) {
-    producer_loop(p, sm, my, ntasks);
+    producer_loop(p);
   } else if (warp == kLoaderWarp) {
-    loader_loop(p, sm, my, ntasks);
+    loader_loop(p);
   } else if (warp == kSignalWarp) {
-    signal_loop(p, sm, ntasks);
+    signal_loop(p);
   } else {
-    consumer_loop(p, sm, ntasks);
+    consumer_loop(p);
   }
   __syncthreads();
 }
@@ -1262,7 +1386,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
 }  // namespace
 
 // Launch one step (or one phase) of the interpreter: cooperative, so that all
-// CTAs are guaranteed co-resident (the counter waits rely on it).
+// CTAs are guaranteed co-resident (the counter waits and the dispenser rely
+// on it).
 cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream) {
   static int configured_bytes = -1;
   if (configured_bytes != p.smem_bytes) {

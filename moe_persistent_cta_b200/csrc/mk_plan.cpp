@@ -1,15 +1,14 @@
-// mk_plan.cpp -- host schedule builder: decode step -> per-CTA task lists.
+// mk_plan.cpp -- host schedule builder: decode step -> one task list.
 //
 // Every operation of the step is cut into tiles, one task per tile, emitted in
-// one global topological order (per layer: residual/norm tiles, QKV and router
-// tiles, top-k, attention chunks, combines, O-proj, expert gate/up, expert
-// down; then the final norm and the LM head).  Each task is appended to the
-// list of the CTA that a small list-scheduling simulation says finishes it
-// first, so any free SM picks up any ready tile and no work is rounded up to
-// whole waves (agenticcommons.xyz, "Cohere North Mini Code megakernel serving
-// engine", section "Three sources of speedup", item 1).  Because every list is
-// a subsequence of one topological order and all CTAs are co-resident, every
-// wait is on work that is earlier in that order, so the step cannot deadlock.
+// one topological order that is also a priority order.  At run time every CTA
+// takes the next task of that list with an atomic add (any free SM picks up
+// the next tile, so no work is rounded up to whole waves: agenticcommons.xyz,
+// "Cohere North Mini Code megakernel serving engine", section "Three sources
+// of speedup", item 1).  A task only ever waits on tasks that are earlier in
+// the list; those were taken earlier by CTAs that are running (all CTAs are
+// co-resident) and that finish their tasks in order, so the step cannot
+// deadlock.
 //
 // Dependencies are counters, one per producer group, with per-step arrival
 // counts; a task waits until counter >= epoch * arrivals (section "How the
@@ -17,6 +16,12 @@
 // O-proj of one KV group waits only for that group's attention, and the down
 // projection of one expert only for that expert's gate/up tiles (section
 // "Three sources of speedup", item 2).
+//
+// Priority order inside a layer: the norm tiles; the router, QKV and top-k
+// (whose weights stream before the norm is known); attention chunks (their
+// cached K/V stream before the new query exists); expert gate/up (the MoE
+// branch is the longer one); then the attention tail (combine, O-proj) and
+// the expert down projections.
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
@@ -30,11 +35,10 @@ namespace mk {
 
 void Plan::release() {
   std::free(desc);
-  std::free(counts);
   std::free(targets);
   std::free(phase_desc);
-  std::free(phase_counts);
-  desc = counts = targets = phase_desc = phase_counts = nullptr;
+  std::free(phase_off);
+  desc = targets = phase_desc = phase_off = nullptr;
 }
 
 static int gcd_int(int a, int b) {
@@ -61,6 +65,7 @@ int validate_shape(const Shape& s) {
   if (s.L < 1 || s.d < 128 || s.d % 64 != 0 || s.d > 16384) return MK_ERR_INVALID;
   if (s.hd != 64 && s.hd != 128) return MK_ERR_INVALID;
   if (s.Hkv < 1 || s.Hq < s.Hkv || s.Hq % s.Hkv != 0) return MK_ERR_INVALID;
+  if (s.Hkv > 16) return MK_ERR_CAPACITY;
   const int G = s.Hq / s.Hkv;
   if (G > 4) return MK_ERR_CAPACITY;
   if ((G * s.hd) % 128 != 0) return MK_ERR_INVALID;
@@ -91,13 +96,13 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
   int sc_topk = B * s.E * 4 + B * 8 * 8 + s.E * 4 + 256;
   int sc_rn = B * 64 * 4 + 64;
-  int sc_comb = max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
+  int sc_comb = 3 * max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
   o->scratch_bytes = round_up(sc, 1024);
   const int fifo = kFifo * kFifoEntryWords * 4;
   const int max_stages = 14;
-  const int bars = round_up((2 * max_stages + 3 * kFifo + 8) * 8, 1024);
-  const int budget = 232448 - 1024;
+  const int bars = round_up((2 * max_stages + 4 * kFifo + 8) * 8, 1024);
+  const int budget = 232448 - 2048;   // max per block, less alignment slack and static smem
   int rest1 = bars + fifo + o->scratch_bytes + o->actA_stride + 2 * o->actB_bytes;
   int rest2 = rest1 + o->actA_stride;
   int nA = ((budget - rest2) / kStageBytes >= 8) ? 2 : 1;
@@ -119,13 +124,9 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
 
 namespace {
 
-enum ActKind { ACT_NONE = 0, ACT_A = 1, ACT_B = 2 };
 
 struct Task {
   int32_t w[kDescWords];
-  double bytes;
-  int act;
-  int keyA;
 };
 
 struct Layout {
@@ -169,9 +170,7 @@ Task make_task(int op, int layer, int phase) {
   t.w[D_MAP0] = -1;
   t.w[D_MAP1] = -1;
   t.w[D_PHASE] = phase;
-  t.bytes = 0.0;
-  t.act = ACT_NONE;
-  t.keyA = -1;
+  t.w[D_ACT] = ACT_NONE;
   return t;
 }
 
@@ -183,78 +182,6 @@ void add_wait(Task& t, int ctr, int n) {
 void add_signal(Task& t, int ctr) {
   int i = t.w[D_NSIG]++;
   t.w[D_S0 + i] = ctr;
-}
-
-// Simulated list scheduling: place each task on the CTA where it would
-// finish first, given per-CTA HBM stream time and consumer time, a ring that
-// lets the stream run ahead of the consumer, and counter-dependency times.
-struct Sim {
-  int n;
-  double bw;        // bytes per microsecond per CTA
-  double hop;       // counter visibility latency
-  double ovh;       // per-task consumer overhead
-  double ring_us;   // how far the stream may run ahead of the consumer
-  std::vector<double> t_stream, t_done;
-  std::vector<double> ctr_time;
-
-  int place(const Task& t) {
-    double dep = 0.0;
-    for (int i = 0; i < t.w[D_NWAIT]; ++i)
-      dep = std::max(dep, ctr_time[t.w[D_W0 + 2 * i]] + hop);
-    double pdep = 0.0;
-    if (t.w[D_PW] >= 0) pdep = ctr_time[t.w[D_PW]] + hop;
-    int best = 0;
-    double best_fin = 1e300, best_ss = 1e300, best_se = 0.0;
-    for (int c = 0; c < n; ++c) {
-      double ss = std::max(std::max(t_stream[c], t_done[c] - ring_us), pdep);
-      double se = ss + t.bytes / bw;
-      double fin = std::max(std::max(se, dep), t_done[c]) + ovh;
-      if (fin < best_fin - 1e-9 || (fin < best_fin + 1e-9 && t_stream[c] < best_ss)) {
-        best = c;
-        best_fin = fin;
-        best_ss = t_stream[c];
-        best_se = se;
-      }
-    }
-    t_stream[best] = std::max(t_stream[best], best_se);
-    t_done[best] = best_fin;
-    for (int i = 0; i < t.w[D_NSIG]; ++i) {
-      int s = t.w[D_S0 + i];
-      ctr_time[s] = std::max(ctr_time[s], best_fin);
-    }
-    return best;
-  }
-};
-
-// Mark slot usage along one CTA list: a normalized-input activation is loaded
-// when its level changes (into alternating buffers when two fit) and released
-// after its last use; every small activation is loaded into the next of two
-// buffers and released after its task.
-void mark_list(std::vector<Task*>& lst, int nA) {
-  int cur_key = -1, cur_buf = -1, n_loads = 0;
-  Task* last_a = nullptr;
-  int nb = 0;
-  for (size_t i = 0; i < lst.size(); ++i) {
-    Task& t = *lst[i];
-    t.w[D_SEQ] = (int32_t)i;
-    t.w[D_FLAGS] &= ~(F_LOAD_A | F_REL_A | F_LOAD_B);
-    if (t.act == ACT_A) {
-      if (t.keyA != cur_key) {
-        if (last_a) last_a->w[D_FLAGS] |= F_REL_A;
-        cur_buf = n_loads % nA;
-        ++n_loads;
-        cur_key = t.keyA;
-        t.w[D_FLAGS] |= F_LOAD_A;
-      }
-      t.w[D_X0] = cur_buf;
-      last_a = &t;
-    } else if (t.act == ACT_B) {
-      t.w[D_FLAGS] |= F_LOAD_B;
-      t.w[D_BSLOT] = nb & 1;
-      ++nb;
-    }
-  }
-  if (last_a) last_a->w[D_FLAGS] |= F_REL_A;
 }
 
 }  // namespace
@@ -299,13 +226,6 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   lay.build(L, B, S, Hkv, NR);
   std::vector<int32_t> targets(lay.total, 0);
 
-  // Expected use of expert slot j: slots are compacted in expert order, so
-  // low slots fill first; estimate E[#distinct experts] under uniform routing.
-  double exp_used = E * (1.0 - std::pow(1.0 - (double)k / E, (double)B));
-  auto p_slot = [&](int j) {
-    double p = exp_used - j;
-    return p >= 1.0 ? 1.0 : (p <= 0.0 ? 0.05 : std::max(0.05, p));
-  };
 
   std::vector<Task> tasks;
   tasks.reserve((size_t)L * (NR + n_qkv + n_rt + 1 + 2 * B * Hkv * max_chunks + NR * Hkv +
@@ -324,6 +244,30 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
       tasks.push_back(t);
     }
     if (l == L) break;
+    // -- router tiles
+    for (int t_i = 0; t_i < n_rt; ++t_i) {
+      Task t = make_task(OP_ROUTER, l, l * PH + 1);
+      t.w[D_A] = t_i;
+      t.w[D_ROW0] = t_i * r_qkv;
+      t.w[D_K0] = 0;
+      t.w[D_KCH] = d / 64;
+      t.w[D_R] = r_qkv;
+      t.w[D_NMAT] = 1;
+      t.w[D_MAP0] = map_of(l, 2);
+      t.w[D_NSTAGE] = (r_qkv / 16) * (d / 64) / 8;
+      add_wait(t, lay.norm(l), NR);
+      add_signal(t, lay.rpart(l));
+      targets[lay.rpart(l)] += 1;
+      t.w[D_ACT] = ACT_A;
+      tasks.push_back(t);
+    }
+    {
+      Task t = make_task(OP_TOPK, l, l * PH + 2);
+      add_wait(t, lay.rpart(l), n_rt);
+      add_signal(t, lay.rtr(l));
+      targets[lay.rtr(l)] += 1;
+      tasks.push_back(t);
+    }
     // -- QKV tiles (grouped by KV group so attention of a group starts early)
     for (int g = 0; g < Hkv; ++g) {
       auto emit_rows = [&](int row_begin, int rows) {
@@ -341,41 +285,13 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
           add_wait(t, lay.norm(l), NR);
           add_signal(t, lay.qkv(l, g));
           targets[lay.qkv(l, g)] += 1;
-          t.bytes = (double)r_qkv * d * 2;
-          t.act = ACT_A;
-          t.keyA = l;
+          t.w[D_ACT] = ACT_A;
           tasks.push_back(t);
         }
       };
       emit_rows(g * G * hd, G * hd);            // q heads of the group
       emit_rows(Hq * hd + g * hd, hd);          // k head
       emit_rows((Hq + Hkv) * hd + g * hd, hd);  // v head
-    }
-    // -- router tiles
-    for (int t_i = 0; t_i < n_rt; ++t_i) {
-      Task t = make_task(OP_ROUTER, l, l * PH + 1);
-      t.w[D_A] = t_i;
-      t.w[D_ROW0] = t_i * r_qkv;
-      t.w[D_K0] = 0;
-      t.w[D_KCH] = d / 64;
-      t.w[D_R] = r_qkv;
-      t.w[D_NMAT] = 1;
-      t.w[D_MAP0] = map_of(l, 2);
-      t.w[D_NSTAGE] = (r_qkv / 16) * (d / 64) / 8;
-      add_wait(t, lay.norm(l), NR);
-      add_signal(t, lay.rpart(l));
-      targets[lay.rpart(l)] += 1;
-      t.bytes = (double)std::min(r_qkv, E - t_i * r_qkv) * d * 2;
-      t.act = ACT_A;
-      t.keyA = l;
-      tasks.push_back(t);
-    }
-    {
-      Task t = make_task(OP_TOPK, l, l * PH + 2);
-      add_wait(t, lay.rpart(l), n_rt);
-      add_signal(t, lay.rtr(l));
-      targets[lay.rtr(l)] += 1;
-      tasks.push_back(t);
     }
     // -- attention chunks, then combines
     for (int g = 0; g < Hkv; ++g) {
@@ -399,8 +315,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
           long p0 = (long)c * out->ppc[b];
           long pages_now = ((long)seq_lens[b] + kPage - 1) / kPage;
           long np = std::max(0L, std::min((long)out->ppc[b], pages_now - p0));
-          t.bytes = (double)np * 2.0 * kPage * hd * 2.0;
-          t.act = ACT_B;
+          t.w[D_ACT] = ACT_B;
           tasks.push_back(t);
         }
       }
@@ -434,8 +349,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         add_wait(t, lay.atto(l, g), B);
         add_signal(t, lay.dt(l, r));
         targets[lay.dt(l, r)] += 1;
-        t.bytes = 64.0 * G * hd * 2;
-        t.act = ACT_B;
+        t.w[D_ACT] = ACT_B;
         tasks.push_back(t);
       }
     }
@@ -458,9 +372,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         add_wait(t, lay.norm(l), NR);
         add_signal(t, lay.slot(l, j));
         targets[lay.slot(l, j)] += 1;
-        t.bytes = 2.0 * r_ff * d * 2 * p_slot(j);
-        t.act = ACT_A;
-        t.keyA = l;
+        t.w[D_ACT] = ACT_A;
         tasks.push_back(t);
       }
     }
@@ -481,8 +393,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         add_wait(t, lay.slot(l, j), n_ff);
         add_signal(t, lay.dt(l, r));
         targets[lay.dt(l, r)] += 1;
-        t.bytes = 64.0 * F * 2 * p_slot(j);
-        t.act = ACT_B;
+        t.w[D_ACT] = ACT_B;
         tasks.push_back(t);
       }
     }
@@ -501,113 +412,72 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
     add_wait(t, lay.norm(L), NR);
     add_signal(t, lay.lmdone);
     targets[lay.lmdone] += 1;
-    t.bytes = 128.0 * d * 2;
-    t.act = ACT_A;
-    t.keyA = L;
+    t.w[D_ACT] = ACT_A;
     tasks.push_back(t);
   }
 
-  // ---- placement
-  Sim sim;
-  sim.n = n_ctas;
-  sim.bw = 6.5e12 / 1e6 / n_ctas;
-  sim.hop = 1.0;
-  sim.ovh = 0.25;
-  sim.ring_us = 160.0 * 1024.0 / sim.bw;
-  sim.t_stream.assign(n_ctas, 0.0);
-  sim.t_done.assign(n_ctas, 0.0);
-  sim.ctr_time.assign(lay.total, 0.0);
-  std::vector<std::vector<Task*>> lists(n_ctas);
-  for (auto& t : tasks) lists[sim.place(t)].push_back(&t);
-
-  // A-slot double buffering only where two buffers fit in shared memory.
+  // ---- priority order: stable sort by (layer, operation rank)
+  static const int kRank[OP_COUNT] = {
+      /*NONE*/ 99, /*RN*/ 0, /*QKV*/ 2, /*ROUTER*/ 1, /*TOPK*/ 3, /*ATTN*/ 4,
+      /*COMBINE*/ 6, /*OPROJ*/ 7, /*GATEUP*/ 5, /*DOWN*/ 8, /*LMHEAD*/ 9};
+  std::stable_sort(tasks.begin(), tasks.end(), [](const Task& x, const Task& y) {
+    if (x.w[D_LAYER] != y.w[D_LAYER]) return x.w[D_LAYER] < y.w[D_LAYER];
+    return kRank[x.w[D_OP]] < kRank[y.w[D_OP]];
+  });
+  // A-slot double buffering where two buffers fit in shared memory
   SmemLayout sl;
   int slrc = smem_layout(s, B, max_chunks, &sl);
   if (slrc != MK_OK) return slrc;
-  const int nA = sl.nA;
-  int max_tasks = 0;
-  for (auto& lst : lists) {
-    mark_list(lst, nA);
-    max_tasks = std::max(max_tasks, (int)lst.size());
-  }
-  max_tasks = std::max(max_tasks, 1);
+
+  const int n_tasks = (int)tasks.size();
+  const int n_phases = L * PH + 2;
+  // task dispensers: one for the fused list, one per phase list
+  const int grab = lay.total;
+  const int grab_phase0 = lay.total + 1;
+  const int n_counters = lay.total + 1 + n_phases;
+  targets.resize(n_counters, 0);
+  targets[grab] = n_tasks + n_ctas;
 
   out->release();
   out->n_ctas = n_ctas;
   out->B = B;
   out->S = S;
   out->max_chunks = max_chunks;
-  out->n_counters = lay.total;
-  out->max_tasks = max_tasks;
-  out->total_tasks = tasks.size();
+  out->n_counters = n_counters;
+  out->n_tasks = n_tasks;
   out->r_qkv = r_qkv;
   out->r_router = r_qkv;
-  out->n_phases = L * PH + 2;
-  out->desc = (int32_t*)std::calloc((size_t)n_ctas * max_tasks * kDescWords, sizeof(int32_t));
-  out->counts = (int32_t*)std::calloc((size_t)n_ctas, sizeof(int32_t));
-  out->targets = (int32_t*)std::calloc((size_t)lay.total, sizeof(int32_t));
-  if (!out->desc || !out->counts || !out->targets) {
+  out->n_phases = n_phases;
+  out->grab = grab;
+  out->grab_phase0 = grab_phase0;
+  out->desc = (int32_t*)std::malloc((size_t)n_tasks * kDescWords * sizeof(int32_t));
+  out->targets = (int32_t*)std::calloc((size_t)n_counters, sizeof(int32_t));
+  out->phase_desc = with_phases
+                        ? (int32_t*)std::malloc((size_t)n_tasks * kDescWords * sizeof(int32_t))
+                        : nullptr;
+  out->phase_off = (int32_t*)std::calloc((size_t)n_phases + 1, sizeof(int32_t));
+  if (!out->desc || !out->targets || !out->phase_off || (with_phases && !out->phase_desc)) {
     out->release();
     return MK_ERR_OOM;
   }
-  for (int c = 0; c < n_ctas; ++c) {
-    out->counts[c] = (int32_t)lists[c].size();
-    for (size_t i = 0; i < lists[c].size(); ++i)
-      std::memcpy(out->desc + ((size_t)c * max_tasks + i) * kDescWords, lists[c][i]->w,
-                  sizeof(int32_t) * kDescWords);
+  for (int i = 0; i < n_tasks; ++i)
+    std::memcpy(out->desc + (size_t)i * kDescWords, tasks[i].w, sizeof(int32_t) * kDescWords);
+  // phase lists: the same tasks grouped by phase, each group in priority order
+  std::vector<int> per_phase(n_phases, 0);
+  for (const auto& t : tasks) per_phase[t.w[D_PHASE]]++;
+  for (int ph = 0; ph < n_phases; ++ph) {
+    out->phase_off[ph + 1] = out->phase_off[ph] + per_phase[ph];
+    targets[grab_phase0 + ph] = per_phase[ph] + n_ctas;
   }
-  std::memcpy(out->targets, targets.data(), sizeof(int32_t) * lay.total);
-
   if (with_phases) {
-    // one launch per phase; inside a phase the tiles are spread like a
-    // conventional kernel's grid: least-loaded CTA by bytes.
-    const int nph = out->n_phases;
-    std::vector<std::vector<std::vector<Task*>>> pl(nph, std::vector<std::vector<Task*>>(n_ctas));
-    std::vector<std::vector<double>> load(nph, std::vector<double>(n_ctas, 0.0));
-    std::vector<int> rr(nph, 0);
-    for (auto& t : tasks) {
-      int ph = t.w[D_PHASE];
-      int best = 0;
-      double bl = 1e300;
-      for (int c = 0; c < n_ctas; ++c) {
-        int cc = (rr[ph] + c) % n_ctas;
-        if (load[ph][cc] < bl - 1e-9) {
-          bl = load[ph][cc];
-          best = cc;
-        }
-      }
-      rr[ph] = (best + 1) % n_ctas;
-      load[ph][best] += t.bytes + 4096.0;
-      pl[ph][best].push_back(&t);
-    }
-    int pmax = 1;
-    for (int ph = 0; ph < nph; ++ph)
-      for (int c = 0; c < n_ctas; ++c) pmax = std::max(pmax, (int)pl[ph][c].size());
-    out->phase_max_tasks = pmax;
-    out->phase_desc =
-        (int32_t*)std::calloc((size_t)nph * n_ctas * pmax * kDescWords, sizeof(int32_t));
-    out->phase_counts = (int32_t*)std::calloc((size_t)nph * n_ctas, sizeof(int32_t));
-    if (!out->phase_desc || !out->phase_counts) {
-      out->release();
-      return MK_ERR_OOM;
-    }
-    for (int ph = 0; ph < nph; ++ph) {
-      for (int c = 0; c < n_ctas; ++c) {
-        auto& lst = pl[ph][c];
-        // flags depend on list order: mark a private copy
-        std::vector<Task> copy;
-        copy.reserve(lst.size());
-        for (auto* t : lst) copy.push_back(*t);
-        std::vector<Task*> ptrs;
-        for (auto& t : copy) ptrs.push_back(&t);
-        mark_list(ptrs, nA);
-        out->phase_counts[(size_t)ph * n_ctas + c] = (int32_t)copy.size();
-        for (size_t i = 0; i < copy.size(); ++i)
-          std::memcpy(out->phase_desc + (((size_t)ph * n_ctas + c) * pmax + i) * kDescWords,
-                      copy[i].w, sizeof(int32_t) * kDescWords);
-      }
+    std::vector<int> fill(out->phase_off, out->phase_off + n_phases);
+    for (const auto& t : tasks) {
+      const int pos = fill[t.w[D_PHASE]]++;
+      std::memcpy(out->phase_desc + (size_t)pos * kDescWords, t.w, sizeof(int32_t) * kDescWords);
     }
   }
+  std::memcpy(out->targets, targets.data(), sizeof(int32_t) * n_counters);
+  (void)sl;
   return MK_OK;
 }
 
@@ -615,8 +485,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
 
 extern "C" mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batch,
                                       const int32_t* seq_lens, const int32_t* plan_len,
-                                      int32_t* meta, int32_t* counts, int32_t* desc,
-                                      int32_t* targets) {
+                                      int32_t* meta, int32_t* desc, int32_t* targets) {
   if (!cfg || !meta) return MK_ERR_INVALID;
   mk::Shape s{cfg->n_layers, cfg->d_model, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
               cfg->n_experts, cfg->top_k, cfg->d_ff, cfg->vocab, cfg->page_size,
@@ -627,19 +496,17 @@ extern "C" mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batc
   int rc = mk::plan_schedule(s, n_ctas, batch, seq_lens, plan_len, false, &p);
   if (rc != MK_OK) return (mk_status)rc;
   std::memset(meta, 0, 16 * sizeof(int32_t));
-  meta[0] = p.n_ctas;
-  meta[1] = p.max_tasks;
-  meta[2] = (int32_t)p.total_tasks;
-  meta[3] = p.n_counters;
-  meta[4] = p.S;
-  meta[5] = p.max_chunks;
-  meta[6] = mk::kDescWords;
-  meta[7] = p.n_phases;
-  meta[8] = p.r_qkv;
-  meta[9] = p.ppc[0];
-  if (counts) std::memcpy(counts, p.counts, sizeof(int32_t) * p.n_ctas);
-  if (desc)
-    std::memcpy(desc, p.desc, sizeof(int32_t) * (size_t)p.n_ctas * p.max_tasks * mk::kDescWords);
+  meta[0] = p.n_tasks;
+  meta[1] = p.n_counters;
+  meta[2] = p.S;
+  meta[3] = p.max_chunks;
+  meta[4] = mk::kDescWords;
+  meta[5] = p.n_phases;
+  meta[6] = p.r_qkv;
+  meta[7] = p.ppc[0];
+  meta[8] = p.grab;
+  meta[9] = p.grab_phase0;
+  if (desc) std::memcpy(desc, p.desc, sizeof(int32_t) * (size_t)p.n_tasks * mk::kDescWords);
   if (targets) std::memcpy(targets, p.targets, sizeof(int32_t) * p.n_counters);
   p.release();
   return MK_OK;

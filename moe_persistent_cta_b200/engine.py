@@ -103,6 +103,15 @@ class Decoder:
         if rc != mk.MK_OK:
             raise mk.MKError(rc, "device status", detail)
 
+    def set_trace(self, enable: bool) -> None:
+        mk.check_status(mk.lib.mk_set_trace(self._ctx, int(bool(enable))), "mk_set_trace")
+
+    def trace(self):
+        """(desc [n_tasks][32], trace [n_tasks][9]) of the last traced step."""
+        desc = self.debug(mk.MK_BUF_PLAN).reshape(-1, 32)
+        stamps = self.debug(mk.MK_BUF_TRACE).reshape(-1, mk.TRACE_WORDS)
+        return desc, stamps
+
     def set_timeout_ms(self, ms: int) -> None:
         mk.check_status(mk.lib.mk_set_timeout_ms(self._ctx, int(ms)), "mk_set_timeout_ms")
 
@@ -110,7 +119,9 @@ class Decoder:
         n = mk.lib.mk_debug_size(self._ctx, which)
         if n == 0:
             raise mk.MKError(mk.MK_ERR_STATE, "mk_debug_size")
-        dtype = np.int32 if which in (mk.MK_BUF_TOPK, mk.MK_BUF_NSLOTS) else np.float32
+        ints = (mk.MK_BUF_TOPK, mk.MK_BUF_NSLOTS, mk.MK_BUF_PLAN)
+        dtype = np.int32 if which in ints else (np.uint32 if which == mk.MK_BUF_TRACE
+                                                else np.float32)
         out = np.empty(n // 4, dtype=dtype)
         mk.check_status(mk.lib.mk_debug_read(self._ctx, which, out.ctypes.data_as(c_void_p), n),
                         "mk_debug_read")
@@ -131,22 +142,20 @@ class Decoder:
 def plan_schedule(shape: Dict, n_ctas: int, seq_lens: Sequence[int],
                   plan_len: Optional[Sequence[int]] = None, max_batch: int = 8,
                   n_pages: int = 1 << 20):
-    """Host-only planner (no GPU): returns (meta, counts, desc [n_ctas][max_tasks][32],
-    targets)."""
+    """Host-only planner (no GPU): returns (meta, desc [n_tasks][32], targets)."""
     cfg = mk.make_config(shape, max_batch, n_pages)
     B = len(seq_lens)
     sl = mk.int32_array(seq_lens)
     pl = mk.int32_array(plan_len) if plan_len is not None else None
     meta = (c_int32 * 16)()
-    mk.check_status(mk.lib.mk_plan_schedule(byref(cfg), n_ctas, B, sl, pl, meta, None, None,
-                                            None), "mk_plan_schedule")
+    mk.check_status(mk.lib.mk_plan_schedule(byref(cfg), n_ctas, B, sl, pl, meta, None, None),
+                    "mk_plan_schedule")
     m = [int(v) for v in meta]
-    max_tasks, n_counters = m[1], m[3]
-    counts = np.zeros(n_ctas, dtype=np.int32)
-    desc = np.zeros((n_ctas, max_tasks, 32), dtype=np.int32)
+    n_tasks, n_counters = m[0], m[1]
+    desc = np.zeros((n_tasks, 32), dtype=np.int32)
     targets = np.zeros(n_counters, dtype=np.int32)
     P = ctypes.POINTER(c_int32)
-    mk.check_status(mk.lib.mk_plan_schedule(
-        byref(cfg), n_ctas, B, sl, pl, meta, counts.ctypes.data_as(P), desc.ctypes.data_as(P),
-        targets.ctypes.data_as(P)), "mk_plan_schedule")
-    return m, counts, desc, targets
+    mk.check_status(mk.lib.mk_plan_schedule(byref(cfg), n_ctas, B, sl, pl, meta,
+                                            desc.ctypes.data_as(P), targets.ctypes.data_as(P)),
+                    "mk_plan_schedule")
+    return m, desc, targets

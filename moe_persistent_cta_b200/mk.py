@@ -18,11 +18,13 @@ MK_ERR_CAPACITY, MK_ERR_STATE, MK_ERR_DEVICE = 5, 6, 7
 
 MK_BUF_X, MK_BUF_QKV, MK_BUF_ATTN_O, MK_BUF_RLOGITS, MK_BUF_TOPK = 0, 1, 2, 3, 4
 MK_BUF_NSLOTS, MK_BUF_EXPERT_A, MK_BUF_MOE, MK_BUF_OPART = 5, 6, 7, 8
+MK_BUF_TRACE, MK_BUF_PLAN = 9, 10
+TRACE_WORDS = 9
 
 # every entry point the header declares (checked by the ABI test)
 EXPORTS = (
     "mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_step_unfused",
-    "mk_check", "mk_set_timeout_ms", "mk_debug_read", "mk_debug_size",
+    "mk_check", "mk_set_timeout_ms", "mk_set_trace", "mk_debug_read", "mk_debug_size",
     "mk_plan_schedule", "mk_strerror", "mk_destroy",
 )
 
@@ -72,10 +74,11 @@ def _load():
         "mk_decode_step_unfused": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_check": (c_int, [c_void_p, P(c_int32), P(c_int32)]),
         "mk_set_timeout_ms": (c_int, [c_void_p, c_int32]),
+        "mk_set_trace": (c_int, [c_void_p, c_int32]),
         "mk_debug_read": (c_int, [c_void_p, c_int, c_void_p, c_size_t]),
         "mk_debug_size": (c_size_t, [c_void_p, c_int]),
         "mk_plan_schedule": (c_int, [P(mk_config), c_int, c_int, P(c_int32), P(c_int32),
-                                     P(c_int32), P(c_int32), P(c_int32), P(c_int32)]),
+                                     P(c_int32), P(c_int32), P(c_int32)]),
         "mk_strerror": (c_char_p, [c_int]),
         "mk_destroy": (None, [c_void_p]),
     }

@@ -1,11 +1,12 @@
 """Host schedule planner: structure, counter targets and deadlock freedom.
 
-The planner's per-CTA lists must (a) contain every tile of every operation
-exactly once, (b) give every counter exactly as many signalling tasks as its
-per-step target, and (c) let a step finish when every CTA executes its list
-in order and each task only waits on counters -- the property that lets the
-persistent kernel spin on counters without deadlocking (every list is a
-subsequence of one topological order, all CTAs co-resident).
+The step is one task list; at run time every CTA takes the next task with an
+atomic add, posts it to its in-order task FIFO and runs it.  The step cannot
+deadlock if (a) every counter a task waits on is signalled only by tasks that
+are earlier in the list (the earlier tasks were taken by running, co-resident
+CTAs that finish their FIFOs in order) and (b) every counter's per-step target
+equals the number of tasks that signal it.  These tests check both, plus the
+list's structure, on CPU.
 """
 
 import collections
@@ -13,70 +14,75 @@ import collections
 import numpy as np
 import pytest
 
-from moe_persistent_cta_b200 import configs, engine
+from moe_persistent_cta_b200 import configs, engine, synth
 
 D_OP, D_LAYER, D_A, D_B, D_C, D_D, D_FLAGS, D_NWAIT = 0, 1, 2, 3, 4, 5, 6, 7
 D_W0, D_W0N, D_PW, D_PWN, D_NSIG, D_S0 = 8, 9, 12, 13, 14, 15
-D_NSTAGE, D_ROW0, D_K0, D_KCH, D_R, D_NMAT, D_BSLOT, D_SEQ, D_X0 = 17, 18, 19, 20, 21, 22, 25, 26, 29
+D_NSTAGE, D_ROW0, D_K0, D_KCH, D_R, D_NMAT, D_ACT, D_PPC, D_PHASE = 17, 18, 19, 20, 21, 22, 25, 27, 28
 OP_RN, OP_QKV, OP_ROUTER, OP_TOPK, OP_ATTN, OP_COMBINE, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM = range(1, 11)
-F_LOAD_A, F_REL_A, F_LOAD_B, F_LAST, F_SINGLE = 1, 2, 4, 8, 16
+ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 
-def lists_of(counts, desc):
-    return [desc[c, : counts[c]] for c in range(len(counts))]
+def check_order_and_targets(desc, targets, n_ctas, grab):
+    """(a) waits only on earlier signallers, (b) targets == signaller counts;
+    then simulate a greedy dynamic execution on n_ctas CTAs."""
+    n = len(desc)
+    first_sig = {}
+    last_sig = {}
+    count = collections.Counter()
+    for i, t in enumerate(desc):
+        for s in range(t[D_NSIG]):
+            c = int(t[D_S0 + s])
+            count[c] += 1
+            first_sig.setdefault(c, i)
+            last_sig[c] = i
+    for i, t in enumerate(desc):
+        waits = [(int(t[D_W0 + 2 * w]), int(t[D_W0N + 2 * w])) for w in range(t[D_NWAIT])]
+        if t[D_PW] >= 0:
+            waits.append((int(t[D_PW]), int(t[D_PWN])))
+        for c, need in waits:
+            assert count[c] == need, f"task {i}: counter {c} has {count[c]} signallers, waits {need}"
+            assert last_sig[c] < i, f"task {i} waits on counter {c} signalled later (task {last_sig[c]})"
+    for c, k in count.items():
+        assert targets[c] == k
+    assert targets[grab] == n + n_ctas
+    # greedy dynamic execution: each CTA takes the next task when it has finished
+    # its previous one; a task finishes when its waits are met (unit time)
+    done_at = {}
+    ctr_done = collections.defaultdict(int)
+    ctr_time = collections.defaultdict(float)
+    free = [0.0] * n_ctas
+    for i, t in enumerate(desc):
+        c = int(np.argmin(free))
+        start = free[c]
+        waits = [int(t[D_W0 + 2 * w]) for w in range(t[D_NWAIT])]
+        if t[D_PW] >= 0:
+            waits.append(int(t[D_PW]))
+        for w in waits:
+            assert ctr_done[w] == count[w]     # every signaller already taken earlier
+            start = max(start, ctr_time[w])
+        free[c] = start + 1.0
+        for s in range(t[D_NSIG]):
+            w = int(t[D_S0 + s])
+            ctr_done[w] += 1
+            ctr_time[w] = max(ctr_time[w], free[c])
+        done_at[i] = free[c]
+    return max(done_at.values())
 
 
-def simulate(counts, desc, targets, epochs=2):
-    """Run every CTA's list in order, a task completing as soon as its loader
-    waits and its producer wait are met.  Returns final counter values."""
-    n = len(counts)
-    ctr = np.zeros(len(targets), dtype=np.int64)
-    for ep in range(1, epochs + 1):
-        pos = [0] * n
-        progress = True
-        while progress:
-            progress = False
-            for c in range(n):
-                while pos[c] < counts[c]:
-                    t = desc[c, pos[c]]
-                    ok = True
-                    for w in range(t[D_NWAIT]):
-                        if ctr[t[D_W0 + 2 * w]] < ep * t[D_W0N + 2 * w]:
-                            ok = False
-                    if t[D_PW] >= 0 and ctr[t[D_PW]] < ep * t[D_PWN]:
-                        ok = False
-                    if not ok:
-                        break
-                    for s in range(t[D_NSIG]):
-                        ctr[t[D_S0 + s]] += 1
-                    pos[c] += 1
-                    progress = True
-        stuck = [c for c in range(n) if pos[c] < counts[c]]
-        assert not stuck, f"epoch {ep}: CTAs {stuck[:5]} cannot make progress (deadlock)"
-        assert np.array_equal(ctr, ep * targets.astype(np.int64))
-    return ctr
-
-
-@pytest.mark.parametrize("name,n_ctas,lens", [
-    ("tiny", 148, [128]),
-    ("tiny", 7, [128]),
-    ("tiny", 3, [0]),
-    ("tiny", 148, [5, 64, 65, 300]),
-])
-def test_tiny_plan_simulates(name, n_ctas, lens):
-    shape = configs.TINY
-    meta, counts, desc, targets = engine.plan_schedule(shape, n_ctas, lens)
-    assert meta[0] == n_ctas
-    assert counts.sum() == meta[2]
-    simulate(counts, desc, targets)
+@pytest.mark.parametrize("n_ctas,lens", [(148, [128]), (7, [128]), (3, [0]),
+                                         (148, [5, 64, 65, 300])])
+def test_tiny_plan(n_ctas, lens):
+    meta, desc, targets = engine.plan_schedule(configs.TINY, n_ctas, lens)
+    assert meta[0] == len(desc)
+    check_order_and_targets(desc, targets, n_ctas, meta[8])
 
 
 def test_30b_b1_plan_structure():
     shape = configs.MOE30B
-    meta, counts, desc, targets = engine.plan_schedule(shape, 148, [8192])
-    simulate(counts, desc, targets, epochs=1)
-    allt = np.concatenate(lists_of(counts, desc))
-    ops = collections.Counter(allt[:, D_OP].tolist())
+    meta, desc, targets = engine.plan_schedule(shape, 148, [8192])
+    check_order_and_targets(desc, targets, 148, meta[8])
+    ops = collections.Counter(desc[:, D_OP].tolist())
     L, d = shape["n_layers"], shape["d_model"]
     qkv_rows = (shape["n_q_heads"] + 2 * shape["n_kv_heads"]) * shape["head_dim"]
     assert ops[OP_RN] == (L + 1) * d // 64
@@ -88,68 +94,46 @@ def test_30b_b1_plan_structure():
     assert ops[OP_GATEUP] == L * S * shape["d_ff"] // 16
     assert ops[OP_DOWN] == L * S * d // 64
     assert ops[OP_LM] == shape["vocab"] // 128
-    # every (layer, tile) of QKV appears exactly once
-    q = allt[allt[:, D_OP] == OP_QKV]
-    keys = set(zip(q[:, D_LAYER].tolist(), q[:, D_ROW0].tolist()))
-    assert len(keys) == len(q)
-    # attention chunks cover all cached pages of every (layer, group)
-    a = allt[allt[:, D_OP] == OP_ATTN]
-    nc = a[0, D_D]
-    ppc = a[0, 27]
+    q = desc[desc[:, D_OP] == OP_QKV]
+    assert len(set(zip(q[:, D_LAYER].tolist(), q[:, D_ROW0].tolist()))) == len(q)
+    a = desc[desc[:, D_OP] == OP_ATTN]
+    nc, ppc = a[0, D_D], a[0, D_PPC]
     assert nc * ppc * 64 >= 8192 + 64
     assert len(a) == L * shape["n_kv_heads"] * nc
-    # balance: the bytes each CTA streams are within a few percent
-    assert counts.max() <= 2 * counts.min() + 64
+    # priority order inside a layer: gate/up ahead of the attention tail
+    lay = desc[desc[:, D_LAYER] == 3]
+    pos = {op: np.where(lay[:, D_OP] == op)[0] for op in (OP_GATEUP, OP_COMBINE, OP_OPROJ,
+                                                           OP_ROUTER, OP_QKV, OP_DOWN)}
+    assert pos[OP_ROUTER].max() < pos[OP_QKV].min()
+    assert pos[OP_GATEUP].max() < pos[OP_COMBINE].min() < pos[OP_OPROJ].min()
+    assert pos[OP_OPROJ].max() < pos[OP_DOWN].min()
 
 
-def test_30b_b8_plan_simulates():
+def test_30b_b8_plan():
     shape = configs.MOE30B
-    from moe_persistent_cta_b200 import synth
     lens = synth.seq_lengths(("uniform", 1024, 16384, 4), 8)
-    meta, counts, desc, targets = engine.plan_schedule(shape, 148, lens)
-    simulate(counts, desc, targets, epochs=1)
-    assert meta[4] == 64   # expert slots = min(E, B*k)
+    meta, desc, targets = engine.plan_schedule(shape, 148, lens)
+    check_order_and_targets(desc, targets, 148, meta[8])
+    assert meta[2] == 64   # expert slots = min(E, B*k)
 
 
-def test_activation_slot_flags():
-    """Slot A is (re)loaded exactly when the normalized-input level changes
-    along a CTA's list and released after the last task of each run; every
-    small-activation task loads and alternates its buffer."""
-    meta, counts, desc, targets = engine.plan_schedule(configs.MOE30B, 148, [8192])
-    a_ops = (OP_QKV, OP_ROUTER, OP_GATEUP, OP_LM)
-    b_ops = (OP_ATTN, OP_OPROJ, OP_DOWN)
-    for lst in lists_of(counts, desc):
-        cur = None
-        nb = 0
-        last_a = None
-        for i, t in enumerate(lst):
-            assert t[D_SEQ] == i
-            op = t[D_OP]
-            if op in a_ops:
-                level = t[D_LAYER]
-                if level != cur:
-                    assert t[D_FLAGS] & F_LOAD_A
-                    if last_a is not None:
-                        assert last_a[D_FLAGS] & F_REL_A
-                    cur = level
-                else:
-                    assert not (t[D_FLAGS] & F_LOAD_A)
-                last_a = t
-            if op in b_ops:
-                assert t[D_FLAGS] & F_LOAD_B
-                assert t[D_BSLOT] == nb % 2
-                nb += 1
-            else:
-                assert not (t[D_FLAGS] & F_LOAD_B)
+def test_activation_levels_never_decrease():
+    """The runtime reuses slot A while consecutive A-tasks read the same
+    level; that is only sound if levels never go back along the list."""
+    for shape, lens in ((configs.TINY, [70, 3]), (configs.MOE30B, [8192])):
+        meta, desc, targets = engine.plan_schedule(shape, 148, lens)
+        a = desc[desc[:, D_ACT] == ACT_A]
+        assert np.all(np.diff(a[:, D_LAYER]) >= 0)
+        assert set(desc[desc[:, D_ACT] == ACT_A][:, D_OP]) <= {OP_QKV, OP_ROUTER, OP_GATEUP, OP_LM}
+        assert set(desc[desc[:, D_ACT] == ACT_B][:, D_OP]) <= {OP_ATTN, OP_OPROJ, OP_DOWN}
 
 
 def test_gemv_tiles_fill_whole_stages():
     """Every GEMV tile streams whole 16 KB stages: n_mat * R/16 * KCH units
     of 2 KB, a multiple of 8 per stage."""
     for shape in (configs.TINY, configs.MOE30B):
-        meta, counts, desc, targets = engine.plan_schedule(shape, 148, [100])
-        allt = np.concatenate(lists_of(counts, desc))
-        g = allt[np.isin(allt[:, D_OP], [OP_QKV, OP_ROUTER, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM])]
+        meta, desc, targets = engine.plan_schedule(shape, 148, [100])
+        g = desc[np.isin(desc[:, D_OP], [OP_QKV, OP_ROUTER, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM])]
         units = g[:, D_NMAT] * (g[:, D_R] // 16) * g[:, D_KCH]
         assert np.all(units % 8 == 0)
         assert np.all(units // 8 == g[:, D_NSTAGE])
@@ -158,11 +142,9 @@ def test_gemv_tiles_fill_whole_stages():
 
 
 def test_invalid_shapes_rejected():
-    import ctypes
     from moe_persistent_cta_b200 import mk
-    bad = dict(configs.TINY, head_dim=96)
     with pytest.raises(mk.MKError):
-        engine.plan_schedule(bad, 148, [10])
+        engine.plan_schedule(dict(configs.TINY, head_dim=96), 148, [10])
     with pytest.raises(mk.MKError):
         engine.plan_schedule(configs.TINY, 148, [10] * 9)      # batch > 8
     with pytest.raises(mk.MKError):
