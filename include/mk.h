@@ -181,12 +181,17 @@ mk_status mk_set_timeout_ms(mk_ctx* ctx, int32_t ms);
  *   MK_BUF_EXPERT_A float [L][S][B][F]       SwiGLU activation per slot
  *   MK_BUF_MOE      float [L][k][B][d]       weighted expert outputs by rank
  *   MK_BUF_OPART    float [L][Hkv][B][d]     O-proj output per KV group
- *   MK_BUF_TRACE    uint32 [n_tasks][9] per task of the last traced step (see
+ *   MK_BUF_TRACE    uint32 [n_tasks][18] per task of the last traced step (see
  *                   mk_set_trace): globaltimer stamps (ns, low 32 bits) of
  *                   producer resolved, producer issued last stage, loader
  *                   deps met, loader activation issued, consumer picked up,
  *                   consumer has activation, consumer math done, consumer
- *                   epilogue done; then the CTA that ran it, plus one
+ *                   epilogue done; then the CTA that ran it, plus one; then
+ *                   SM clock cycles the consumer waited for stage data, of
+ *                   the consumer's whole stage loop, and the producer waited
+ *                   for free stages; then the consumer's SM clock (low 32
+ *                   bits) at pickup, activation ready, tile routine entry,
+ *                   stage loop end, reduction end, epilogue end
  *   MK_BUF_PLAN     int32 [n_tasks][32] descriptors of the schedule
  * `bytes` must equal the buffer's size for the current schedule.            */
 enum {

@@ -330,10 +330,10 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   const int B = batch, L = s.L, d = s.d, G = s.Hq / s.Hkv, NR = d / 64, S = plan.S;
   const int qkvR = (s.Hq + 2 * s.Hkv) * s.hd;
   const int part_stride = round_up(2 * G + G * s.hd, 4);
-  const int actA_frag = 4 * d * B;
-  const int actA_bytes = actA_frag + round_up(NR * B * 4, 16);
-  const int ofrag_bytes = 4 * G * s.hd * B;
-  const int afrag_bytes = 4 * s.F * B;
+  const int actA_rows = 4 * (d + mk::kActPad) * B;
+  const int actA_bytes = actA_rows + round_up(NR * B * 4, 16);
+  const int ofrag_bytes = 4 * (G * s.hd + mk::kActPad) * B;
+  const int afrag_bytes = 4 * (s.F + mk::kActPad) * B;
   const int rwords = mk::route_words(B, s.k, S);
   auto fail = [&](mk_status st) {
     plan.release();
@@ -385,7 +385,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.part_stride = part_stride;
   p.eps = s.eps;
   p.actA_bytes = actA_bytes;
-  p.actA_frag_bytes = actA_frag;
+  p.actA_rows_bytes = actA_rows;
   p.ofrag_bytes = ofrag_bytes;
   p.afrag_bytes = afrag_bytes;
   p.route_words = rwords;
@@ -451,7 +451,9 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   p.logits = logits;
-  p.timeout_ns = c->timeout_ns;
+  // deadlines count SM cycles: 2 per ns bounds the wall time from below at
+  // any clock up to 2 GHz (a slower clock only lengthens the deadline)
+  p.timeout_cycles = c->timeout_ns * 2ull;
   p.epoch = c->epoch + 1;
   cudaError_t e = cudaSuccess;
   p.n_ctas = c->plan.n_ctas;

@@ -34,7 +34,11 @@ constexpr int kThreads = (kFirstConsumerWarp + kConsumerWarps) * 32;   // 352
 constexpr int kFifo = 16;            // task entries in flight per CTA
 constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words
 constexpr int kMapsPerLayer = 8;     // qkv, o, router, gate, up, down, kpool, vpool
-constexpr int kTraceWords = 9;       // per task: see TraceField
+// Activation rows are padded by 8 floats so that the 8 columns a warp reads
+// at one k land in different shared-memory banks.
+constexpr int kActPad = 8;
+constexpr int kRnStage = 4096;       // floats of residual partials staged per round
+constexpr int kTraceWords = 18;      // per task: see TraceField
 
 // Per-task trace words: globaltimer stamps (low 32 bits, ns) and the CTA
 // that ran the task.
@@ -47,7 +51,16 @@ enum TraceField : int {
   T_C_ACT = 5,        // consumers have the activation
   T_C_MATH = 6,       // consumers finished the streamed stages
   T_C_END = 7,        // consumers finished the epilogue
-  T_CTA = 8           // CTA index + 1
+  T_CTA = 8,          // CTA index + 1
+  T_C_WAITCYC = 9,    // SM cycles consumer warp 0 waited for stage data
+  T_C_LOOPCYC = 10,   // SM cycles of the consumer's stage loop
+  T_P_WAITCYC = 11,   // SM cycles the producer waited for free stages
+  T_K0 = 12,          // SM clock (low 32 bits) at: consumer pickup,
+  T_K1 = 13,          //   activation ready,
+  T_K2 = 14,          //   tile routine entry,
+  T_K3 = 15,          //   stage loop end,
+  T_K4 = 16,          //   cross-warp reduction end,
+  T_K5 = 17           //   epilogue end
 };
 
 // ---------------------------------------------------------------- opcodes --
@@ -122,10 +135,10 @@ struct Params {
   int max_chunks, max_pages, n_pages, part_stride;
   float eps;
   // byte sizes of the activation formats
-  int actA_bytes;      // per level: B-fragment fp32 of gamma*x + ss partials
-  int actA_frag_bytes; // per level: the fragment part
-  int ofrag_bytes;     // per (layer, group)
-  int afrag_bytes;     // per (layer, slot)
+  int actA_bytes;      // per level: rows of gamma*x (fp32) + ss partials
+  int actA_rows_bytes; // per level: the rows part, B x (d + kActPad) floats
+  int ofrag_bytes;     // per (layer, group): B x (G*hd + kActPad) floats
+  int afrag_bytes;     // per (layer, slot): B x (F + kActPad) floats
   int route_words;     // per layer
   // schedule: one list in topological priority order; CTAs take the next
   // task with an atomic add on counters[grab]
@@ -166,7 +179,7 @@ struct Params {
   float* moe_part;   // [L][k][B][d]
   int32_t* status;   // [16]
   uint32_t* trace;   // null, or [n_tasks][kTraceWords]
-  unsigned long long timeout_ns;
+  unsigned long long timeout_cycles;   // per-wait deadline in SM clock cycles
   // shared-memory layout (byte offsets from the 1024-aligned base)
   int n_stages, nA, actA_stride;
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, actB_bytes, off_ring;

@@ -44,6 +44,8 @@ constexpr unsigned FULL = 0xffffffffu;
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// %globaltimer is slow to read: used for trace stamps only.  Deadlines of
+// the wait loops count SM clock cycles (clock64), which is cheap.
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -76,6 +78,20 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
+}
+// Same test, but a thread whose phase is not complete is suspended (up to
+// the hint, in ns) until it completes instead of returning at once, so
+// waiting warps do not take issue slots from the math warps.
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
 }
 __device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar,
                                        uint64_t policy) {
@@ -144,6 +160,26 @@ __device__ __forceinline__ int cbar_or(int pred) {
   return r;
 }
 
+// Approximate PTX math (each within ~2^-22 relative): short instruction
+// sequences keep the interpreter's code, and so its instruction-cache
+// footprint, small.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float fexp(float x) { return ex2(x * 1.4426950408889634f); }
+__device__ __forceinline__ float frcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float frsqrt(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // bf16 helpers
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -151,12 +187,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16r(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
-}
-// B-operand fragment entry for 16 consecutive k of one column: the four
-// fp32 values the lane of the quad owns, in mma register order.
-__device__ __forceinline__ uint4 frag_entry(float v0, float v1, float v2, float v3) {
-  return make_uint4(__float_as_uint(v0), __float_as_uint(v1), __float_as_uint(v2),
-                    __float_as_uint(v3));
 }
 // Split a pair of fp32 values into three bf16x2 terms hi + mid + lo that sum
 // to the pair within 2^-27 relative (each difference is exact in fp32).
@@ -233,12 +263,11 @@ __device__ __noinline__ void raise_error(const Params& p, int code, int task, in
 }
 
 // Bounded spin on a global counter (one lane).
-__device__ __noinline__ bool wait_counter(const Params& p, int ctr, uint32_t target, int task,
-                                          int op) {
+__device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_t target,
+                                               int task, int op) {
   const uint32_t* c = p.counters + ctr;
-  uint32_t v = ld_acquire(c);
-  if (v >= target) return true;
-  const uint64_t t0 = gtimer();
+  uint32_t v;
+  const uint64_t t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     v = ld_acquire(c);
     if (v >= target) return true;
@@ -248,7 +277,7 @@ __device__ __noinline__ bool wait_counter(const Params& p, int ctr, uint32_t tar
         set_abort();
         return false;
       }
-      if (gtimer() - t0 > p.timeout_ns) {
+      if ((uint64_t)clock64() - t0 > p.timeout_cycles) {
         raise_error(p, MK_ERR_TIMEOUT, task, op, ctr, v, target, 0);
         set_abort();
         return false;
@@ -257,16 +286,21 @@ __device__ __noinline__ bool wait_counter(const Params& p, int ctr, uint32_t tar
   }
 }
 
+__device__ __forceinline__ bool wait_counter(const Params& p, int ctr, uint32_t target, int task,
+                                             int op) {
+  if (ld_acquire(p.counters + ctr) >= target) return true;
+  return wait_counter_slow(p, ctr, target, task, op);
+}
+
 // Bounded wait on a shared-memory mbarrier phase (every calling lane): the
 // common already-complete case inline, the spin out of line.
 __device__ __noinline__ bool wait_bar_slow(const Params& p, uint32_t bar, uint32_t parity,
                                            int aux) {
-  const uint64_t t0 = gtimer();
+  const uint64_t t0 = clock64();
   for (;;) {
-    for (int i = 0; i < 8; ++i)
-      if (mbar_test(bar, parity)) return true;
+    if (mbar_wait_hint(bar, parity)) return true;
     if (aborted()) return false;
-    if (gtimer() - t0 > p.timeout_ns) {
+    if ((uint64_t)clock64() - t0 > p.timeout_cycles) {
       raise_error(p, MK_ERR_TIMEOUT, -1, -1, -1, 0, 0, aux);
       set_abort();
       return false;
@@ -289,9 +323,9 @@ __device__ __forceinline__ bool warp_wait(const Params& p, uint32_t bar, uint32_
 
 // Wait for a phase that is known to complete (copies in flight), bounded.
 __device__ __noinline__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = gtimer();
-  while (!mbar_test(bar, parity)) {
-    if (gtimer() - t0 > p.timeout_ns) break;
+  const uint64_t t0 = clock64();
+  while (!mbar_wait_hint(bar, parity)) {
+    if ((uint64_t)clock64() - t0 > p.timeout_cycles) break;
   }
 }
 
@@ -299,6 +333,13 @@ __device__ __forceinline__ void stamp(const Params& p, int task, int field) {
   if (p.trace) p.trace[(size_t)task * kTraceWords + field] = (uint32_t)gtimer();
 }
 
+
+__device__ __forceinline__ void trace_put(const Params& p, int task, int field, uint32_t v) {
+  if (p.trace) p.trace[(size_t)task * kTraceWords + field] = v;
+}
+__device__ __forceinline__ void cstamp(const Params& p, int task, int field) {
+  if (p.trace) p.trace[(size_t)task * kTraceWords + field] = (uint32_t)clock64();
+}
 
 __device__ __forceinline__ const void* tmap(const Params& p, int idx) {
   return static_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
@@ -334,6 +375,7 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     const int layer = __shfl_sync(FULL, dw, D_LAYER);
     int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
     int32_t rw = 0;  // resolved word `lane`
+    uint32_t pwait = 0;
     int expert = -1, ntok = 0, p0 = 0, seqlen = 0, phys_new = -1;
     bool fail = false;
     if (op == OP_GATEUP || op == OP_DOWN) {
@@ -468,10 +510,12 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       for (int s = 0; s < nstage; ++s) {
         const uint32_t slot = stage_ctr % NS;
         const uint32_t ph = (stage_ctr / NS) & 1;
+        const uint64_t w0 = clock64();
         if (!warp_wait(p, sm.empty(slot), ph ^ 1, 102)) {
           fail = true;
           break;
         }
+        pwait += (uint32_t)(clock64() - w0);
         if (lane == 0) {
           const uint32_t fb = sm.full(slot);
           mbar_expect_tx(fb, kStageBytes);
@@ -487,7 +531,10 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       }
       if (fail) break;
     }
-    if (lane == 0) stamp(p, t, T_P_ISSUED);
+    if (lane == 0) {
+      stamp(p, t, T_P_ISSUED);
+      trace_put(p, t, T_P_WAITCYC, pwait);
+    }
   }
   // drain: every fill issued must land before the CTA may exit (stage s was
   // filled (stage_ctr - 1 - s) / NS + 1 times; wait for the last fill's phase)
@@ -623,76 +670,212 @@ __device__ __noinline__ void signal_loop(const Params& p) {
 __device__ __forceinline__ void level_rstd(const Params& p, const uint8_t* actA, float* rstd_out) {
   MK_CONSUMER_IDS;
   if (cw < p.B) {
-    const float* ss = reinterpret_cast<const float*>(actA + p.actA_frag_bytes);
+    const float* ss = reinterpret_cast<const float*>(actA + p.actA_rows_bytes);
     float acc = 0.f;
     for (int r = lane; r < p.NR; r += 32) acc += ss[r * p.B + cw];
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if (lane == 0) rstd_out[cw] = 1.0f / sqrtf(acc / (float)p.d + p.eps);
+    if (lane == 0) rstd_out[cw] = frsqrt(acc / (float)p.d + p.eps);
   }
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Stage ring position: slot and phase advance together (no division in
+// the stage loops).
+struct Ring {
+  uint32_t slot, phase;
+  int NS;
+  __device__ void init(uint32_t stage_ctr, int ns) {
+    NS = ns;
+    slot = stage_ctr % (uint32_t)ns;
+    phase = (stage_ctr / (uint32_t)ns) & 1u;
+  }
+  __device__ void next() {
+    if (++slot == (uint32_t)NS) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// CUDA-core stage loop for 1 or 2 activation columns: exact fp32 FMAs of
+// bf16 weights (widened by a shift/mask) with fp32 activations.  Lane l reads
+// 16-byte chunk (l & 7) of rows (l >> 3) + 4i of its warp's 16-row unit, so a
+// warp's 32 lanes cover the unit's 512 bytes per row group without bank
+// conflicts; partial sums are reduced over the 8 lanes of a row at the end.
+template <int NB>
+__device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm, int nstage,
+                                                 int kcps, int kl, uint32_t xaddr0,
+                                                 uint32_t xaddr1, Ring& ring, float* part_w,
+                                                 uint32_t& waitcyc) {
+  MK_CONSUMER_IDS;
+  const int c = lane & 7, rg = lane >> 3;
+  float acc[4][NB];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[i][b] = 0.f;
+  uint32_t woff[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rg + 4 * i;
+    woff[i] = r * 128 + ((c ^ (r & 7)) << 4);
+  }
+  const uint32_t ring0 = saddr(sm.ring) + cw * kUnitBytes;
+  for (int s = 0; s < nstage; ++s) {
+    const uint64_t w0 = clock64();
+    wait_bar(p, sm.full(ring.slot), ring.phase, 400);
+    waitcyc += (uint32_t)(clock64() - w0);
+    __syncwarp();
+    const uint32_t ub = ring0 + ring.slot * kStageBytes;
+    const uint32_t koff = (uint32_t)((s * kcps + kl) * 64 + 8 * c) * 4u;
+    uint4 w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = lds128(ub + woff[i]);
+    float4 xa[NB], xb[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const uint32_t xo = (b == 0 ? xaddr0 : xaddr1) + koff;
+      const uint4 u0 = lds128(xo), u1 = lds128(xo + 16);
+      xa[b] = make_float4(__uint_as_float(u0.x), __uint_as_float(u0.y), __uint_as_float(u0.z),
+                          __uint_as_float(u0.w));
+      xb[b] = make_float4(__uint_as_float(u1.x), __uint_as_float(u1.y), __uint_as_float(u1.z),
+                          __uint_as_float(u1.w));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(ring.slot));
+    ring.next();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        float a = acc[i][b];
+        a = fmaf(lo_bf16(w[i].x), xa[b].x, a);
+        a = fmaf(hi_bf16(w[i].x), xa[b].y, a);
+        a = fmaf(lo_bf16(w[i].y), xa[b].z, a);
+        a = fmaf(hi_bf16(w[i].y), xa[b].w, a);
+        a = fmaf(lo_bf16(w[i].z), xb[b].x, a);
+        a = fmaf(hi_bf16(w[i].z), xb[b].y, a);
+        a = fmaf(lo_bf16(w[i].w), xb[b].z, a);
+        a = fmaf(hi_bf16(w[i].w), xb[b].w, a);
+        acc[i][b] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float a = acc[i][b];
+      a += __shfl_xor_sync(FULL, a, 1);
+      a += __shfl_xor_sync(FULL, a, 2);
+      a += __shfl_xor_sync(FULL, a, 4);
+      if (c == 0) part_w[(rg + 4 * i) * 8 + b] = a;
+    }
+}
+
+// Tensor-core stage loop for 3..8 activation columns: weights as the 16-row
+// A operand (ldmatrix from the swizzled tile), the fp32 activation columns
+// as the B operand split into three bf16 terms (hi + mid + lo, exact
+// differences, ~24 bits), accumulated into three independent fp32 chains.
+__device__ __forceinline__ void gemv_stages_mma(const Params& p, const Smem& sm, int nstage,
+                                                int kcps, int kl, uint32_t xaddr, Ring& ring,
+                                                float* part_w, uint32_t& waitcyc) {
+  MK_CONSUMER_IDS;
+  const int g8 = lane >> 2, q = lane & 3;
+  float ah[4] = {0.f, 0.f, 0.f, 0.f}, am[4] = {0.f, 0.f, 0.f, 0.f},
+        al[4] = {0.f, 0.f, 0.f, 0.f};
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int achunk_hi = lane >> 4;
+  const uint32_t ring0 = saddr(sm.ring) + cw * kUnitBytes + arow * 128;
+  for (int s = 0; s < nstage; ++s) {
+    const uint64_t w0 = clock64();
+    wait_bar(p, sm.full(ring.slot), ring.phase, 400);
+    waitcyc += (uint32_t)(clock64() - w0);
+    __syncwarp();
+    const uint32_t ub = ring0 + ring.slot * kStageBytes;
+    const uint32_t kbase = xaddr + (uint32_t)((s * kcps + kl) * 64 + 2 * q) * 4u;
+    uint32_t a[4][4];
+    float2 b0[4], b1[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int chunk = 2 * i + achunk_hi;
+      ldsm_x4(ub + ((chunk ^ (arow & 7)) << 4), a[i][0], a[i][1], a[i][2], a[i][3]);
+      b0[i] = lds64f(kbase + i * 64);
+      b1[i] = lds64f(kbase + i * 64 + 32);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(ring.slot));
+    ring.next();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t h0, m0, l0, h1, m1, l1;
+      split3(b0[i].x, b0[i].y, h0, m0, l0);
+      split3(b1[i].x, b1[i].y, h1, m1, l1);
+      mma16816(ah, a[i][0], a[i][1], a[i][2], a[i][3], h0, h1);
+      mma16816(am, a[i][0], a[i][1], a[i][2], a[i][3], m0, m1);
+      mma16816(al, a[i][0], a[i][1], a[i][2], a[i][3], l0, l1);
+    }
+  }
+  part_w[g8 * 8 + 2 * q] = ah[0] + (am[0] + al[0]);
+  part_w[g8 * 8 + 2 * q + 1] = ah[1] + (am[1] + al[1]);
+  part_w[(g8 + 8) * 8 + 2 * q] = ah[2] + (am[2] + al[2]);
+  part_w[(g8 + 8) * 8 + 2 * q + 1] = ah[3] + (am[3] + al[3]);
+}
+
 // Generic skinny GEMV tile: n_mat matrices x R rows x (KCH*64) columns
-// against the <=8 activation columns in `act` ([kstep][B][4][16 B] fp32
-// fragment layout).  Leaves the result in scratch res[m][row][n] (floats).
-__device__ __noinline__ uint32_t gemv_tile(const Params& p, const int32_t* ent, const uint8_t* act,
-                                           int colsel, float* res, uint32_t stage_ctr) {
+// against up to 8 activation columns.  `act` holds the activation as fp32
+// rows of `stride` floats; output column n reads row colrow(n) (the slot's
+// token list for expert gate/up, else n); columns >= ncols read row 0 and
+// are ignored by the epilogues.  Leaves res[(m*R + row)*8 + n] in scratch.
+__device__ __forceinline__ uint32_t gemv_tile(const Params& p, const int32_t* ent, const float* act,
+                                           int stride, const int32_t* tokmap, int ncols,
+                                           float* res, uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int nstage = ent[32 + R_NSTAGE];
   const int nm = ent[D_NMAT], R = ent[D_R];
   const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
   const int kl = cw / MTn;
-  const int g8 = lane >> 2, q = lane & 3;
-  const int B = p.B;
-  // three independent accumulators (hi, mid, lo terms) keep the mma chains
-  // short; all smem reads of a stage are issued before the stage is released
-  float ah[4] = {0.f, 0.f, 0.f, 0.f}, am[4] = {0.f, 0.f, 0.f, 0.f},
-        al[4] = {0.f, 0.f, 0.f, 0.f};
-  // A-operand row/chunk of this lane inside a 16x64 unit (128B-swizzled)
-  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int achunk_hi = lane >> 4;
-  const uint32_t aoff = arow * 128;
-  const uint8_t* bbase = act + ((size_t)(colsel < 0 ? 0 : colsel) * 4 + q) * 16;
-  const size_t bstride = (size_t)B * 64;   // bytes per k-step
-  for (int s = 0; s < nstage; ++s) {
-    const uint32_t slot = stage_ctr % sm.NS;
-    const uint32_t ph = (stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm.full(slot), ph, 400);
-    __syncwarp();
-    const uint32_t ubase = saddr(sm.ring + (size_t)slot * kStageBytes + cw * kUnitBytes);
-    const int kc = s * kcps + kl;
-    uint32_t a[4][4];
-    float4 bv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int chunk = 2 * i + achunk_hi;
-      ldsm_x4(ubase + aoff + ((chunk ^ (arow & 7)) << 4), a[i][0], a[i][1], a[i][2], a[i][3]);
-      bv[i] = colsel >= 0 ? *reinterpret_cast<const float4*>(bbase + (size_t)(kc * 4 + i) * bstride)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(slot));
-    ++stage_ctr;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t h0, m0, l0, h1, m1, l1;
-      split3(bv[i].x, bv[i].y, h0, m0, l0);
-      split3(bv[i].z, bv[i].w, h1, m1, l1);
-      mma16816(ah, a[i][0], a[i][1], a[i][2], a[i][3], h0, h1);
-      mma16816(am, a[i][0], a[i][1], a[i][2], a[i][3], m0, m1);
-      mma16816(al, a[i][0], a[i][1], a[i][2], a[i][3], l0, l1);
-    }
-  }
-  float acc[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) acc[j] = ah[j] + (am[j] + al[j]);
-  // cross-warp reduction over the column chunks that shared a row tile
+  Ring ring;
+  ring.init(stage_ctr, sm.NS);
   float* part = reinterpret_cast<float*>(sm.scratch);  // [8][16][8]
   float* pw = part + cw * 128;
-  pw[g8 * 8 + 2 * q] = acc[0];
-  pw[g8 * 8 + 2 * q + 1] = acc[1];
-  pw[(g8 + 8) * 8 + 2 * q] = acc[2];
-  pw[(g8 + 8) * 8 + 2 * q + 1] = acc[3];
+  const uint32_t xbase = saddr(act);
+  auto row_of = [&](int n) { return n < ncols ? (tokmap ? tokmap[n] : n) : 0; };
+  uint32_t waitcyc = 0;
+  if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K2);
+  const uint64_t l0 = clock64();
+  if (p.B == 1) {
+    gemv_stages_ffma<1>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4, 0, ring, pw,
+                        waitcyc);
+  } else if (p.B == 2) {
+    gemv_stages_ffma<2>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4,
+                        xbase + row_of(1) * stride * 4, ring, pw, waitcyc);
+  } else {
+    gemv_stages_mma(p, sm, nstage, kcps, kl, xbase + row_of(lane >> 2) * stride * 4, ring, pw,
+                    waitcyc);
+  }
+  if (ct == 0) {
+    trace_put(p, ent[32 + R_TASK], T_C_LOOPCYC, (uint32_t)(clock64() - l0));
+    trace_put(p, ent[32 + R_TASK], T_C_WAITCYC, waitcyc);
+    cstamp(p, ent[32 + R_TASK], T_K3);
+  }
+  stage_ctr += (uint32_t)nstage;
+  // cross-warp reduction over the column chunks that shared a row tile
   cbar();
   const int nout = nm * R * 8;
   for (int idx = ct; idx < nout; idx += 256) {
@@ -705,30 +888,28 @@ __device__ __noinline__ uint32_t gemv_tile(const Params& p, const int32_t* ent, 
     res[idx] = v;  // res[(m*R + row)*8 + n]
   }
   cbar();
-  if (ct == 0) stamp(p, ent[32 + R_TASK], T_C_MATH);
+  if (ct == 0) {
+    stamp(p, ent[32 + R_TASK], T_C_MATH);
+    cstamp(p, ent[32 + R_TASK], T_K4);
+  }
   return stage_ctr;
 }
 
 // Write the normalized attention output o[G][hd] (smem) of token b, group g:
 // fp32 copy and the O-proj B-operand fragments.
-__device__ __noinline__ void write_attn_out(const Params& p, int layer, int b, int g,
+__device__ __forceinline__ void write_attn_out(const Params& p, int layer, int b, int g,
                                            const float* o) {
   MK_CONSUMER_IDS;
   const int G = p.G, hd = p.hd, B = p.B;
   float* dst = p.attn_o + ((size_t)layer * B + b) * (size_t)p.Hq * hd + (size_t)g * G * hd;
   for (int idx = ct; idx < G * hd; idx += 256) dst[idx] = o[idx];
-  uint8_t* fr = p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes;
-  const int nent = (G * hd / 16) * 4;
-  for (int t = ct; t < nent; t += 256) {
-    const int ks = t >> 2, q = t & 3;
-    const float* v = o + ks * 16 + 2 * q;
-    *reinterpret_cast<uint4*>(fr + (((size_t)ks * B + b) * 4 + q) * 16) =
-        frag_entry(v[0], v[1], v[8], v[9]);
-  }
+  float* row = reinterpret_cast<float*>(p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes) +
+               (size_t)b * (G * hd + kActPad);
+  for (int idx = ct; idx < G * hd; idx += 256) row[idx] = o[idx];
 }
 
 template <int HD>
-__device__ __noinline__ uint32_t attn_task(const Params& p, const int32_t* ent, const uint8_t* act,
+__device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* ent, const uint8_t* act,
                                            uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
@@ -856,8 +1037,8 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const int32_t* ent, 
     mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
     const float m_new = fmaxf(m_run, mx);
-    const float alpha = exp2f(m_run - m_new);
-    const float e0 = exp2f(s0 - m_new), e1 = exp2f(s1 - m_new);
+    const float alpha = ex2(m_run - m_new);
+    const float e0 = ex2(s0 - m_new), e1 = ex2(s1 - m_new);
     float ps = e0 + e1;
     ps += __shfl_xor_sync(FULL, ps, 1);
     ps += __shfl_xor_sync(FULL, ps, 2);
@@ -932,12 +1113,12 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const int32_t* ent, 
     float Lsum = 0.f, O = 0.f;
     for (int w = 0; w < 8; ++w) {
       const float* mwp = mrg + (w * G + h) * (HD + 4);
-      const float sc = exp2f(mwp[HD] - M);
+      const float sc = ex2(mwp[HD] - M);
       Lsum += sc * mwp[HD + 1];
       O += sc * mwp[i];
     }
     if (single) {
-      osm[idx] = O / Lsum;
+      osm[idx] = O * frcp(Lsum);
     } else {
       part[2 * G + idx] = O;
       if (i == 0) {
@@ -955,7 +1136,7 @@ __device__ __noinline__ uint32_t attn_task(const Params& p, const int32_t* ent, 
 
 // Log-sum-exp merge of the chunk partials of (token b, KV group g).  Every
 // load is issued in parallel across the CTA (no per-chunk dependency chain).
-__device__ __noinline__ void combine_task(const Params& p, const int32_t* ent) {
+__device__ __forceinline__ void combine_task(const Params& p, const int32_t* ent) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], nc = ent[D_D];
@@ -979,15 +1160,15 @@ __device__ __noinline__ void combine_task(const Params& p, const int32_t* ent) {
     for (int ch = lane; ch < nc; ch += 32) M = fmaxf(M, msm[ch * G + h]);
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
     float Ls = 0.f;
-    for (int ch = lane; ch < nc; ch += 32) Ls += exp2f(msm[ch * G + h] - M) * lsm[ch * G + h];
+    for (int ch = lane; ch < nc; ch += 32) Ls += ex2(msm[ch * G + h] - M) * lsm[ch * G + h];
     for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(FULL, Ls, o);
     if (lane == 0) {
       ML[h] = M;
-      ML[G + h] = 1.0f / Ls;
+      ML[G + h] = frcp(Ls);
     }
   }
   cbar();
-  for (int t = ct; t < nc * G; t += 256) wsm[t] = exp2f(msm[t] - ML[t % G]) * ML[G + t % G];
+  for (int t = ct; t < nc * G; t += 256) wsm[t] = ex2(msm[t] - ML[t % G]) * ML[G + t % G];
   cbar();
   for (int idx = ct; idx < G * hd; idx += 256) {
     const int h = idx / hd;
@@ -1009,92 +1190,89 @@ __device__ __noinline__ void combine_task(const Params& p, const int32_t* ent) {
   write_attn_out(p, layer, b, g, osm);
 }
 
-// fused residual add + RMSNorm statistics for one 64-row tile of level l:
-// x_l = x_{l-1} + sum_g o_part[g] + sum_j moe_part[j] (fixed order), the
-// gamma-scaled fragments the next projections read, and the tile's sum of
-// squares (the norm's 1/rms is applied in the consumers' epilogues).
-__device__ __noinline__ void rn_task(const Params& p, const int32_t* ent) {
-  const Smem sm = smem_view(p);
+// RoPE cos/sin of this step's positions (angle in double: a 262144-token
+// position loses ~0.03 rad in fp32), plus the position check.  Runs once per
+// step, out of line.
+__device__ __noinline__ void rope_table(const Params& p, int task) {
   MK_CONSUMER_IDS;
-  const int l = ent[D_LAYER], r = ent[D_A];
-  const int B = p.B, d = p.d;
-  float* xs = reinterpret_cast<float*>(sm.scratch);  // [B][64] gamma * x
-  const int b = cw;
-  const int col = r * 64 + 2 * lane;
-  if (b < B) {
-    float2 x;
-    if (l == 0) {
-      int tok = __ldg(p.tokens + b);
-      if (tok < 0 || tok >= p.V) {
-        if (lane == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
-        tok = 0;
-      }
-      const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(p.embed + (size_t)tok * d + col));
-      x = make_float2(__uint_as_float(pr << 16), __uint_as_float(pr & 0xffff0000u));
-    } else {
-      // all partial loads in flight at once, then a fixed-order sum
-      constexpr int kMaxParts = 1 + 16 + kMaxTopK;
-      const int nparts = 1 + p.Hkv + p.k;
-      const size_t o = (size_t)b * d + col;
-      float2 v[kMaxParts];
-#pragma unroll
-      for (int t = 0; t < kMaxParts; ++t) {
-        const float* src;
-        if (t == 0)
-          src = p.x + (size_t)(l - 1) * B * d;
-        else if (t <= p.Hkv)
-          src = p.o_part + ((size_t)(l - 1) * p.Hkv + (t - 1)) * B * d;
-        else
-          src = p.moe_part + ((size_t)(l - 1) * p.k + (t - 1 - p.Hkv)) * B * d;
-        v[t] = t < nparts ? __ldcg(reinterpret_cast<const float2*>(src + o))
-                          : make_float2(0.f, 0.f);
-      }
-      x = v[0];
-#pragma unroll
-      for (int t = 1; t < kMaxParts; ++t) {
-        if (t < nparts) {
-          x.x += v[t].x;
-          x.y += v[t].y;
-        }
-      }
-    }
-    *reinterpret_cast<float2*>(p.x + ((size_t)l * B + b) * d + col) = x;
-    const uint16_t* gam = (l < p.L) ? p.attn_norm[l] : p.final_norm;
-    const uint32_t gp = __ldg(reinterpret_cast<const uint32_t*>(gam + col));
-    xs[b * 64 + 2 * lane] = x.x * __uint_as_float(gp << 16);
-    xs[b * 64 + 2 * lane + 1] = x.y * __uint_as_float(gp & 0xffff0000u);
-    float ss = x.x * x.x + x.y * x.y;
-    for (int o2 = 16; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(FULL, ss, o2);
-    if (lane == 0) {
-      float* ssd = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_frag_bytes);
-      ssd[r * B + b] = ss;
-    }
-  }
-  cbar();
-  uint8_t* fr = p.actA + (size_t)l * p.actA_bytes;
-  for (int t = ct; t < 16 * B; t += 256) {
-    const int ksl = t / (4 * B), n = (t >> 2) % B, q = t & 3;
-    const float* v = xs + n * 64 + ksl * 16 + 2 * q;
-    *reinterpret_cast<uint4*>(fr + (((size_t)(4 * r + ksl) * B + n) * 4 + q) * 16) =
-        frag_entry(v[0], v[1], v[8], v[9]);
-  }
-  if (l == 0 && r == 0) {
-    const int half = p.hd / 2;
-    for (int t = ct; t < B * half; t += 256) {
-      const int bb = t / half, i = t % half;
-      const int pos = __ldg(p.positions + bb);
-      const int sl = __ldg(p.seq_lens + bb);
-      if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, pos, sl, 5);
-      double sv, cv;
-      sincos((double)pos * p.inv_freq[i], &sv, &cv);
-      p.cs[(size_t)bb * p.hd + i] = (float)cv;
-      p.cs[(size_t)bb * p.hd + half + i] = (float)sv;
-    }
+  const int half = p.hd / 2;
+  for (int t = ct; t < p.B * half; t += 256) {
+    const int bb = t / half, i = t % half;
+    const int pos = __ldg(p.positions + bb);
+    const int sl = __ldg(p.seq_lens + bb);
+    if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, task, OP_RN, -1, pos, sl, 5);
+    double sv, cv;
+    sincos((double)pos * p.inv_freq[i], &sv, &cv);
+    p.cs[(size_t)bb * p.hd + i] = (float)cv;
+    p.cs[(size_t)bb * p.hd + half + i] = (float)sv;
   }
 }
 
+// Fused residual add + RMSNorm statistics for one 64-column tile of level l:
+// x_l = x_{l-1} + sum_g o_part[g] + sum_j moe_part[j] (fixed order), the
+// gamma-scaled rows the next projections read, and the tile's sum of squares
+// per token (1/rms is applied in the consumers' epilogues).  The partials are
+// staged through shared memory in rounds so that all loads of a round are in
+// flight at once.
+__device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
+  const Smem sm = smem_view(p);
+  MK_CONSUMER_IDS;
+  const int l = ent[D_LAYER], r = ent[D_A];
+  const int B = p.B, d = p.d, per = B * 64;
+  float* xs = reinterpret_cast<float*>(sm.scratch);  // [B][64]
+  float* stage = xs + kMaxBatch * 64;                 // [kRnStage] staged partials
+  const int nparts = (l == 0) ? 1 : 1 + p.Hkv + p.k;
+  const int per_round = kRnStage / per;
+  for (int j0 = 0; j0 < nparts; j0 += per_round) {
+    const int nj = min(per_round, nparts - j0);
+#pragma unroll 4
+    for (int t = ct; t < nj * per; t += 256) {
+      const int j = j0 + t / per, e = t % per, b = e >> 6, col = r * 64 + (e & 63);
+      float v;
+      if (l == 0) {
+        int tok = __ldg(p.tokens + b);
+        if (tok < 0 || tok >= p.V) {
+          if ((e & 63) == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
+          tok = 0;
+        }
+        v = __uint_as_float((uint32_t)__ldg(p.embed + (size_t)tok * d + col) << 16);
+      } else {
+        const float* src =
+            j == 0 ? p.x + (size_t)(l - 1) * B * d
+            : j <= p.Hkv ? p.o_part + ((size_t)(l - 1) * p.Hkv + (j - 1)) * B * d
+                         : p.moe_part + ((size_t)(l - 1) * p.k + (j - 1 - p.Hkv)) * B * d;
+        v = __ldcg(src + (size_t)b * d + col);
+      }
+      stage[t] = v;
+    }
+    cbar();
+    for (int e = ct; e < per; e += 256) {
+      float x = j0 == 0 ? 0.f : xs[e];
+      for (int j = 0; j < nj; ++j) x += stage[j * per + e];
+      xs[e] = x;
+    }
+    cbar();
+  }
+  float* rows = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes);
+  const uint16_t* gam = (l < p.L) ? p.attn_norm[l] : p.final_norm;
+  for (int e = ct; e < per; e += 256) {
+    const int b = e >> 6, col = r * 64 + (e & 63);
+    const float x = xs[e];
+    p.x[((size_t)l * B + b) * d + col] = x;
+    rows[(size_t)b * (d + kActPad) + col] = x * __uint_as_float((uint32_t)__ldg(gam + col) << 16);
+  }
+  if (cw < B) {
+    const float x0 = xs[cw * 64 + lane], x1 = xs[cw * 64 + 32 + lane];
+    float ss = x0 * x0 + x1 * x1;
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
+    if (lane == 0)
+      reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_rows_bytes)[r * B + cw] = ss;
+  }
+  if (l == 0 && r == 0) rope_table(p, ent[32 + R_TASK]);
+}
+
 // top-k (logit desc, index asc) + softmax over the selected + slot compaction
-__device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
+__device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int l = ent[D_LAYER];
@@ -1144,11 +1322,11 @@ __device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
     if (lane == 0) {
       float ws[8], sum = 0.f;
       for (int j = 0; j < K; ++j) {
-        ws[j] = expf(selv[j] - selv[0]);
+        ws[j] = fexp(selv[j] - selv[0]);
         sum += ws[j];
       }
       for (int j = 0; j < K; ++j) {
-        const float w = ws[j] / sum;
+        const float w = ws[j] * frcp(sum);
         wsel[b * 8 + j] = w;
         rt[route_topk_idx(B, K) + b * K + j] = sel[b * 8 + j];
         reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + j] = w;
@@ -1214,7 +1392,10 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
       break;
     }
     const int t = ent[32 + R_TASK];
-    if (ct == 0) stamp(p, t, T_C_READY);
+    if (ct == 0) {
+      stamp(p, t, T_C_READY);
+      cstamp(p, t, T_K0);
+    }
     const int act = ent[D_ACT];
     if (act == ACT_A && ent[D_LAYER] != curA) {
       // a new level: the previous level's buffer is free (its tasks are done)
@@ -1229,11 +1410,14 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
       wait_bar(p, sm.afullB(bufB), (uint32_t)((nloadB >> 1) & 1), 502);
       ++nloadB;
     }
-    if (ct == 0) stamp(p, t, T_C_ACT);
+    if (ct == 0) {
+      stamp(p, t, T_C_ACT);
+      cstamp(p, t, T_K1);
+    }
     const uint8_t* actA = sm.actA + (size_t)bufA * p.actA_stride;
     const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
     const int layer = ent[D_LAYER];
-    const int n = lane >> 2;
+
     switch (op) {
       case OP_RN:
         rn_task(p, ent);
@@ -1250,95 +1434,86 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
         else
           stage_ctr = attn_task<64>(p, ent, actB, stage_ctr);
         break;
-      case OP_QKV:
-      case OP_ROUTER:
-      case OP_LMHEAD: {
-        level_rstd(p, actA, rstd);
-        stage_ctr = gemv_tile(p, ent, actA, n < p.B ? n : -1, res, stage_ctr);
+      default: {
+        // projection tiles: one tile routine, then the operation's epilogue
+        const float* act;
+        int stride, ncols = p.B;
+        const int32_t* tokmap = nullptr;
+        const bool expert = (op == OP_GATEUP || op == OP_DOWN);
+        if (expert) {
+          ncols = ent[32 + R_NTOK];
+          if (ent[32 + R_EXPERT] < 0) break;   // empty slot: nothing streamed
+        }
+        if (op == OP_OPROJ) {
+          act = reinterpret_cast<const float*>(actB);
+          stride = p.G * p.hd + kActPad;
+        } else if (op == OP_DOWN) {
+          act = reinterpret_cast<const float*>(actB);
+          stride = p.F + kActPad;
+        } else {
+          act = reinterpret_cast<const float*>(actA);
+          stride = p.d + kActPad;
+          if (op == OP_GATEUP) tokmap = ent + 32 + R_TOK;
+          level_rstd(p, actA, rstd);
+        }
+        stage_ctr = gemv_tile(p, ent, act, stride, tokmap, ncols, res, stage_ctr);
+        const int layer = ent[D_LAYER];
         const int R = ent[D_R], row0 = ent[D_ROW0];
-        for (int idx = ct; idx < R * 8; idx += 256) {
-          const int nn = idx / R, r = idx % R;  // r fastest: coalesced rows
-          if (nn >= p.B) continue;
-          const float v = res[r * 8 + nn] * rstd[nn];
-          const int row = row0 + r;
-          if (op == OP_QKV) {
-            p.qkv[((size_t)layer * p.B + nn) * p.qkvR + row] = v;
-          } else if (op == OP_ROUTER) {
-            if (row < p.E) {
-              const float* bias = p.router_bias[layer];
-              p.rlogits[((size_t)layer * p.B + nn) * p.E + row] = v + (bias ? bias[row] : 0.f);
+        if (op == OP_QKV || op == OP_ROUTER || op == OP_LMHEAD) {
+          for (int idx = ct; idx < R * 8; idx += 256) {
+            const int nn = idx / R, r = idx % R;  // r fastest: coalesced rows
+            if (nn >= p.B) continue;
+            const float v = res[r * 8 + nn] * rstd[nn];
+            const int row = row0 + r;
+            if (op == OP_QKV) {
+              p.qkv[((size_t)layer * p.B + nn) * p.qkvR + row] = v;
+            } else if (op == OP_ROUTER) {
+              if (row < p.E) {
+                const float* bias = p.router_bias[layer];
+                p.rlogits[((size_t)layer * p.B + nn) * p.E + row] = v + (bias ? bias[row] : 0.f);
+              }
+            } else if (row < p.V) {
+              p.logits[(size_t)nn * p.V + row] = v;
             }
-          } else {
-            if (row < p.V) p.logits[(size_t)nn * p.V + row] = v;
           }
-        }
-        break;
-      }
-      case OP_OPROJ: {
-        stage_ctr = gemv_tile(p, ent, actB, n < p.B ? n : -1, res, stage_ctr);
-        const int g = ent[D_B], row0 = ent[D_ROW0];
-        for (int idx = ct; idx < 64 * 8; idx += 256) {
-          const int nn = idx / 64, r = idx % 64;
-          if (nn >= p.B) continue;
-          p.o_part[(((size_t)layer * p.Hkv + g) * p.B + nn) * p.d + row0 + r] = res[r * 8 + nn];
-        }
-        break;
-      }
-      case OP_GATEUP: {
-        const int ntok = ent[32 + R_NTOK];
-        if (ent[32 + R_EXPERT] < 0) break;
-        const int col = n < ntok ? ent[32 + R_TOK + n] : -1;
-        level_rstd(p, actA, rstd);
-        stage_ctr = gemv_tile(p, ent, actA, col, res, stage_ctr);
-        const int R = ent[D_R], f = ent[D_B], j = ent[D_A];
-        float* asm_ = res + 2 * R * 8;  // [R][8] activations
-        for (int idx = ct; idx < R * 8; idx += 256) {
-          const int nn = idx / R, r = idx % R;
-          float a = 0.f;
-          if (nn < ntok) {
+        } else if (op == OP_OPROJ) {
+          const int g = ent[D_B];
+          for (int idx = ct; idx < 64 * 8; idx += 256) {
+            const int nn = idx / 64, r = idx % 64;
+            if (nn >= p.B) continue;
+            p.o_part[(((size_t)layer * p.Hkv + g) * p.B + nn) * p.d + row0 + r] = res[r * 8 + nn];
+          }
+        } else if (op == OP_GATEUP) {
+          const int f = ent[D_B], j = ent[D_A];
+          float* arow = reinterpret_cast<float*>(p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes);
+          for (int idx = ct; idx < R * 8; idx += 256) {
+            const int nn = idx / R, r = idx % R;
+            if (nn >= ncols) continue;
             const float rs = rstd[ent[32 + R_TOK + nn]];
             const float gt = res[r * 8 + nn] * rs;
             const float ut = res[(R + r) * 8 + nn] * rs;
-            a = gt / (1.0f + expf(-gt)) * ut;
+            const float a = gt * frcp(1.0f + fexp(-gt)) * ut;
             p.expert_a[(((size_t)layer * p.S + j) * p.B + nn) * p.F + f * R + r] = a;
+            arow[(size_t)nn * (p.F + kActPad) + f * R + r] = a;
           }
-          asm_[r * 8 + nn] = a;
-        }
-        cbar();
-        uint8_t* fr = p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes;
-        const int nent = (R / 16) * ntok * 4;
-        for (int t = ct; t < nent; t += 256) {
-          const int ksl = t / (4 * ntok), nn = (t >> 2) % ntok, q = t & 3;
-          const int r0 = ksl * 16 + 2 * q;
-          const uint4 fe = frag_entry(asm_[r0 * 8 + nn], asm_[(r0 + 1) * 8 + nn],
-                                      asm_[(r0 + 8) * 8 + nn], asm_[(r0 + 9) * 8 + nn]);
-          const int ks = f * (R / 16) + ksl;
-          *reinterpret_cast<uint4*>(fr + (((size_t)ks * p.B + nn) * 4 + q) * 16) = fe;
+        } else {  // OP_DOWN
+          for (int idx = ct; idx < 64 * 8; idx += 256) {
+            const int nn = idx / 64, r = idx % 64;
+            if (nn >= ncols) continue;
+            const int tok = ent[32 + R_TOK + nn];
+            const int rank = ent[32 + R_RANK + nn];
+            const float w = __int_as_float(ent[32 + R_W + nn]);
+            p.moe_part[(((size_t)layer * p.k + rank) * p.B + tok) * p.d + row0 + r] =
+                w * res[r * 8 + nn];
+          }
         }
         break;
       }
-      case OP_DOWN: {
-        const int ntok = ent[32 + R_NTOK];
-        if (ent[32 + R_EXPERT] < 0) break;
-        stage_ctr = gemv_tile(p, ent, actB, n < ntok ? n : -1, res, stage_ctr);
-        const int row0 = ent[D_ROW0];
-        for (int idx = ct; idx < 64 * 8; idx += 256) {
-          const int nn = idx / 64, r = idx % 64;
-          if (nn >= ntok) continue;
-          const int tok = ent[32 + R_TOK + nn];
-          const int rank = ent[32 + R_RANK + nn];
-          const float w = __int_as_float(ent[32 + R_W + nn]);
-          p.moe_part[(((size_t)layer * p.k + rank) * p.B + tok) * p.d + row0 + r] =
-              w * res[r * 8 + nn];
-        }
-        break;
-      }
-      default:
-        break;
     }
     cbar();
     if (ct == 0) {
       stamp(p, t, T_C_END);
+      cstamp(p, t, T_K5);
       if (act == ACT_B) mbar_arrive(sm.aemptyB(bufB));
       mbar_arrive(sm.done(e));
     }

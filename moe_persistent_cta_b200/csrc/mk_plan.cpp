@@ -88,14 +88,15 @@ static int round_up(int x, int a) { return (x + a - 1) / a * a; }
 int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   const int G = s.Hq / s.Hkv;
   const int NR = s.d / 64;
-  const int actA_bytes = 4 * s.d * B + round_up(NR * B * 4, 16);
+  const int actA_bytes = 4 * (s.d + kActPad) * B + round_up(NR * B * 4, 16);
   o->actA_stride = round_up(actA_bytes, 128);
-  int b_need = std::max(4 * G * s.hd * B, std::max(4 * s.F * B, (G + 3) * s.hd * 4));
+  int b_need = std::max(4 * (G * s.hd + kActPad) * B,
+                        std::max(4 * (s.F + kActPad) * B, (G + 3) * s.hd * 4));
   o->actB_bytes = round_up(b_need, 128);
   int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
   int sc_topk = B * s.E * 4 + B * 8 * 8 + s.E * 4 + 256;
-  int sc_rn = B * 64 * 4 + 64;
+  int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
   int sc_comb = 3 * max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
   o->scratch_bytes = round_up(sc, 1024);

@@ -107,7 +107,7 @@ class Decoder:
         mk.check_status(mk.lib.mk_set_trace(self._ctx, int(bool(enable))), "mk_set_trace")
 
     def trace(self):
-        """(desc [n_tasks][32], trace [n_tasks][9]) of the last traced step."""
+        """(desc [n_tasks][32], trace [n_tasks][18]) of the last traced step."""
         desc = self.debug(mk.MK_BUF_PLAN).reshape(-1, 32)
         stamps = self.debug(mk.MK_BUF_TRACE).reshape(-1, mk.TRACE_WORDS)
         return desc, stamps

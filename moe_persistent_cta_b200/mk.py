@@ -19,7 +19,7 @@ MK_ERR_CAPACITY, MK_ERR_STATE, MK_ERR_DEVICE = 5, 6, 7
 MK_BUF_X, MK_BUF_QKV, MK_BUF_ATTN_O, MK_BUF_RLOGITS, MK_BUF_TOPK = 0, 1, 2, 3, 4
 MK_BUF_NSLOTS, MK_BUF_EXPERT_A, MK_BUF_MOE, MK_BUF_OPART = 5, 6, 7, 8
 MK_BUF_TRACE, MK_BUF_PLAN = 9, 10
-TRACE_WORDS = 9
+TRACE_WORDS = 18
 
 # every entry point the header declares (checked by the ABI test)
 EXPORTS = (

@@ -19,7 +19,8 @@ OP_NAMES = {1: "rn", 2: "qkv", 3: "router", 4: "topk", 5: "attn", 6: "combine", 
             8: "gateup", 9: "down", 10: "lmhead"}
 D_OP, D_LAYER, D_A, D_B = 0, 1, 2, 3
 (T_P_RESOLVED, T_P_ISSUED, T_L_DEPS, T_L_ACT, T_C_READY, T_C_ACT, T_C_MATH,
- T_C_END, T_CTA) = range(9)
+ T_C_END, T_CTA, T_C_WAITCYC, T_C_LOOPCYC, T_P_WAITCYC, T_K0, T_K1, T_K2, T_K3, T_K4,
+ T_K5) = range(18)
 
 
 def _times(stamps: np.ndarray) -> np.ndarray:
@@ -48,6 +49,11 @@ def summarize(desc, stamps) -> Dict:
             d["math"].append(s[T_C_MATH] - s[T_C_ACT])
             d["epilogue"].append(s[T_C_END] - s[T_C_MATH])
         d["deps_before_pickup"].append(s[T_C_READY] - s[T_L_DEPS])
+        if stamps.shape[1] > T_P_WAITCYC and stamps[i, T_C_LOOPCYC]:
+            ghz = 1.965e3   # cycles per us at the max SM clock
+            d["loop_us"].append(stamps[i, T_C_LOOPCYC] / ghz)
+            d["stage_wait_us"].append(stamps[i, T_C_WAITCYC] / ghz)
+            d["producer_wait_us"].append(stamps[i, T_P_WAITCYC] / ghz)
         d["issued_before_pickup"].append(s[T_C_READY] - s[T_P_ISSUED])
     out = {"step_us": float(np.nanmax(t[:, T_C_END])), "ops": {}}
     for op, d in per_op.items():
