@@ -204,6 +204,9 @@ def main():
     ap.add_argument("--workload", default="moe30b_b1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-layers", type=int, default=2)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="cut the workload's model to this many layers (small cases for "
+                         "hardware-counter captures; not a full-size measurement)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -213,7 +216,9 @@ def main():
     import torch
     from moe_persistent_cta_b200 import configs, synth
 
-    wl = configs.WORKLOADS[args.workload]
+    wl = dict(configs.WORKLOADS[args.workload])
+    if args.layers > 0:
+        wl["shape"] = dict(wl["shape"], n_layers=args.layers)
     shape = wl["shape"]
     B = wl["batch"]
     lens = synth.seq_lengths(wl["seq_lens"], B)

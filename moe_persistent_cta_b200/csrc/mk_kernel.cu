@@ -577,7 +577,17 @@ __device__ __noinline__ void loader_loop(const Params& p) {
     }
     if (!ok) break;
     if (lane == 0) stamp(p, t, T_L_DEPS);
+    bool is_ready = false;
     if (act == ACT_A && layer != curA) {
+      // The consumer frees the previous level's buffer when it picks up the
+      // first task of the new level, so that task is marked ready before the
+      // buffer is waited for (with a single buffer the two would otherwise
+      // wait on each other); the consumer then waits for afullA.
+      if (lane == 0) {
+        stamp(p, t, T_L_ACT);
+        mbar_arrive(sm.ready(e));
+      }
+      is_ready = true;
       const int buf = nloadA % nA;
       if (!warp_wait(p, sm.aemptyA(buf), (uint32_t)(((nloadA / nA) & 1) ^ 1), 201)) break;
       ++nloadA;
@@ -624,7 +634,7 @@ __device__ __noinline__ void loader_loop(const Params& p) {
       }
       __syncwarp();
     }
-    if (lane == 0) {
+    if (lane == 0 && !is_ready) {
       stamp(p, t, T_L_ACT);
       mbar_arrive(sm.ready(e));
     }

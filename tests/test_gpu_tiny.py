@@ -107,6 +107,24 @@ def test_ragged_batch(lens, shuffled):
         rig.close()
 
 
+def test_wide_model_batch8_single_activation_buffer():
+    """d_model 2048 at batch 8 leaves room for one activation-A buffer only:
+    the first task of each new layer must still be picked up (it frees the
+    buffer) before its activation is loaded."""
+    shape = dict(configs.TINY, d_model=2048, n_q_heads=16, n_kv_heads=4, head_dim=128,
+                 d_ff=768, n_experts=16, top_k=4)
+    lens = [3, 64, 65, 130, 200, 17, 90, 127]
+    rig = TinyRig(shape, lens, seed=5)
+    try:
+        got = rig.step()
+        ref = rig.oracle_step()
+        err, rel = compare_logits(got, ref)
+        assert err <= TIGHT and rel <= REL_L2, (err, rel)
+        assert list(np.argmax(got, axis=1)) == list(np.argmax(ref, axis=1))
+    finally:
+        rig.close()
+
+
 def test_zipf_routing_batch8():
     lens = [100, 200, 300, 400, 500, 600, 700, 800]
     rig = TinyRig(configs.TINY, lens, seed=5, routing="zipf")
