@@ -154,6 +154,41 @@ mk_status mk_decode_step_unfused(mk_ctx* ctx, const int32_t* tokens,
                                  const int32_t* positions, const int32_t* page_table,
                                  const int32_t* seq_lens, float* logits, void* stream);
 
+/* Capacity of the fixed scratch array used by mk_decode_step_static. */
+#define MK_STATIC_SCRATCH_MAX_BYTES (32u * 1024u * 1024u)
+
+/* The same fused step as mk_decode_step, for callers that must not allocate
+ * device memory while they run: for example a serving process whose own
+ * memory pool has already reserved the device's free memory, or code that
+ * runs where an allocation's implicit device synchronization would stall
+ * other streams.  The pages describe no such entry point; it is an addition
+ * of this library.
+ *
+ * The step's scratch (counters, routing words, activations, attention and
+ * expert partials) lives in one file-scope device array of
+ * MK_STATIC_SCRATCH_MAX_BYTES (32 MiB) instead of the context's buffers;
+ * the array is reserved on every device that loads the library until the
+ * process exits.  The call itself allocates nothing.  The context (from
+ * mk_create and mk_build_schedule, which do allocate) supplies the schedule,
+ * tensor maps and status word; arguments and device inputs are those of
+ * mk_decode_step.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call, from every context, shares the one array and leaves its
+ *    contents in place; each call clears the counters and routing words on
+ *    `stream` before the launch.  Calls that overlap on the GPU (other
+ *    streams, other contexts on the same device) race on the array: order
+ *    them on one stream.
+ *  - Returns MK_ERR_CAPACITY, before any launch, when the current schedule
+ *    needs more than MK_STATIC_SCRATCH_MAX_BYTES (the 30B-MoE shape fits at
+ *    batch 1, not at batch 8); MK_ERR_STATE before any schedule was built.
+ *  - It records no trace and does not update the buffers mk_debug_read
+ *    returns; device errors surface through mk_check as usual.             */
+mk_status mk_decode_step_static(mk_ctx* ctx, const int32_t* tokens, const int32_t* positions,
+                                const int32_t* page_table, const int32_t* seq_lens,
+                                float* logits, void* stream);
+
 /* Synchronize the context's last stream and read the device status word.
  * device_status (may be NULL) receives MK_OK or the latched device error;
  * detail (may be NULL) receives int32[8]: {code, cta, task, opcode, counter,

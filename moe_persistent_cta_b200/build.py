@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(REPO_DIR, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libmk.so")
 
-SOURCES = ["mk_kernel.cu", "mk_host.cpp", "mk_plan.cpp"]
+SOURCES = ["mk_kernel.cu", "mk_host.cpp", "mk_plan.cpp", "mk_static.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

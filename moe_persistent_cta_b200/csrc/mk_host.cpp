@@ -588,3 +588,90 @@ mk_status mk_debug_read(mk_ctx* c, int which, void* dst, size_t bytes) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Step with caller-supplied scratch (used by the fixed-array entry point).
+namespace mk {
+
+int ctx_device(const mk_ctx* c) { return c ? c->device : -1; }
+
+namespace {
+// Carves the per-step buffers of the current schedule out of one region, in
+// a fixed order, each start rounded up to 256 bytes.  Returns the bytes used.
+size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* q = base ? base + off : nullptr;
+    off += (bytes + 255) & ~size_t(255);
+    return q;
+  };
+  const size_t L = b.L, B = b.B, d = b.d;
+  uint8_t* counters = take(sizeof(uint32_t) * (size_t)n_counters);
+  uint8_t* route = take((size_t)L * b.route_words * 4);
+  uint8_t* x = take((L + 1) * B * d * 4);
+  uint8_t* actA = take((L + 1) * (size_t)b.actA_bytes);
+  uint8_t* qkv = take(L * B * b.qkvR * 4);
+  uint8_t* cs = take(B * b.hd * 4);
+  uint8_t* attn_part = take(L * B * b.Hkv * b.max_chunks * b.part_stride * 4);
+  uint8_t* attn_o = take(L * B * b.Hq * b.hd * 4);
+  uint8_t* ofrag = take(L * b.Hkv * (size_t)b.ofrag_bytes);
+  uint8_t* o_part = take(L * b.Hkv * B * d * 4);
+  uint8_t* rlogits = take(L * B * b.E * 4);
+  uint8_t* expert_a = take(L * b.S * B * b.F * 4);
+  uint8_t* afrag = take(L * b.S * (size_t)b.afrag_bytes);
+  uint8_t* moe_part = take(L * b.k * B * d * 4);
+  if (p) {
+    p->counters = reinterpret_cast<uint32_t*>(counters);
+    p->route = reinterpret_cast<int32_t*>(route);
+    p->x = reinterpret_cast<float*>(x);
+    p->actA = actA;
+    p->qkv = reinterpret_cast<float*>(qkv);
+    p->cs = reinterpret_cast<float*>(cs);
+    p->attn_part = reinterpret_cast<float*>(attn_part);
+    p->attn_o = reinterpret_cast<float*>(attn_o);
+    p->ofrag = ofrag;
+    p->o_part = reinterpret_cast<float*>(o_part);
+    p->rlogits = reinterpret_cast<float*>(rlogits);
+    p->expert_a = reinterpret_cast<float*>(expert_a);
+    p->afrag = afrag;
+    p->moe_part = reinterpret_cast<float*>(moe_part);
+  }
+  return off;
+}
+}  // namespace
+
+// One fused step whose per-step buffers and counters live in `scratch`
+// (device memory of `cap` bytes) instead of the context's own.  Clears the
+// counters and routing words on the stream first, then runs at epoch 1.
+// The context's buffers, epoch and trace are left untouched.
+mk_status launch_step_in(mk_ctx* c, const int32_t* tokens, const int32_t* positions,
+                         const int32_t* page_table, const int32_t* seq_lens, float* logits,
+                         void* stream, void* scratch, size_t cap) {
+  if (!c) return MK_ERR_INVALID;
+  if (!c->have_schedule) return MK_ERR_STATE;
+  if (!tokens || !positions || !page_table || !seq_lens || !logits || !scratch)
+    return MK_ERR_INVALID;
+  const size_t need = carve_scratch(c->base, c->plan.n_counters, nullptr, nullptr);
+  if (need > cap) return MK_ERR_CAPACITY;
+  MK_CUDA(cudaSetDevice(c->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = c->base;
+  carve_scratch(c->base, c->plan.n_counters, static_cast<uint8_t*>(scratch), &p);
+  const size_t zero_bytes = reinterpret_cast<uint8_t*>(p.x) - static_cast<uint8_t*>(scratch);
+  MK_CUDA(cudaMemsetAsync(scratch, 0, zero_bytes, st));   // counters + routing words
+  p.tokens = tokens;
+  p.positions = positions;
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.logits = logits;
+  p.timeout_cycles = c->timeout_ns * 2ull;
+  p.epoch = 1;
+  p.trace = nullptr;
+  p.n_ctas = c->plan.n_ctas;
+  p.desc = static_cast<const int32_t*>(c->desc.ptr);
+  p.n_tasks = c->plan.n_tasks;
+  p.grab = c->plan.grab;
+  return from_cuda(mk::launch_interp(p, c->plan.n_ctas, st));
+}
+
+}  // namespace mk

@@ -19,11 +19,13 @@ MK_ERR_CAPACITY, MK_ERR_STATE, MK_ERR_DEVICE = 5, 6, 7
 MK_BUF_X, MK_BUF_QKV, MK_BUF_ATTN_O, MK_BUF_RLOGITS, MK_BUF_TOPK = 0, 1, 2, 3, 4
 MK_BUF_NSLOTS, MK_BUF_EXPERT_A, MK_BUF_MOE, MK_BUF_OPART = 5, 6, 7, 8
 MK_BUF_TRACE, MK_BUF_PLAN = 9, 10
+MK_STATIC_SCRATCH_MAX_BYTES = 32 * 1024 * 1024
 TRACE_WORDS = 18
 
 # every entry point the header declares (checked by the ABI test)
 EXPORTS = (
     "mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_step_unfused",
+    "mk_decode_step_static",
     "mk_check", "mk_set_timeout_ms", "mk_set_trace", "mk_debug_read", "mk_debug_size",
     "mk_plan_schedule", "mk_strerror", "mk_destroy",
 )
@@ -72,6 +74,7 @@ def _load():
         "mk_build_schedule": (c_int, [c_void_p, c_int, P(c_int32), P(c_int32), c_int32]),
         "mk_decode_step": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_decode_step_unfused": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
+        "mk_decode_step_static": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_check": (c_int, [c_void_p, P(c_int32), P(c_int32)]),
         "mk_set_timeout_ms": (c_int, [c_void_p, c_int32]),
         "mk_set_trace": (c_int, [c_void_p, c_int32]),

@@ -34,4 +34,6 @@ def test_strerror_and_argument_validation_without_gpu():
     assert mk.lib.mk_create(None, None, 0, None) == mk.MK_ERR_INVALID
     assert mk.lib.mk_check(None, None, None) == mk.MK_ERR_INVALID
     assert mk.lib.mk_decode_step(None, None, None, None, None, None, None) == mk.MK_ERR_INVALID
+    assert mk.lib.mk_decode_step_static(None, None, None, None, None, None,
+                                        None) == mk.MK_ERR_INVALID
     mk.lib.mk_destroy(None)
