@@ -5,7 +5,7 @@ contexts, 256K context, continuous batching) are the stand-ins for the pages'
 North Mini Code serving runs (agenticcommons.xyz, "Cohere North Mini Code
 megakernel serving engine", section "Why decode is slow": 30B total / a few B
 active parameters, BF16, 8K context, batch 1 to 8, up to 256K context).  All
-inputs are seeded and synthetic; see the design doc for the recipe.
+inputs are seeded and synthetic (generators in ``synth``).
 """
 
 from __future__ import annotations

@@ -20,7 +20,7 @@ Model (per token b, residual x in float64):
       x_{l+1} = x_l + Attn_l(n) + MoE_l(n)
   logits = W_lm . RMSNorm(x_L; gamma_final)
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * RMSNorm: h / sqrt(mean(h^2) + eps) * gamma, eps = 1e-6.
   * RoPE: rotate-half pairs (i, i + hd/2), angle = pos * theta^(-2i/hd).
   * Cached K is post-RoPE; the new token's K and V are rounded to bf16 before
