@@ -113,22 +113,25 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
-// 2D bf16 view [outer][inner], box {64, box_rows}, 128-byte swizzle: each
-// box row is one 128-byte line, matching the ldmatrix addressing of the
-// tile routines.
-mk_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                    uint32_t box_rows) {
+// 3D bf16 view of a row-major [rows][K] matrix as {64 columns, rows, K/64
+// column chunks} (strides K*2 and 128 bytes), box {64, box_rows, box_chunks},
+// 128-byte swizzle: one copy lands box_chunks consecutive 2 KB-per-16-rows
+// units ([chunk][row][128 B]), the layout the tile routines read, so a whole
+// ring stage of one matrix is a single TMA instruction.
+mk_status encode_3d(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows,
+                    uint32_t box_rows, uint32_t box_chunks) {
   auto fn = get_encoder();
   if (!fn) return MK_ERR_CUDA;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+  cuuint64_t dims[3] = {64, rows, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MK_OK : MK_ERR_INVALID;
 }
+
 
 int round_up(int x, int a) { return (x + a - 1) / a * a; }
 
@@ -222,21 +225,30 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
   for (int l = 0; l < L; ++l) {
     CUtensorMap* m = &maps[l * mk::kMapsPerLayer];
     mk_status st;
-    if ((st = encode_2d(m + 0, t->w_qkv[l], s.d, qkvR, c->r_qkv)) != MK_OK) return fail(st);
-    if ((st = encode_2d(m + 1, t->w_o[l], (uint64_t)s.Hq * s.hd, s.d, 64)) != MK_OK) return fail(st);
-    if ((st = encode_2d(m + 2, t->w_router[l], s.d, s.E, c->r_qkv)) != MK_OK) return fail(st);
-    if ((st = encode_2d(m + 3, t->w_gate[l], s.d, (uint64_t)s.E * s.F, c->r_ff)) != MK_OK)
+    // box chunks = the column chunks one 16 KB stage holds: 8 units of 16 rows
+    // shared by the tile's matrices and row tiles
+    const uint32_t ch_qkv = 128u / (uint32_t)c->r_qkv, ch_ff = 64u / (uint32_t)c->r_ff;
+    if ((st = encode_3d(m + 0, t->w_qkv[l], s.d, qkvR, c->r_qkv, ch_qkv)) != MK_OK)
       return fail(st);
-    if ((st = encode_2d(m + 4, t->w_up[l], s.d, (uint64_t)s.E * s.F, c->r_ff)) != MK_OK)
+    if ((st = encode_3d(m + 1, t->w_o[l], (uint64_t)s.Hq * s.hd, s.d, 64, 2)) != MK_OK)
       return fail(st);
-    if ((st = encode_2d(m + 5, t->w_down[l], s.F, (uint64_t)s.E * s.d, 64)) != MK_OK)
+    if ((st = encode_3d(m + 2, t->w_router[l], s.d, s.E, c->r_qkv, ch_qkv)) != MK_OK)
       return fail(st);
+    if ((st = encode_3d(m + 3, t->w_gate[l], s.d, (uint64_t)s.E * s.F, c->r_ff, ch_ff)) != MK_OK)
+      return fail(st);
+    if ((st = encode_3d(m + 4, t->w_up[l], s.d, (uint64_t)s.E * s.F, c->r_ff, ch_ff)) != MK_OK)
+      return fail(st);
+    if ((st = encode_3d(m + 5, t->w_down[l], s.F, (uint64_t)s.E * s.d, 64, 2)) != MK_OK)
+      return fail(st);
+    // K/V pools: one (page, head) block of 64 tokens x hd per copy
     const uint64_t kvrows = (uint64_t)s.n_pages * s.Hkv * mk::kPage;
-    if ((st = encode_2d(m + 6, t->k_pool[l], s.hd, kvrows, 64)) != MK_OK) return fail(st);
-    if ((st = encode_2d(m + 7, t->v_pool[l], s.hd, kvrows, 64)) != MK_OK) return fail(st);
+    if ((st = encode_3d(m + 6, t->k_pool[l], s.hd, kvrows, 64, s.hd / 64)) != MK_OK)
+      return fail(st);
+    if ((st = encode_3d(m + 7, t->v_pool[l], s.hd, kvrows, 64, s.hd / 64)) != MK_OK)
+      return fail(st);
   }
   {
-    mk_status st = encode_2d(&maps[L * mk::kMapsPerLayer], t->lm_head, s.d, s.V, 128);
+    mk_status st = encode_3d(&maps[L * mk::kMapsPerLayer], t->lm_head, s.d, s.V, 128, 1);
     if (st != MK_OK) return fail(st);
   }
   (void)G;
@@ -422,6 +434,8 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.off_actB = sl.off_actB;
   p.actB_bytes = sl.actB_bytes;
   p.off_ring = sl.off_ring;
+  p.off_epi = sl.off_epi;
+  p.part_cols = sl.part_cols;
   p.smem_bytes = sl.dyn_bytes;
 
   c->plan.release();

@@ -30,7 +30,11 @@ constexpr int kProducerWarp = 0;     // TMA weight/KV streamer + task resolver
 constexpr int kLoaderWarp = 1;       // dependency waits + activation loads
 constexpr int kSignalWarp = 2;       // completion signals (release adds)
 constexpr int kFirstConsumerWarp = 3;
-constexpr int kThreads = (kFirstConsumerWarp + kConsumerWarps) * 32;   // 352
+constexpr int kEpilogueWarp = kFirstConsumerWarp + kConsumerWarps;   // 11
+constexpr int kThreads = (kEpilogueWarp + 1) * 32;                    // 384
+constexpr int kRstdRing = 4;         // per-level 1/rms slots (levels in flight)
+constexpr int kTopkScratch = 2048;   // epilogue warp's top-k scratch (bytes)
+constexpr int kMaxParts = 1 + 16 + kMaxTopK;   // residual + O-proj groups + expert ranks
 constexpr int kFifo = 16;            // task entries in flight per CTA
 constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words
 constexpr int kMapsPerLayer = 8;     // qkv, o, router, gate, up, down, kpool, vpool
@@ -103,14 +107,20 @@ enum DescField : int {
                     // (slot A, reused while the level repeats), 2 small (slot B)
   D_PPC = 27,       // attention: pages per chunk
   D_PHASE = 28,     // operation phase (for the unfused launcher)
-  D_X0 = 29, D_X1 = 30, D_X2 = 31
+  D_X0 = 29, D_X1 = 30, D_X2 = 31   // last-arriver: arrival counter, arrivals, join signal
 };
 
 enum ActKind : int32_t { ACT_NONE = 0, ACT_A = 1, ACT_B = 2 };
 
 enum Flags : int32_t {
   F_LAST_CHUNK = 8,  // attention chunk that owns the new token (and appends it)
-  F_SINGLE = 16      // attention of (b, g) in one chunk: write the final output
+  F_SINGLE = 16,     // attention of (b, g) in one chunk: write the final output
+  // Last-arriver work: after its own outputs, the task adds 1 to counter
+  // D_X0 (D_X1 arrivals per step); the task that completes the count does the
+  // join below and then signals counter D_X2.
+  F_NORM = 32,       // O-proj / down tile: residual add + RMSNorm of its 64 columns
+  F_TOPK = 64,       // router tile: top-k, softmax and expert-slot compaction
+  F_COMBINE = 128    // attention chunk: log-sum-exp merge of the (b, g) chunks
 };
 
 // ------------------------------------------------- resolved entry words ---
@@ -183,6 +193,10 @@ struct Params {
   // shared-memory layout (byte offsets from the 1024-aligned base)
   int n_stages, nA, actA_stride;
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, actB_bytes, off_ring;
+  int off_epi;       // GEMV partials [2][kConsumerWarps][16][part_cols], then the
+                     // per-level 1/rms ring [kRstdRing][kMaxBatch], then the
+                     // epilogue warp's top-k scratch (kTopkScratch bytes)
+  int part_cols;     // token columns per partial row: B for B <= 2, else 8
   int smem_bytes;
 };
 
@@ -235,7 +249,8 @@ struct SmemLayout {
   int actB_bytes;     // bytes per small-activation buffer (two of them)
   int scratch_bytes;
   int n_stages;       // ring stages of kStageBytes
-  int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring;
+  int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring, off_epi;
+  int part_cols;
   int total;          // bytes from the 1024-aligned base
   int dyn_bytes;      // dynamic shared memory to request (total + alignment slack)
 };

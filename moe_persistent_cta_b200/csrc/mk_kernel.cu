@@ -74,6 +74,16 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 // L2 policy for streamed tensors (weights, cached K/V): evict first, so the
 // once-per-step stream does not push code, activations and counters out of L2.
+// 3D tiled copy {x, y, z} (the weight and KV views are {64 columns, rows,
+// 64-column chunks}).
+__device__ __forceinline__ void tma_3d(uint32_t dst, const void* map, int x, int y, int z,
+                                       uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -93,14 +103,6 @@ __device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void tma_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar,
-                                       uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
                                          uint32_t bar) {
   asm volatile(
@@ -116,6 +118,14 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(a), "r"(v)
+               : "memory");
+  return old;
 }
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -147,13 +157,16 @@ __device__ __forceinline__ void mma1688(float* c, uint32_t a0, uint32_t a1, uint
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(b0));
 }
-// named barrier among the 8 consumer warps only
+// Named barriers among the 8 consumer warps only: barrier 1 inside tile
+// routines, barrier 2 for the consumers' agreement on leaving the task loop
+// (every exit and every task with internal barriers passes through it, so
+// all consumer warps execute the same sequence of barrier-1 waits).
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ int cbar_or(int pred) {
   int r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+      "bar.red.or.pred q, 2, 256, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"(pred)
       : "memory");
@@ -213,6 +226,7 @@ struct Smem {
   uint8_t* scratch;
   uint8_t* actA;
   uint8_t* actB;
+  uint8_t* epi;
   int32_t* fifo;
   uint32_t bars;  // shared-window address of barrier 0
   int NS;
@@ -227,6 +241,8 @@ struct Smem {
   __device__ uint32_t aemptyA(int i) const { return bar(2 * NS + 4 * kFifo + 2 + i); }
   __device__ uint32_t afullB(int i) const { return bar(2 * NS + 4 * kFifo + 4 + i); }
   __device__ uint32_t aemptyB(int i) const { return bar(2 * NS + 4 * kFifo + 6 + i); }
+  __device__ uint32_t pfull(int i) const { return bar(2 * NS + 4 * kFifo + 8 + i); }
+  __device__ uint32_t pempty(int i) const { return bar(2 * NS + 4 * kFifo + 10 + i); }
 };
 
 __device__ __forceinline__ Smem smem_view(const Params& p) {
@@ -238,6 +254,7 @@ __device__ __forceinline__ Smem smem_view(const Params& p) {
   s.scratch = base + p.off_scratch;
   s.actA = base + p.off_actA;
   s.actB = base + p.off_actB;
+  s.epi = base + p.off_epi;
   s.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
   s.bars = raw + pad + (uint32_t)p.off_bars;
   s.NS = p.n_stages;
@@ -346,34 +363,61 @@ __device__ __forceinline__ const void* tmap(const Params& p, int idx) {
 }
 
 // ============================================================== producer ==
-// The producer takes the next task of the step's list from the dispenser
-// (an atomic add on a counter that advances by n_tasks + n_ctas per step),
-// posts it in the CTA's task FIFO, and streams its tiles.  A taken index past
-// the end posts a stop entry.
+// The producer takes tasks of the step's list from the dispenser (an atomic
+// add on a counter that advances by n_tasks + n_ctas per step), posts each in
+// the CTA's task FIFO, and streams its tiles.  A taken index past the end
+// posts a stop entry.  The next task is taken only once the current task's
+// last stage is issued: taking it earlier holds it on this CTA while other
+// CTAs could already run it, which measured slower.
+__device__ __forceinline__ void prefetch_tmap(const void* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
+}
+
 __device__ __noinline__ void producer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
-  uint32_t stage_ctr = 0;
   const int NS = sm.NS;
+  uint32_t slot = 0, phase = 0;   // ring position of the next stage
   const uint32_t base = (p.epoch - 1u) * (uint32_t)(p.n_tasks + p.n_ctas);
   const uint64_t pol = l2_evict_first();
+  auto valid = [&](int t) { return t >= 0 && t < p.n_tasks; };
+  int t_next = 0;
+  int32_t dw_next = 0;
+  auto take = [&]() {   // next task index and its descriptor (word `lane`)
+    uint32_t raw = 0;
+    if (lane == 0) raw = atomicAdd(p.counters + p.grab, 1u);
+    t_next = __shfl_sync(FULL, (int)(raw - base), 0);
+    dw_next = valid(t_next) ? __ldg(p.desc + (size_t)t_next * kDescWords + lane) : 0;
+  };
+  int pw_done_ctr = -1;          // producer wait already seen satisfied (this step)
+  uint32_t pw_done_tgt = 0;
+  auto ring_next = [&]() {
+    if (++slot == (uint32_t)NS) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  };
+  take();
   for (int i = 0;; ++i) {
     const int e = i % kFifo;
     if (!warp_wait(p, sm.fempty(e), ((i / kFifo) & 1) ^ 1, 100)) break;
-    int t = 0;
-    if (lane == 0) t = (int)(atomicAdd(p.counters + p.grab, 1u) - base);
-    t = __shfl_sync(FULL, t, 0);
+    const int t = t_next;
+    const int32_t dw = dw_next;
     int32_t* ent = sm.fifo + e * kFifoEntryWords;
-    if (t < 0 || t >= p.n_tasks) {
+    if (!valid(t)) {
       ent[D_OP] = OP_NONE;
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.posted(e));
       break;
     }
-    const int32_t dw = __ldg(p.desc + (size_t)t * kDescWords + lane);
     const int op = __shfl_sync(FULL, dw, D_OP);
     const int layer = __shfl_sync(FULL, dw, D_LAYER);
     int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
+    const int map0 = __shfl_sync(FULL, dw, D_MAP0), map1 = __shfl_sync(FULL, dw, D_MAP1);
+    if (lane == 0 && (nstage > 0 || op == OP_ATTN)) {
+      prefetch_tmap(tmap(p, map0));
+      if (op == OP_GATEUP || op == OP_ATTN) prefetch_tmap(tmap(p, map1));
+    }
     int32_t rw = 0;  // resolved word `lane`
     uint32_t pwait = 0;
     int expert = -1, ntok = 0, p0 = 0, seqlen = 0, phys_new = -1;
@@ -381,36 +425,41 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     if (op == OP_GATEUP || op == OP_DOWN) {
       const int ctr = __shfl_sync(FULL, dw, D_PW);
       const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
-      int ok = 1;
-      if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
-      ok = __shfl_sync(FULL, ok, 0);
-      if (!ok) break;
-      __syncwarp();
+      if (ctr != pw_done_ctr || tgt > pw_done_tgt) {
+        int ok = 1;
+        if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
+        ok = __shfl_sync(FULL, ok, 0);
+        if (!ok) break;
+        pw_done_ctr = ctr;
+        pw_done_tgt = tgt;
+      }
+      // every routing word of the slot in one round trip: lane R_EXPERT the
+      // expert, R_NTOK the token count, R_TOK/R_RANK/R_W + n token n's id,
+      // rank and weight (words past the count are read and then dropped)
       const int j = __shfl_sync(FULL, dw, D_A);
       const int32_t* rt = p.route + (size_t)layer * p.route_words;
       const int B = p.B, K = p.k, S = p.S;
-      expert = __ldcg(rt + route_slot_expert(B, K) + j);
-      ntok = __ldcg(rt + route_slot_ntok(B, K, S) + j);
-      if (expert < 0 || expert >= p.E || ntok < 0 || ntok > B) {
-        if (expert >= p.E || ntok < 0 || ntok > B) {
-          if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, expert, ntok, 1);
-          set_abort();
-          break;
-        }
+      int idx = -1;
+      if (lane == R_EXPERT) idx = route_slot_expert(B, K) + j;
+      else if (lane == R_NTOK) idx = route_slot_ntok(B, K, S) + j;
+      else if (lane >= R_TOK && lane < R_TOK + 8) idx = route_slot_tok(B, K, S) + j * 8 + lane - R_TOK;
+      else if (lane >= R_RANK && lane < R_RANK + 8)
+        idx = route_slot_rank(B, K, S) + j * 8 + lane - R_RANK;
+      else if (lane >= R_W && lane < R_W + 8) idx = route_slot_w(B, K, S) + j * 8 + lane - R_W;
+      const int32_t v = idx >= 0 ? __ldcg(rt + idx) : 0;
+      expert = __shfl_sync(FULL, v, R_EXPERT);
+      ntok = __shfl_sync(FULL, v, R_NTOK);
+      if (expert >= p.E || ntok < 0 || ntok > B) {
+        if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, expert, ntok, 1);
+        set_abort();
+        break;
+      }
+      if (expert < 0) {
         expert = -1;
         ntok = 0;
         nstage = 0;
       }
-      if (lane >= R_TOK && lane < R_TOK + 8) {
-        int t = lane - R_TOK;
-        rw = t < ntok ? __ldcg(rt + route_slot_tok(B, K, S) + j * 8 + t) : 0;
-      } else if (lane >= R_RANK && lane < R_RANK + 8) {
-        int t = lane - R_RANK;
-        rw = t < ntok ? __ldcg(rt + route_slot_rank(B, K, S) + j * 8 + t) : 0;
-      } else if (lane >= R_W && lane < R_W + 8) {
-        int t = lane - R_W;
-        rw = t < ntok ? __ldcg(rt + route_slot_w(B, K, S) + j * 8 + t) : 0;
-      }
+      if (lane >= R_TOK && lane < R_W + 8) rw = ((lane - R_TOK) & 7) < ntok ? v : 0;
     } else if (op == OP_ATTN) {
       const int b = __shfl_sync(FULL, dw, D_A);
       const int c = __shfl_sync(FULL, dw, D_C);
@@ -459,8 +508,8 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     if (op == OP_ATTN) {
       const int b = __shfl_sync(FULL, dw, D_A);
       const int g = __shfl_sync(FULL, dw, D_B);
-      const void* mk_ = tmap(p, __shfl_sync(FULL, dw, D_MAP0));
-      const void* mv_ = tmap(p, __shfl_sync(FULL, dw, D_MAP1));
+      const void* mk_ = tmap(p, map0);
+      const void* mv_ = tmap(p, map1);
       const int np = ntok;
       int pg = -1;
       const int* pt = p.page_table + (size_t)b * p.max_pages;
@@ -478,9 +527,7 @@ __device__ __noinline__ void producer_loop(const Params& p) {
         }
         if (fail) break;
         const int phys = __shfl_sync(FULL, pg, pi & 31);
-        const uint32_t slot = stage_ctr % NS;
-        const uint32_t ph = (stage_ctr / NS) & 1;
-        if (!warp_wait(p, sm.empty(slot), ph ^ 1, 101)) {
+        if (!warp_wait(p, sm.empty(slot), phase ^ 1, 101)) {
           fail = true;
           break;
         }
@@ -491,56 +538,58 @@ __device__ __noinline__ void producer_loop(const Params& p) {
           const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
           const int y = (phys * p.Hkv + g) * kPage;
           const void* m = (s & 1) ? mv_ : mk_;
-          for (int xb = 0; xb < p.hd / 64; ++xb) tma_2d(dst + xb * 8192, m, xb * 64, y, fb, pol);
+          tma_3d(dst, m, 0, y, 0, fb, pol);   // [hd/64 chunks][64 tokens][128 B]
         }
         __syncwarp();
-        ++stage_ctr;
+        ring_next();
       }
       if (fail) break;
     } else if (nstage > 0) {
       const int nm = __shfl_sync(FULL, dw, D_NMAT);
       const int R = __shfl_sync(FULL, dw, D_R);
-      const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
+      const int MT = R / 16, kcps = 8 / (nm * MT);
       const int k0 = __shfl_sync(FULL, dw, D_K0);
       int row0 = __shfl_sync(FULL, dw, D_ROW0);
       if (op == OP_GATEUP) row0 += expert * p.F;
       if (op == OP_DOWN) row0 += expert * p.d;
-      const void* m0 = tmap(p, __shfl_sync(FULL, dw, D_MAP0));
-      const void* m1 = nm > 1 ? tmap(p, __shfl_sync(FULL, dw, D_MAP1)) : m0;
+      const void* m0 = tmap(p, map0);
+      const void* m1 = nm > 1 ? tmap(p, map1) : m0;
       for (int s = 0; s < nstage; ++s) {
-        const uint32_t slot = stage_ctr % NS;
-        const uint32_t ph = (stage_ctr / NS) & 1;
         const uint64_t w0 = clock64();
-        if (!warp_wait(p, sm.empty(slot), ph ^ 1, 102)) {
+        if (!warp_wait(p, sm.empty(slot), phase ^ 1, 102)) {
           fail = true;
           break;
         }
         pwait += (uint32_t)(clock64() - w0);
         if (lane == 0) {
+          // one copy per matrix: kcps chunks x R rows, landing as units
+          // [matrix][chunk][row tile] of 16 rows x 64 columns
           const uint32_t fb = sm.full(slot);
           mbar_expect_tx(fb, kStageBytes);
           const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
-          for (int kl = 0; kl < kcps; ++kl) {
-            const int x = k0 + (s * kcps + kl) * 64;
-            tma_2d(dst + (kl * nm + 0) * MT * kUnitBytes, m0, x, row0, fb, pol);
-            if (nm > 1) tma_2d(dst + (kl * nm + 1) * MT * kUnitBytes, m1, x, row0, fb, pol);
-          }
+          const int z = k0 / 64 + s * kcps;
+          tma_3d(dst, m0, 0, row0, z, fb, pol);
+          if (nm > 1) tma_3d(dst + kcps * MT * kUnitBytes, m1, 0, row0, z, fb, pol);
         }
         __syncwarp();
-        ++stage_ctr;
+        ring_next();
       }
       if (fail) break;
     }
+    take();
     if (lane == 0) {
       stamp(p, t, T_P_ISSUED);
       trace_put(p, t, T_P_WAITCYC, pwait);
     }
   }
-  // drain: every fill issued must land before the CTA may exit (stage s was
-  // filled (stage_ctr - 1 - s) / NS + 1 times; wait for the last fill's phase)
-  for (int s = 0; s < NS; ++s)
-    if ((int)stage_ctr > s)
-      drain_bar(p, sm.full(s), (uint32_t)((((int)stage_ctr - 1 - s) / NS) & 1));
+  // drain: every fill issued must land before the CTA may exit.  A slot
+  // already filled in the current lap of the ring completes phase `phase`
+  // with its last fill, the others phase `phase ^ 1` (for a slot never
+  // filled that wait passes at once)
+  for (int s2 = 0; s2 < NS; ++s2) {
+    const uint32_t st2 = (uint32_t)s2 < slot ? phase : (phase ^ 1u);
+    drain_bar(p, sm.full(s2), st2);
+  }
 }
 
 // ================================================================ loader ==
@@ -569,12 +618,13 @@ __device__ __noinline__ void loader_loop(const Params& p) {
     const int act = __shfl_sync(FULL, dw, D_ACT);
     const int nwait = __shfl_sync(FULL, dw, D_NWAIT);
     int ok = 1;
-    for (int w = 0; w < nwait && ok; ++w) {
-      const int ctr = __shfl_sync(FULL, dw, D_W0 + 2 * w);
-      const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_W0N + 2 * w);
-      if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
-      ok = __shfl_sync(FULL, ok, 0);
+    // lane w polls the task's w-th counter: all counters in one round trip
+    if (lane < nwait) {
+      const int ctr = ent[D_W0 + 2 * lane];
+      const uint32_t tgt = p.epoch * (uint32_t)ent[D_W0N + 2 * lane];
+      ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
     }
+    ok = __all_sync(FULL, ok);
     if (!ok) break;
     if (lane == 0) stamp(p, t, T_L_DEPS);
     bool is_ready = false;
@@ -675,19 +725,6 @@ __device__ __noinline__ void signal_loop(const Params& p) {
   (void)cw;                                                    \
   (void)lane
 
-// rstd of each token from the level's sum-of-squares partials (slot A tail):
-// warp b reduces token b's partials into rstd_out[b].  Read after a barrier.
-__device__ __forceinline__ void level_rstd(const Params& p, const uint8_t* actA, float* rstd_out) {
-  MK_CONSUMER_IDS;
-  if (cw < p.B) {
-    const float* ss = reinterpret_cast<const float*>(actA + p.actA_rows_bytes);
-    float acc = 0.f;
-    for (int r = lane; r < p.NR; r += 32) acc += ss[r * p.B + cw];
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if (lane == 0) rstd_out[cw] = frsqrt(acc / (float)p.d + p.eps);
-  }
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -730,6 +767,7 @@ template <int NB>
 __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm, int nstage,
                                                  int kcps, int kl, uint32_t xaddr0,
                                                  uint32_t xaddr1, Ring& ring, float* part_w,
+                                                 uint32_t pe_bar, uint32_t pe_par,
                                                  uint32_t& waitcyc) {
   MK_CONSUMER_IDS;
   const int c = lane & 7, rg = lane >> 3;
@@ -793,8 +831,15 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
       a += __shfl_xor_sync(FULL, a, 1);
       a += __shfl_xor_sync(FULL, a, 2);
       a += __shfl_xor_sync(FULL, a, 4);
-      if (c == 0) part_w[(rg + 4 * i) * 8 + b] = a;
+      acc[i][b] = a;
     }
+  wait_bar(p, pe_bar, pe_par, 403);   // the epilogue warp has read this buffer's last use
+  if (c == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) part_w[(rg + 4 * i) * NB + b] = acc[i][b];
+  }
 }
 
 // Tensor-core stage loop for 3..8 activation columns: weights as the 16-row
@@ -803,7 +848,8 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
 // differences, ~24 bits), accumulated into three independent fp32 chains.
 __device__ __forceinline__ void gemv_stages_mma(const Params& p, const Smem& sm, int nstage,
                                                 int kcps, int kl, uint32_t xaddr, Ring& ring,
-                                                float* part_w, uint32_t& waitcyc) {
+                                                float* part_w, uint32_t pe_bar, uint32_t pe_par,
+                                                uint32_t& waitcyc) {
   MK_CONSUMER_IDS;
   const int g8 = lane >> 2, q = lane & 3;
   float ah[4] = {0.f, 0.f, 0.f, 0.f}, am[4] = {0.f, 0.f, 0.f, 0.f},
@@ -840,30 +886,33 @@ __device__ __forceinline__ void gemv_stages_mma(const Params& p, const Smem& sm,
       mma16816(al, a[i][0], a[i][1], a[i][2], a[i][3], l0, l1);
     }
   }
+  wait_bar(p, pe_bar, pe_par, 403);   // the epilogue warp has read this buffer's last use
   part_w[g8 * 8 + 2 * q] = ah[0] + (am[0] + al[0]);
   part_w[g8 * 8 + 2 * q + 1] = ah[1] + (am[1] + al[1]);
   part_w[(g8 + 8) * 8 + 2 * q] = ah[2] + (am[2] + al[2]);
   part_w[(g8 + 8) * 8 + 2 * q + 1] = ah[3] + (am[3] + al[3]);
 }
 
-// Generic skinny GEMV tile: n_mat matrices x R rows x (KCH*64) columns
-// against up to 8 activation columns.  `act` holds the activation as fp32
-// rows of `stride` floats; output column n reads row colrow(n) (the slot's
-// token list for expert gate/up, else n); columns >= ncols read row 0 and
-// are ignored by the epilogues.  Leaves res[(m*R + row)*8 + n] in scratch.
-__device__ __forceinline__ uint32_t gemv_tile(const Params& p, const int32_t* ent, const float* act,
-                                           int stride, const int32_t* tokmap, int ncols,
-                                           float* res, uint32_t stage_ctr) {
+// Generic skinny GEMV tile, consumer side: n_mat matrices x R rows x
+// (KCH*64) columns against up to 8 activation columns.  `act` holds the
+// activation as fp32 rows of `stride` floats; output column n reads row
+// colrow(n) (the slot's token list for expert gate/up, else n); columns >=
+// ncols read row 0 and are ignored by the epilogue.  Each warp streams its
+// own 16-row unit of every stage and leaves its partial sums in `pw`
+// ([16][part_cols]); the epilogue warp reduces the warps' partials.
+__device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t* ent,
+                                                 const float* act, int stride,
+                                                 const int32_t* tokmap, int ncols, float* pw,
+                                                 uint32_t pe_bar, uint32_t pe_par,
+                                                 uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int nstage = ent[32 + R_NSTAGE];
   const int nm = ent[D_NMAT], R = ent[D_R];
-  const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
-  const int kl = cw / MTn;
+  const int MT = R / 16, kcps = 8 / (nm * MT);
+  const int kl = (cw / MT) % kcps;   // unit cw = (matrix * kcps + chunk) * MT + row tile
   Ring ring;
   ring.init(stage_ctr, sm.NS);
-  float* part = reinterpret_cast<float*>(sm.scratch);  // [8][16][8]
-  float* pw = part + cw * 128;
   const uint32_t xbase = saddr(act);
   auto row_of = [&](int n) { return n < ncols ? (tokmap ? tokmap[n] : n) : 0; };
   uint32_t waitcyc = 0;
@@ -871,38 +920,90 @@ __device__ __forceinline__ uint32_t gemv_tile(const Params& p, const int32_t* en
   const uint64_t l0 = clock64();
   if (p.B == 1) {
     gemv_stages_ffma<1>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4, 0, ring, pw,
-                        waitcyc);
+                        pe_bar, pe_par, waitcyc);
   } else if (p.B == 2) {
     gemv_stages_ffma<2>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4,
-                        xbase + row_of(1) * stride * 4, ring, pw, waitcyc);
+                        xbase + row_of(1) * stride * 4, ring, pw, pe_bar, pe_par, waitcyc);
   } else {
     gemv_stages_mma(p, sm, nstage, kcps, kl, xbase + row_of(lane >> 2) * stride * 4, ring, pw,
-                    waitcyc);
+                    pe_bar, pe_par, waitcyc);
   }
   if (ct == 0) {
     trace_put(p, ent[32 + R_TASK], T_C_LOOPCYC, (uint32_t)(clock64() - l0));
     trace_put(p, ent[32 + R_TASK], T_C_WAITCYC, waitcyc);
     cstamp(p, ent[32 + R_TASK], T_K3);
-  }
-  stage_ctr += (uint32_t)nstage;
-  // cross-warp reduction over the column chunks that shared a row tile
-  cbar();
-  const int nout = nm * R * 8;
-  for (int idx = ct; idx < nout; idx += 256) {
-    const int n = idx & 7;
-    const int row = (idx >> 3) % R;
-    const int m = (idx >> 3) / R;
-    const int mt = row >> 4, r16 = row & 15;
-    float v = 0.f;
-    for (int k2 = 0; k2 < kcps; ++k2) v += part[(k2 * MTn + m * MT + mt) * 128 + r16 * 8 + n];
-    res[idx] = v;  // res[(m*R + row)*8 + n]
-  }
-  cbar();
-  if (ct == 0) {
     stamp(p, ent[32 + R_TASK], T_C_MATH);
-    cstamp(p, ent[32 + R_TASK], T_K4);
   }
-  return stage_ctr;
+  return stage_ctr + (uint32_t)nstage;
+}
+
+// GEMV tile, epilogue side (one warp): sums the consumer warps' partials
+// over the column chunks that shared a row tile, in chunk order, and writes
+// the operation's outputs.  `rs` is the level's 1/rms per token (A-input
+// operations).
+__device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* ent,
+                                              const float* part, const float* rs) {
+  const int lane = threadIdx.x & 31;
+  const int op = ent[D_OP], layer = ent[D_LAYER];
+  const int nm = ent[D_NMAT], R = ent[D_R], row0 = ent[D_ROW0];
+  const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
+  const int PC = p.part_cols;
+  const bool expert = (op == OP_GATEUP || op == OP_DOWN);
+  const int ncols = expert ? ent[32 + R_NTOK] : p.B;
+  if (expert && ent[32 + R_EXPERT] < 0) return;   // empty slot
+  const int n_out = R * ncols;
+  for (int idx = lane; idx < n_out; idx += 32) {
+    const int n = idx / R, r = idx - n * R;   // r fastest: coalesced output rows
+    const int mt = r >> 4, r16 = r & 15;
+    float s0 = 0.f, s1 = 0.f;
+    for (int kc = 0; kc < kcps; ++kc) {
+      s0 += part[((kc * MT + mt) * 16 + r16) * PC + n];
+      if (nm > 1) s1 += part[(((kcps + kc) * MT + mt) * 16 + r16) * PC + n];
+    }
+    const int row = row0 + r;
+    switch (op) {
+      case OP_QKV:
+        p.qkv[((size_t)layer * p.B + n) * p.qkvR + row] = s0 * rs[n];
+        break;
+      case OP_ROUTER:
+        if (row < p.E) {
+          const float* bias = p.router_bias[layer];
+          p.rlogits[((size_t)layer * p.B + n) * p.E + row] = s0 * rs[n] + (bias ? bias[row] : 0.f);
+        }
+        break;
+      case OP_LMHEAD:
+        if (row < p.V) p.logits[(size_t)n * p.V + row] = s0 * rs[n];
+        break;
+      case OP_OPROJ: {
+        const int g = ent[D_B];
+        p.o_part[(((size_t)layer * p.Hkv + g) * p.B + n) * p.d + row] = s0;
+        break;
+      }
+      case OP_GATEUP: {
+        const int f = ent[D_B], j = ent[D_A];
+        const float rt = rs[ent[32 + R_TOK + n]];
+        const float gt = s0 * rt, ut = s1 * rt;
+        const float a = gt * frcp(1.0f + fexp(-gt)) * ut;
+        p.expert_a[(((size_t)layer * p.S + j) * p.B + n) * p.F + f * R + r] = a;
+        float* arow =
+            reinterpret_cast<float*>(p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes);
+        arow[(size_t)n * (p.F + kActPad) + f * R + r] = a;
+        break;
+      }
+      default: {  // OP_DOWN
+        const int tok = ent[32 + R_TOK + n];
+        const int rank = ent[32 + R_RANK + n];
+        const float w = __int_as_float(ent[32 + R_W + n]);
+        p.moe_part[(((size_t)layer * p.k + rank) * p.B + tok) * p.d + row] = w * s0;
+        break;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool is_gemv(int op) {
+  return op == OP_QKV || op == OP_ROUTER || op == OP_OPROJ || op == OP_GATEUP ||
+         op == OP_DOWN || op == OP_LMHEAD;
 }
 
 // Write the normalized attention output o[G][hd] (smem) of token b, group g:
@@ -1282,6 +1383,7 @@ __device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
 }
 
 // top-k (logit desc, index asc) + softmax over the selected + slot compaction
+
 __device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
@@ -1386,34 +1488,56 @@ __device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
 __device__ __noinline__ void consumer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
-  uint32_t stage_ctr = 0;
+  uint32_t stage_ctr = 0, ngemv = 0;
   int curA = -1, nloadA = 0, nloadB = 0, bufA = 0;
   const int nA = p.nA;
-  float* res = reinterpret_cast<float*>(sm.scratch) + 8 * 128;  // after the partials
-  float* rstd = res + 1024;                                       // [8] per-token 1/rms
+  const int PC = p.part_cols;
+  float* part0 = reinterpret_cast<float*>(sm.epi);
+  float* rstd_ring = part0 + 2 * kConsumerWarps * 16 * PC;
   for (int i = 0;; ++i) {
     const int e = i % kFifo;
-    const bool ok = wait_bar(p, sm.ready(e), (i / kFifo) & 1, 500);
-    if (cbar_or(!ok || aborted())) break;
+    // Each warp runs the FIFO on its own through GEMV tiles (no barrier);
+    // leaving the loop, and entering a task with internal barriers, goes
+    // through one agreement among all consumer warps.
+    const bool ok = __all_sync(FULL, wait_bar(p, sm.ready(e), (i / kFifo) & 1, 500));
+    if (!ok) {
+      cbar_or(1);
+      break;
+    }
     const int32_t* ent = sm.fifo + e * kFifoEntryWords;
     const int op = ent[D_OP];
     if (op == OP_NONE) {
       if (ct == 0) mbar_arrive(sm.done(e));
+      cbar_or(1);
       break;
     }
+    const bool gemv = is_gemv(op);
+    if (!gemv && cbar_or(aborted())) break;
     const int t = ent[32 + R_TASK];
     if (ct == 0) {
       stamp(p, t, T_C_READY);
       cstamp(p, t, T_K0);
     }
     const int act = ent[D_ACT];
-    if (act == ACT_A && ent[D_LAYER] != curA) {
-      // a new level: the previous level's buffer is free (its tasks are done)
-      if (curA >= 0 && ct == 0) mbar_arrive(sm.aemptyA(bufA));
+    const int layer = ent[D_LAYER];
+    if (act == ACT_A && layer != curA) {
+      // a new level: this warp is done with the previous level's buffer
+      if (curA >= 0 && lane == 0) mbar_arrive(sm.aemptyA(bufA));
       bufA = nloadA % nA;
       wait_bar(p, sm.afullA(bufA), (uint32_t)((nloadA / nA) & 1), 501);
       ++nloadA;
-      curA = ent[D_LAYER];
+      curA = layer;
+      if (cw < p.B) {
+        // 1/rms of token cw from the level's sum-of-squares partials, once
+        // per level; the epilogue warp reads it after this warp's pfull
+        const float* ss = reinterpret_cast<const float*>(sm.actA + (size_t)bufA * p.actA_stride +
+                                                         p.actA_rows_bytes);
+        float acc = 0.f;
+        for (int r = lane; r < p.NR; r += 32) acc += ss[r * p.B + cw];
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+        if (lane == 0) rstd_ring[(layer & (kRstdRing - 1)) * kMaxBatch + cw] =
+            frsqrt(acc / (float)p.d + p.eps);
+      }
     }
     const int bufB = nloadB & 1;
     if (act == ACT_B) {
@@ -1426,7 +1550,40 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
     }
     const uint8_t* actA = sm.actA + (size_t)bufA * p.actA_stride;
     const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
-    const int layer = ent[D_LAYER];
+
+    if (gemv) {
+      const int pb = (int)(ngemv & 1u);
+      const uint32_t pe_par = ((ngemv >> 1) & 1u) ^ 1u;
+      float* pw = part0 + (pb * kConsumerWarps + cw) * 16 * PC;
+      const float* a;
+      int stride, ncols = p.B;
+      const int32_t* tokmap = nullptr;
+      bool skip = false;
+      if (op == OP_GATEUP || op == OP_DOWN) {
+        ncols = ent[32 + R_NTOK];
+        skip = ent[32 + R_EXPERT] < 0;   // empty slot: nothing streamed
+      }
+      if (op == OP_OPROJ) {
+        a = reinterpret_cast<const float*>(actB);
+        stride = p.G * p.hd + kActPad;
+      } else if (op == OP_DOWN) {
+        a = reinterpret_cast<const float*>(actB);
+        stride = p.F + kActPad;
+      } else {
+        a = reinterpret_cast<const float*>(actA);
+        stride = p.d + kActPad;
+        if (op == OP_GATEUP) tokmap = ent + 32 + R_TOK;
+      }
+      if (skip)
+        wait_bar(p, sm.pempty(pb), pe_par, 403);
+      else
+        stage_ctr = gemv_consume(p, ent, a, stride, tokmap, ncols, pw, sm.pempty(pb), pe_par,
+                                 stage_ctr);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pfull(pb));
+      ++ngemv;
+      continue;   // the epilogue warp completes the task
+    }
 
     switch (op) {
       case OP_RN:
@@ -1438,87 +1595,26 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
       case OP_COMBINE:
         combine_task(p, ent);
         break;
-      case OP_ATTN:
+      default:  // OP_ATTN
         if (p.hd == 128)
           stage_ctr = attn_task<128>(p, ent, actB, stage_ctr);
         else
           stage_ctr = attn_task<64>(p, ent, actB, stage_ctr);
-        break;
-      default: {
-        // projection tiles: one tile routine, then the operation's epilogue
-        const float* act;
-        int stride, ncols = p.B;
-        const int32_t* tokmap = nullptr;
-        const bool expert = (op == OP_GATEUP || op == OP_DOWN);
-        if (expert) {
-          ncols = ent[32 + R_NTOK];
-          if (ent[32 + R_EXPERT] < 0) break;   // empty slot: nothing streamed
-        }
-        if (op == OP_OPROJ) {
-          act = reinterpret_cast<const float*>(actB);
-          stride = p.G * p.hd + kActPad;
-        } else if (op == OP_DOWN) {
-          act = reinterpret_cast<const float*>(actB);
-          stride = p.F + kActPad;
-        } else {
-          act = reinterpret_cast<const float*>(actA);
-          stride = p.d + kActPad;
-          if (op == OP_GATEUP) tokmap = ent + 32 + R_TOK;
-          level_rstd(p, actA, rstd);
-        }
-        stage_ctr = gemv_tile(p, ent, act, stride, tokmap, ncols, res, stage_ctr);
-        const int layer = ent[D_LAYER];
-        const int R = ent[D_R], row0 = ent[D_ROW0];
-        if (op == OP_QKV || op == OP_ROUTER || op == OP_LMHEAD) {
-          for (int idx = ct; idx < R * 8; idx += 256) {
-            const int nn = idx / R, r = idx % R;  // r fastest: coalesced rows
-            if (nn >= p.B) continue;
-            const float v = res[r * 8 + nn] * rstd[nn];
-            const int row = row0 + r;
-            if (op == OP_QKV) {
-              p.qkv[((size_t)layer * p.B + nn) * p.qkvR + row] = v;
-            } else if (op == OP_ROUTER) {
-              if (row < p.E) {
-                const float* bias = p.router_bias[layer];
-                p.rlogits[((size_t)layer * p.B + nn) * p.E + row] = v + (bias ? bias[row] : 0.f);
-              }
-            } else if (row < p.V) {
-              p.logits[(size_t)nn * p.V + row] = v;
-            }
+        if (ent[D_FLAGS] & F_COMBINE) {
+          // the chunk that completes (b, g) merges all its chunks' partials
+          cbar();
+          int last = 0;
+          if (ct == 0) {
+            const uint32_t old = atom_add_acq_rel(p.counters + ent[D_X0], 1u);
+            last = old + 1u == p.epoch * (uint32_t)ent[D_X1];
           }
-        } else if (op == OP_OPROJ) {
-          const int g = ent[D_B];
-          for (int idx = ct; idx < 64 * 8; idx += 256) {
-            const int nn = idx / 64, r = idx % 64;
-            if (nn >= p.B) continue;
-            p.o_part[(((size_t)layer * p.Hkv + g) * p.B + nn) * p.d + row0 + r] = res[r * 8 + nn];
-          }
-        } else if (op == OP_GATEUP) {
-          const int f = ent[D_B], j = ent[D_A];
-          float* arow = reinterpret_cast<float*>(p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes);
-          for (int idx = ct; idx < R * 8; idx += 256) {
-            const int nn = idx / R, r = idx % R;
-            if (nn >= ncols) continue;
-            const float rs = rstd[ent[32 + R_TOK + nn]];
-            const float gt = res[r * 8 + nn] * rs;
-            const float ut = res[(R + r) * 8 + nn] * rs;
-            const float a = gt * frcp(1.0f + fexp(-gt)) * ut;
-            p.expert_a[(((size_t)layer * p.S + j) * p.B + nn) * p.F + f * R + r] = a;
-            arow[(size_t)nn * (p.F + kActPad) + f * R + r] = a;
-          }
-        } else {  // OP_DOWN
-          for (int idx = ct; idx < 64 * 8; idx += 256) {
-            const int nn = idx / 64, r = idx % 64;
-            if (nn >= ncols) continue;
-            const int tok = ent[32 + R_TOK + nn];
-            const int rank = ent[32 + R_RANK + nn];
-            const float w = __int_as_float(ent[32 + R_W + nn]);
-            p.moe_part[(((size_t)layer * p.k + rank) * p.B + tok) * p.d + row0 + r] =
-                w * res[r * 8 + nn];
+          if (cbar_or(last)) {
+            combine_task(p, ent);
+            cbar();
+            if (ct == 0) red_release_add(p.counters + ent[D_X2], 1u);
           }
         }
         break;
-      }
     }
     cbar();
     if (ct == 0) {
@@ -1527,7 +1623,264 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
       if (act == ACT_B) mbar_arrive(sm.aemptyB(bufB));
       mbar_arrive(sm.done(e));
     }
-    if (cbar_or(aborted())) break;
+  }
+}
+
+// ========================================================== last arriver ==
+// A group of tasks that feeds one join (the 64-column norm tile, the layer's
+// top-k, the (b, g) attention merge) counts its arrivals on a counter; the
+// task whose arrival completes this step's count does the join.  The arrival
+// is an acquire-release add by one thread after a barrier of the writers:
+// release publishes this task's outputs (the barrier orders the other
+// writers' stores before it), acquire makes the earlier arrivals' outputs
+// visible to the last one, which reads them through L2.
+__device__ __forceinline__ bool warp_arrive_last(const Params& p, int ctr, int arrivals) {
+  __syncwarp();
+  uint32_t old = 0;
+  if ((threadIdx.x & 31) == 0) old = atom_add_acq_rel(p.counters + ctr, 1u);
+  old = __shfl_sync(FULL, old, 0);
+  return old + 1u == p.epoch * (uint32_t)arrivals;
+}
+__device__ __forceinline__ void warp_signal(const Params& p, int ctr) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) red_release_add(p.counters + ctr, 1u);
+}
+__device__ __forceinline__ float4 ldcg4(const float* a) {
+  return __ldcg(reinterpret_cast<const float4*>(a));
+}
+
+// Residual add + RMSNorm statistics of the 64 columns [64 r, 64 r + 64) for
+// level lv >= 1, by one warp: x_lv = x_{lv-1} + the O-proj partials of every
+// KV group + the expert partials of every rank (in that order), written to x;
+// gamma * x into the level's activation rows; and per token the tile's sum of
+// squares, from which every reader of the level forms 1/rms.  Half-warp h
+// takes tokens h, h + 2, ...; lane q of a half its 4 columns.
+__device__ __noinline__ void fused_norm(const Params& p, int lv, int r) {
+  const int lane = threadIdx.x & 31;
+  const int B = p.B, d = p.d, Hkv = p.Hkv, K = p.k;
+  const int q = lane & 15, col = r * 64 + 4 * q;
+  const int l = lv - 1;
+  const uint16_t* gam = (lv < p.L) ? p.attn_norm[lv] : p.final_norm;
+  const uint2 gw = __ldg(reinterpret_cast<const uint2*>(gam + col));
+  const float g0 = lo_bf16(gw.x), g1 = hi_bf16(gw.x), g2 = lo_bf16(gw.y), g3 = hi_bf16(gw.y);
+  float* rows = reinterpret_cast<float*>(p.actA + (size_t)lv * p.actA_bytes);
+  float* ssp = reinterpret_cast<float*>(p.actA + (size_t)lv * p.actA_bytes + p.actA_rows_bytes);
+  const int nparts = 1 + Hkv + K;
+  for (int b0 = 0; b0 < B; b0 += 2) {
+    const int b = b0 + (lane >> 4);
+    float ss = 0.f;
+    if (b < B) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < nparts; j0 += 8) {   // 8 loads in flight per round
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          if (j < nparts) {
+            const float* src =
+                j == 0 ? p.x + (size_t)l * B * d
+                : j <= Hkv ? p.o_part + ((size_t)l * Hkv + (j - 1)) * B * d
+                           : p.moe_part + ((size_t)l * K + (j - 1 - Hkv)) * B * d;
+            v[u] = ldcg4(src + (size_t)b * d + col);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < nparts) {
+            x.x += v[u].x;
+            x.y += v[u].y;
+            x.z += v[u].z;
+            x.w += v[u].w;
+          }
+        }
+      }
+      *reinterpret_cast<float4*>(p.x + ((size_t)lv * B + b) * d + col) = x;
+      *reinterpret_cast<float4*>(rows + (size_t)b * (d + kActPad) + col) =
+          make_float4(x.x * g0, x.y * g1, x.z * g2, x.w * g3);
+      ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    }
+    for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);   // within the half
+    if (q == 0 && b < B) ssp[r * B + b] = ss;
+  }
+}
+
+// Top-k + softmax + expert-slot compaction of layer l (one warp), from the
+// router logits: per token the k largest logits by (value descending, expert
+// ascending), weights softmax over the selected logits; the experts any token
+// selected get slots in ascending expert order, each slot listing its tokens
+// (ascending) with their rank and weight; unused slots are marked empty.
+__device__ __noinline__ void fused_topk(const Params& p, int l) {
+  const Smem sm = smem_view(p);
+  const int lane = threadIdx.x & 31;
+  const int B = p.B, E = p.E, K = p.k, S = p.S;
+  int32_t* rt = p.route + (size_t)l * p.route_words;
+  int* sel = reinterpret_cast<int*>(sm.epi + 2 * kConsumerWarps * 16 * p.part_cols * 4 +
+                                    kRstdRing * kMaxBatch * 4);   // [8][8]
+  float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [8][8] logits, then weights
+  int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8);  // [256]
+  uint32_t used = 0u;   // lane w < 8: bit e of experts 32 w + e selected by any token
+  for (int b = 0; b < B; ++b) {
+    const float* lg = p.rlogits + ((size_t)l * B + b) * E;
+    uint32_t key[8];   // order-preserving unsigned keys; 0 marks taken / absent
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int e = lane + 32 * t;
+      uint32_t k = 0u;
+      if (e < E) {
+        const uint32_t u = __float_as_uint(__ldcg(lg + e));
+        k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      }
+      key[t] = k;
+    }
+#pragma unroll 1
+    for (int j = 0; j < K; ++j) {
+      uint32_t bk = 0u;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (key[t] > bk) {   // ascending e within a lane: first max has the smallest e
+          bk = key[t];
+          bi = lane + 32 * t;
+        }
+      }
+      const uint32_t mk = __reduce_max_sync(FULL, bk);
+      const int wi = __reduce_min_sync(FULL, bk == mk ? bi : 0x7fffffff);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (lane + 32 * t == wi) key[t] = 0u;
+      if (lane == (wi >> 5)) used |= 1u << (wi & 31);
+      if (lane == 0) {
+        sel[b * 8 + j] = wi;
+        wsel[b * 8 + j] = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      // softmax over the selected logits (in place)
+      const float m0 = wsel[b * 8];
+      float sum = 0.f;
+      for (int j = 0; j < K; ++j) {
+        const float w = fexp(wsel[b * 8 + j] - m0);
+        wsel[b * 8 + j] = w;
+        sum += w;
+      }
+      const float inv = frcp(sum);
+      for (int j = 0; j < K; ++j) {
+        const float w = wsel[b * 8 + j] * inv;
+        wsel[b * 8 + j] = w;
+        rt[route_topk_idx(B, K) + b * K + j] = sel[b * 8 + j];
+        reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + j] = w;
+      }
+    }
+    __syncwarp();
+  }
+  // slot of each used expert = number of used experts below it (every lane
+  // takes all 8 words first; the per-expert loop below only reads them)
+  uint32_t words[8];
+  int below[8], n_used = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    words[w] = __shfl_sync(FULL, used, w);
+    below[w] = n_used;
+    n_used += __popc(words[w]);
+  }
+  for (int e = lane; e < E; e += 32) {
+    const int w = e >> 5;
+    uint32_t word = 0u;
+    int bw = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) {
+      if (w2 == w) {
+        word = words[w2];
+        bw = below[w2];
+      }
+    }
+    const int cnt = bw + __popc(word & ((1u << (e & 31)) - 1u));
+    slot_of[e] = ((word >> (e & 31)) & 1u) ? cnt : -1;
+  }
+  for (int s2 = lane; s2 < S; s2 += 32) {
+    if (s2 >= n_used) {
+      rt[route_slot_expert(B, K) + s2] = -1;
+      rt[route_slot_ntok(B, K, S) + s2] = 0;
+    }
+  }
+  if (lane == 0) rt[0] = n_used;
+  __syncwarp();
+  // one (token, rank) pair per lane: its position in the slot's token list
+  for (int idx = lane; idx < B * K; idx += 32) {
+    const int bb = idx / K, j = idx % K;
+    const int e = sel[bb * 8 + j];
+    const int s2 = slot_of[e];
+    int pos = 0;
+    for (int b2 = 0; b2 < bb; ++b2)
+      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
+    rt[route_slot_tok(B, K, S) + s2 * 8 + pos] = bb;
+    rt[route_slot_rank(B, K, S) + s2 * 8 + pos] = j;
+    reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s2 * 8 + pos] = wsel[bb * 8 + j];
+    if (pos == 0) {
+      int cnt = 0;
+      for (int b2 = 0; b2 < B; ++b2)
+        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
+      rt[route_slot_expert(B, K) + s2] = e;
+      rt[route_slot_ntok(B, K, S) + s2] = cnt;
+    }
+  }
+}
+
+// ============================================================== epilogue ==
+// One warp follows the FIFO behind the consumers.  For a GEMV tile it waits
+// for the consumer warps' partials, reduces them, writes the outputs and
+// completes the task (partials buffer, B activation buffer, done); every
+// entry it passes is released to the producer together with the signaler.
+__device__ __noinline__ void epilogue_loop(const Params& p) {
+  const Smem sm = smem_view(p);
+  const int lane = threadIdx.x & 31;
+  const int PC = p.part_cols;
+  const float* part0 = reinterpret_cast<const float*>(sm.epi);
+  const float* rstd_ring = part0 + 2 * kConsumerWarps * 16 * PC;
+  uint32_t ngemv = 0;
+  int nloadB = 0;
+  for (int i = 0;; ++i) {
+    const int e = i % kFifo;
+    if (!warp_wait(p, sm.ready(e), (i / kFifo) & 1, 600)) break;
+    const int32_t* ent = sm.fifo + e * kFifoEntryWords;
+    const int op = ent[D_OP];
+    if (op == OP_NONE) break;
+    const int act = ent[D_ACT];
+    if (!is_gemv(op)) {
+      if (act == ACT_B) ++nloadB;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.fempty(e));
+      continue;
+    }
+    const int pb = (int)(ngemv & 1u);
+    if (!warp_wait(p, sm.pfull(pb), (ngemv >> 1) & 1u, 601)) break;
+    const int t = ent[32 + R_TASK];
+    if (lane == 0) cstamp(p, t, T_K4);
+    gemv_epilogue(p, ent, part0 + pb * kConsumerWarps * 16 * PC,
+                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch);
+    const int flags = ent[D_FLAGS];
+    if (flags & (F_NORM | F_TOPK)) {
+      if (warp_arrive_last(p, ent[D_X0], ent[D_X1])) {
+        if (flags & F_NORM)
+          fused_norm(p, ent[D_LAYER] + 1, op == OP_OPROJ ? ent[D_A] : ent[D_B]);
+        else
+          fused_topk(p, ent[D_LAYER]);
+        warp_signal(p, ent[D_X2]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      stamp(p, t, T_C_END);
+      cstamp(p, t, T_K5);
+      mbar_arrive(sm.pempty(pb));
+      if (act == ACT_B) mbar_arrive(sm.aemptyB(nloadB & 1));
+      mbar_arrive(sm.done(e));
+      mbar_arrive(sm.fempty(e));
+    }
+    __syncwarp();
+    if (act == ACT_B) ++nloadB;
+    ++ngemv;
   }
 }
 
@@ -1544,13 +1897,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
       mbar_init(sm.posted(e), 1);
       mbar_init(sm.ready(e), 1);
       mbar_init(sm.done(e), 1);
-      mbar_init(sm.fempty(e), 1);
+      mbar_init(sm.fempty(e), 2);   // signaler + epilogue warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sm.afullA(b), 1);
-      mbar_init(sm.aemptyA(b), 1);
+      mbar_init(sm.aemptyA(b), kConsumerWarps);
       mbar_init(sm.afullB(b), 1);
       mbar_init(sm.aemptyB(b), 1);
+      mbar_init(sm.pfull(b), kConsumerWarps);
+      mbar_init(sm.pempty(b), 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1562,6 +1917,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
     loader_loop(p);
   } else if (warp == kSignalWarp) {
     signal_loop(p);
+  } else if (warp == kEpilogueWarp) {
+    epilogue_loop(p);
   } else {
     consumer_loop(p);
   }

@@ -20,38 +20,63 @@ D_OP, D_LAYER, D_A, D_B, D_C, D_D, D_FLAGS, D_NWAIT = 0, 1, 2, 3, 4, 5, 6, 7
 D_W0, D_W0N, D_PW, D_PWN, D_NSIG, D_S0 = 8, 9, 12, 13, 14, 15
 D_NSTAGE, D_ROW0, D_K0, D_KCH, D_R, D_NMAT, D_ACT, D_PPC, D_PHASE = 17, 18, 19, 20, 21, 22, 25, 27, 28
 OP_RN, OP_QKV, OP_ROUTER, OP_TOPK, OP_ATTN, OP_COMBINE, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM = range(1, 11)
+NR_30B = 2048 // 64
 ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 
-def check_order_and_targets(desc, targets, n_ctas, grab):
-    """(a) waits only on earlier signallers, (b) targets == signaller counts;
-    then simulate a greedy dynamic execution on n_ctas CTAs."""
-    n = len(desc)
-    first_sig = {}
-    last_sig = {}
+D_X0, D_X1, D_X2 = 29, 30, 31
+F_NORM, F_TOPK, F_COMBINE = 32, 64, 128
+FUSED = F_NORM | F_TOPK | F_COMBINE
+
+
+def signal_sets(desc, targets):
+    """Per counter: (signals per step, tasks that may send them).  A task
+    signals each counter of its list once; the tasks of a last-arriver group
+    (same arrival counter D_X0) together signal their join counter D_X2 once,
+    and any of them may be the sender."""
     count = collections.Counter()
+    senders = collections.defaultdict(list)
+    groups = collections.defaultdict(list)
     for i, t in enumerate(desc):
         for s in range(t[D_NSIG]):
             c = int(t[D_S0 + s])
             count[c] += 1
-            first_sig.setdefault(c, i)
-            last_sig[c] = i
+            senders[c].append(i)
+        if t[D_FLAGS] & FUSED:
+            groups[int(t[D_X0])].append(i)
+    for a, members in groups.items():
+        arrivals = {int(desc[i][D_X1]) for i in members}
+        joins = {int(desc[i][D_X2]) for i in members}
+        assert arrivals == {len(members)}, f"arrival counter {a}: {len(members)} arrive, {arrivals}"
+        assert targets[a] == len(members)
+        assert len(joins) == 1
+        j = joins.pop()
+        count[j] += 1
+        senders[j].extend(members)
+    return count, senders
+
+
+def check_order_and_targets(desc, targets, n_ctas, grab):
+    """(a) waits only on earlier senders, (b) targets == signals per step;
+    then simulate a greedy dynamic execution on n_ctas CTAs."""
+    count, senders = signal_sets(desc, targets)
+    last_sig = {c: max(v) for c, v in senders.items()}
     for i, t in enumerate(desc):
         waits = [(int(t[D_W0 + 2 * w]), int(t[D_W0N + 2 * w])) for w in range(t[D_NWAIT])]
         if t[D_PW] >= 0:
             waits.append((int(t[D_PW]), int(t[D_PWN])))
         for c, need in waits:
-            assert count[c] == need, f"task {i}: counter {c} has {count[c]} signallers, waits {need}"
-            assert last_sig[c] < i, f"task {i} waits on counter {c} signalled later (task {last_sig[c]})"
+            assert count[c] == need, f"task {i}: counter {c} gets {count[c]} signals, waits {need}"
+            assert last_sig[c] < i, f"task {i} waits on counter {c} sent later (task {last_sig[c]})"
     for c, k in count.items():
         assert targets[c] == k
-    assert targets[grab] == n + n_ctas
-    # greedy dynamic execution: each CTA takes the next task when it has finished
-    # its previous one; a task finishes when its waits are met (unit time)
-    done_at = {}
-    ctr_done = collections.defaultdict(int)
-    ctr_time = collections.defaultdict(float)
+    assert targets[grab] == len(desc) + n_ctas
+    # greedy dynamic execution: each CTA takes the next task when it has
+    # finished its previous one; a task finishes when its waits are met
+    remaining = {c: len(v) for c, v in senders.items()}
+    done_time = collections.defaultdict(float)
     free = [0.0] * n_ctas
+    finish = 0.0
     for i, t in enumerate(desc):
         c = int(np.argmin(free))
         start = free[c]
@@ -59,15 +84,17 @@ def check_order_and_targets(desc, targets, n_ctas, grab):
         if t[D_PW] >= 0:
             waits.append(int(t[D_PW]))
         for w in waits:
-            assert ctr_done[w] == count[w]     # every signaller already taken earlier
-            start = max(start, ctr_time[w])
+            assert remaining[w] == 0      # every possible sender already taken earlier
+            start = max(start, done_time[w])
         free[c] = start + 1.0
-        for s in range(t[D_NSIG]):
-            w = int(t[D_S0 + s])
-            ctr_done[w] += 1
-            ctr_time[w] = max(ctr_time[w], free[c])
-        done_at[i] = free[c]
-    return max(done_at.values())
+        finish = max(finish, free[c])
+        sent = [int(t[D_S0 + s]) for s in range(t[D_NSIG])]
+        if t[D_FLAGS] & FUSED:
+            sent.append(int(t[D_X2]))
+        for w in sent:
+            remaining[w] -= 1
+            done_time[w] = max(done_time[w], free[c])
+    return finish
 
 
 @pytest.mark.parametrize("n_ctas,lens", [(148, [128]), (7, [128]), (3, [0]),
@@ -85,10 +112,26 @@ def test_30b_b1_plan_structure():
     ops = collections.Counter(desc[:, D_OP].tolist())
     L, d = shape["n_layers"], shape["d_model"]
     qkv_rows = (shape["n_q_heads"] + 2 * shape["n_kv_heads"]) * shape["head_dim"]
-    assert ops[OP_RN] == (L + 1) * d // 64
     assert ops[OP_QKV] == L * qkv_rows // 16
     assert ops[OP_ROUTER] == L * shape["n_experts"] // 16
-    assert ops[OP_TOPK] == L
+    # each join is done one way or the other, never both: as its own tasks,
+    # or by the last-arriving producer tile of its group
+    fl = desc[:, D_FLAGS]
+
+    def all_or_none(op, flag):
+        f = fl[desc[:, D_OP] == op] & flag
+        assert np.all(f) or not np.any(f)
+        return bool(np.all(f))
+
+    fused_norm = all_or_none(OP_OPROJ, F_NORM)
+    assert all_or_none(OP_DOWN, F_NORM) == fused_norm
+    assert ops[OP_RN] == (1 if fused_norm else L + 1) * d // 64
+    assert ops[OP_TOPK] == (0 if all_or_none(OP_ROUTER, F_TOPK) else L)
+    a_multi = desc[(desc[:, D_OP] == OP_ATTN) & (desc[:, D_D] > 1)]
+    assert len(a_multi)
+    fused_comb = bool(np.all(a_multi[:, D_FLAGS] & F_COMBINE))
+    assert fused_comb or not np.any(a_multi[:, D_FLAGS] & F_COMBINE)
+    assert ops[OP_COMBINE] == (0 if fused_comb else L * shape["n_kv_heads"])
     assert ops[OP_OPROJ] == L * shape["n_kv_heads"] * d // 64
     S = min(shape["n_experts"], shape["top_k"])
     assert ops[OP_GATEUP] == L * S * shape["d_ff"] // 16
@@ -100,13 +143,17 @@ def test_30b_b1_plan_structure():
     nc, ppc = a[0, D_D], a[0, D_PPC]
     assert nc * ppc * 64 >= 8192 + 64
     assert len(a) == L * shape["n_kv_heads"] * nc
-    # priority order inside a layer: gate/up ahead of the attention tail
-    lay = desc[desc[:, D_LAYER] == 3]
-    pos = {op: np.where(lay[:, D_OP] == op)[0] for op in (OP_GATEUP, OP_COMBINE, OP_OPROJ,
-                                                           OP_ROUTER, OP_QKV, OP_DOWN)}
-    assert pos[OP_ROUTER].max() < pos[OP_QKV].min()
-    assert pos[OP_GATEUP].max() < pos[OP_COMBINE].min() < pos[OP_OPROJ].min()
-    assert pos[OP_OPROJ].max() < pos[OP_DOWN].min()
+    # the dispensing order comes from a simulation, but each layer still ends
+    # with tiles feeding the next norm
+    for l in (0, 3, 47):
+        ops = desc[desc[:, D_LAYER] == l][:, D_OP]
+        assert ops[-1] in (OP_OPROJ, OP_DOWN)
+    # every task of a layer is dispensed before the next layer's first
+    # projection tile that reads its output
+    for l in range(shape["n_layers"] - 1):
+        last = np.where(desc[:, D_LAYER] == l)[0].max()
+        nxt = np.where((desc[:, D_LAYER] == l + 1) & (desc[:, D_OP] != OP_RN))[0].min()
+        assert last < nxt
 
 
 def test_30b_b8_plan():
