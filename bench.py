@@ -35,10 +35,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "c980422a520ec43c844025fb128db23c3bbbc6165a6fb25e3aca048292bfdbf0",
+    "kernel_sha256": "4ff998f5244ea6e29918bd4bb993839f0c616eb51046f9910f0bf3e07e122e2d",
     "workload": "moe30b_b1",
-    "fixed_bytes": 623.8e6,
-    "per_layer_bytes": 114.2e6,
+    "fixed_bytes": 623.96e6,
+    "per_layer_bytes": 114.28e6,
 }
 
 

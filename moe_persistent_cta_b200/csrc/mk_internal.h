@@ -33,7 +33,7 @@ constexpr int kFirstConsumerWarp = 3;
 constexpr int kEpilogueWarp = kFirstConsumerWarp + kConsumerWarps;   // 11
 constexpr int kThreads = (kEpilogueWarp + 1) * 32;                    // 384
 constexpr int kRstdRing = 4;         // per-level 1/rms slots (levels in flight)
-constexpr int kTopkScratch = 2048;   // epilogue warp's top-k scratch (bytes)
+constexpr int kTopkScratch = 2048;   // epilogue warp scratch: top-k join (1.5 KB), router bias (512 B)
 constexpr int kMaxParts = 1 + 16 + kMaxTopK;   // residual + O-proj groups + expert ranks
 constexpr int kFifo = 16;            // task entries in flight per CTA
 constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words

@@ -942,7 +942,8 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
 // the operation's outputs.  `rs` is the level's 1/rms per token (A-input
 // operations).
 __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* ent,
-                                              const float* part, const float* rs) {
+                                              const float* part, const float* rs,
+                                              const float* bias_s) {
   const int lane = threadIdx.x & 31;
   const int op = ent[D_OP], layer = ent[D_LAYER];
   const int nm = ent[D_NMAT], R = ent[D_R], row0 = ent[D_ROW0];
@@ -966,10 +967,7 @@ __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* en
         p.qkv[((size_t)layer * p.B + n) * p.qkvR + row] = s0 * rs[n];
         break;
       case OP_ROUTER:
-        if (row < p.E) {
-          const float* bias = p.router_bias[layer];
-          p.rlogits[((size_t)layer * p.B + n) * p.E + row] = s0 * rs[n] + (bias ? bias[row] : 0.f);
-        }
+        if (row < p.E) p.rlogits[((size_t)layer * p.B + n) * p.E + row] = s0 * rs[n] + bias_s[r];
         break;
       case OP_LMHEAD:
         if (row < p.V) p.logits[(size_t)n * p.V + row] = s0 * rs[n];
@@ -1838,6 +1836,10 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
   const int PC = p.part_cols;
   const float* part0 = reinterpret_cast<const float*>(sm.epi);
   const float* rstd_ring = part0 + 2 * kConsumerWarps * 16 * PC;
+  // router bias of the current tile: the tail of the warp's top-k scratch
+  // (the top-k join uses its first 1.5 KB)
+  float* bias_s = reinterpret_cast<float*>(sm.epi + 2 * kConsumerWarps * 16 * PC * 4 +
+                                           kRstdRing * kMaxBatch * 4 + 1536);
   uint32_t ngemv = 0;
   int nloadB = 0;
   for (int i = 0;; ++i) {
@@ -1854,11 +1856,20 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
       continue;
     }
     const int pb = (int)(ngemv & 1u);
+    if (op == OP_ROUTER) {
+      // the tile's bias values, staged while the consumers stream the tile
+      // (the pointer and the values are two dependent global loads)
+      const float* bias = p.router_bias ? p.router_bias[ent[D_LAYER]] : nullptr;
+      const int R = ent[D_R], row0 = ent[D_ROW0];
+      for (int r = lane; r < R; r += 32)
+        bias_s[r] = (bias && row0 + r < p.E) ? __ldg(bias + row0 + r) : 0.f;
+      __syncwarp();
+    }
     if (!warp_wait(p, sm.pfull(pb), (ngemv >> 1) & 1u, 601)) break;
     const int t = ent[32 + R_TASK];
     if (lane == 0) cstamp(p, t, T_K4);
     gemv_epilogue(p, ent, part0 + pb * kConsumerWarps * 16 * PC,
-                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch);
+                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch, bias_s);
     const int flags = ent[D_FLAGS];
     if (flags & (F_NORM | F_TOPK)) {
       if (warp_arrive_last(p, ent[D_X0], ent[D_X1])) {
