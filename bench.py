@@ -35,10 +35,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "4ff998f5244ea6e29918bd4bb993839f0c616eb51046f9910f0bf3e07e122e2d",
+    "kernel_sha256": "2cd0675218d225fe7199fa3249644841366d5c669aa9896630b1faa858f22f4a",
     "workload": "moe30b_b1",
-    "fixed_bytes": 623.96e6,
-    "per_layer_bytes": 114.28e6,
+    "fixed_bytes": 623.99e6,
+    "per_layer_bytes": 114.30e6,
 }
 
 

@@ -1332,27 +1332,30 @@ __device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
   float* stage = xs + kMaxBatch * 64;                 // [kRnStage] staged partials
   const int nparts = (l == 0) ? 1 : 1 + p.Hkv + p.k;
   const int per_round = kRnStage / per;
+  const int per4 = per / 4;   // float4 units (4 consecutive columns) per part
   for (int j0 = 0; j0 < nparts; j0 += per_round) {
     const int nj = min(per_round, nparts - j0);
+    // every load of the round is issued before any is used (one L2 round trip)
 #pragma unroll 4
-    for (int t = ct; t < nj * per; t += 256) {
-      const int j = j0 + t / per, e = t % per, b = e >> 6, col = r * 64 + (e & 63);
-      float v;
+    for (int t4 = ct; t4 < nj * per4; t4 += 256) {
+      const int j = j0 + t4 / per4, e4 = t4 % per4, b = e4 >> 4, col = r * 64 + 4 * (e4 & 15);
+      float4 v;
       if (l == 0) {
         int tok = __ldg(p.tokens + b);
         if (tok < 0 || tok >= p.V) {
-          if ((e & 63) == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
+          if ((e4 & 15) == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
           tok = 0;
         }
-        v = __uint_as_float((uint32_t)__ldg(p.embed + (size_t)tok * d + col) << 16);
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.embed + (size_t)tok * d + col));
+        v = make_float4(lo_bf16(w.x), hi_bf16(w.x), lo_bf16(w.y), hi_bf16(w.y));
       } else {
         const float* src =
             j == 0 ? p.x + (size_t)(l - 1) * B * d
             : j <= p.Hkv ? p.o_part + ((size_t)(l - 1) * p.Hkv + (j - 1)) * B * d
                          : p.moe_part + ((size_t)(l - 1) * p.k + (j - 1 - p.Hkv)) * B * d;
-        v = __ldcg(src + (size_t)b * d + col);
+        v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * d + col));
       }
-      stage[t] = v;
+      reinterpret_cast<float4*>(stage)[t4] = v;
     }
     cbar();
     for (int e = ct; e < per; e += 256) {
