@@ -19,8 +19,8 @@
  *    through a fused residual add + RMSNorm; per-KV-group O-proj and
  *    per-expert down-projection dependencies; weight prefetch before the
  *    activation dependency resolves).
- *  - aimodeling.com, "Cohere open-sources a megakernel inference engine":
- *    sections "One persistent kernel runs the whole decode step" and "From
+ *  - aimodeling.com, "Cohere megakernel engine: one CUDA file, 1.58x vLLM on H100":
+ *    sections "One persistent kernel for the whole decode step" and "From
  *    demo to a full serving system" (continuous batching, paged attention,
  *    ragged sequence lengths, at most 8 sequences, one calling convention).
  *
@@ -195,6 +195,20 @@ mk_status mk_decode_step_static(mk_ctx* ctx, const int32_t* tokens, const int32_
  * observed, target, aux}.  Returns MK_OK if the device status is clean, else
  * the device status.  Clears the latched status.                           */
 mk_status mk_check(mk_ctx* ctx, int32_t* device_status, int32_t* detail);
+
+/* Failure-detection self-test: runs the task interpreter on a one-task list
+ * whose only dependency is a counter that nothing signals, with a deadline
+ * of `timeout_ms` per device wait.  The wait runs out by design (no fault,
+ * no trap, no unbounded spin): the kernel latches MK_ERR_TIMEOUT in the
+ * status word, every CTA leaves its task loop, and this call synchronizes,
+ * reads and clears the status (device_status and detail as for mk_check).
+ * Returns MK_ERR_TIMEOUT when detection works, MK_ERR_STATE before any
+ * schedule was built.  Uses its own counters: the step's counters, epoch and
+ * outputs are untouched, and the next mk_decode_step runs normally.
+ * (The pages describe no failure handling; the bounded waits are this
+ * library's own.)                                                           */
+mk_status mk_selftest_timeout(mk_ctx* ctx, int32_t timeout_ms, int32_t* device_status,
+                              int32_t* detail);
 
 /* Record per-task timestamps in every following fused step (enable != 0),
  * readable with mk_debug_read(MK_BUF_TRACE).  Costs a few global stores per

@@ -52,6 +52,7 @@ struct mk_ctx {
   DevBuf desc, phase_desc;
   DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, route, expert_a, afrag,
       moe_part, trace;
+  DevBuf selftest;   // one descriptor + two counters for mk_selftest_timeout
   bool tracing = false;
   // schedule
   bool have_schedule = false;
@@ -168,7 +169,7 @@ void mk_destroy(mk_ctx* c) {
   for (DevBuf* b : {&c->desc, &c->phase_desc, &c->x, &c->actA,
                     &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
                     &c->rlogits, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
-                    &c->trace})
+                    &c->trace, &c->selftest})
     release(*b);
   c->plan.release();
   delete c;
@@ -689,3 +690,60 @@ mk_status launch_step_in(mk_ctx* c, const int32_t* tokens, const int32_t* positi
 }
 
 }  // namespace mk
+
+// ---------------------------------------------------------------------------
+// Failure-detection self-test: a one-task list whose only wait is on a
+// counter nothing signals, run with a short deadline.  The bounded wait runs
+// out by design; the kernel latches MK_ERR_TIMEOUT, every CTA leaves its task
+// loop, and the status is read back and cleared here.  The step's own
+// counters and epoch are not touched.
+mk_status mk_selftest_timeout(mk_ctx* c, int32_t timeout_ms, int32_t* device_status,
+                              int32_t* detail) {
+  if (!c || timeout_ms <= 0) return MK_ERR_INVALID;
+  if (!c->have_schedule) return MK_ERR_STATE;
+  MK_CUDA(cudaSetDevice(c->device));
+  const size_t bytes = sizeof(int32_t) * (mk::kDescWords + 4);
+  MK_TRY(ensure(c->selftest, bytes));
+  int32_t h[mk::kDescWords + 4];
+  std::memset(h, 0, sizeof(h));
+  h[mk::D_OP] = mk::OP_RN;       // never runs: its wait cannot be met
+  h[mk::D_LAYER] = 0;
+  h[mk::D_NWAIT] = 1;
+  h[mk::D_W0] = 0;               // self-test counter 0: nothing signals it
+  h[mk::D_W0N] = 1;
+  h[mk::D_W1] = -1;
+  h[mk::D_PW] = -1;
+  h[mk::D_S0] = -1;
+  h[mk::D_S1] = -1;
+  h[mk::D_MAP0] = -1;
+  h[mk::D_MAP1] = -1;
+  h[mk::D_ACT] = mk::ACT_NONE;
+  // words kDescWords.. : counter 0 (never signalled), counter 1 (dispenser)
+  MK_CUDA(cudaMemcpy(c->selftest.ptr, h, bytes, cudaMemcpyHostToDevice));
+  MK_CUDA(cudaMemset(c->d_status, 0, sizeof(int32_t) * 16));
+  Params p = c->base;
+  p.desc = static_cast<const int32_t*>(c->selftest.ptr);
+  p.counters = reinterpret_cast<uint32_t*>(static_cast<int32_t*>(c->selftest.ptr) + mk::kDescWords);
+  p.n_tasks = 1;
+  p.grab = 1;
+  p.n_ctas = c->plan.n_ctas;
+  p.epoch = 1;
+  p.trace = nullptr;
+  p.timeout_cycles = (unsigned long long)timeout_ms * 2000000ull;
+  // step inputs are never read (the task does not run); any device address
+  int32_t* d0 = static_cast<int32_t*>(c->selftest.ptr);
+  p.tokens = d0;
+  p.positions = d0;
+  p.page_table = d0;
+  p.seq_lens = d0;
+  p.logits = reinterpret_cast<float*>(c->x.ptr);
+  MK_CUDA(mk::launch_interp(p, c->plan.n_ctas, nullptr));
+  MK_CUDA(cudaDeviceSynchronize());
+  int32_t st[16];
+  MK_CUDA(cudaMemcpy(st, c->d_status, sizeof(st), cudaMemcpyDeviceToHost));
+  MK_CUDA(cudaMemset(c->d_status, 0, sizeof(st)));
+  if (device_status) *device_status = st[mk::ST_CODE];
+  if (detail)
+    for (int i = 0; i < 8; ++i) detail[i] = st[i];
+  return st[mk::ST_CODE] != 0 ? (mk_status)st[mk::ST_CODE] : MK_OK;
+}

@@ -103,6 +103,13 @@ class Decoder:
         if rc != mk.MK_OK:
             raise mk.MKError(rc, "device status", detail)
 
+    def selftest_timeout(self, timeout_ms: int = 10):
+        """Run the failure-detection self-test; returns (status, detail list)."""
+        st = c_int32(0)
+        detail = (c_int32 * 8)()
+        rc = mk.lib.mk_selftest_timeout(self._ctx, int(timeout_ms), byref(st), detail)
+        return int(rc), [int(v) for v in detail]
+
     def set_trace(self, enable: bool) -> None:
         mk.check_status(mk.lib.mk_set_trace(self._ctx, int(bool(enable))), "mk_set_trace")
 

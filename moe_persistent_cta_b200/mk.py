@@ -26,7 +26,8 @@ TRACE_WORDS = 18
 EXPORTS = (
     "mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_step_unfused",
     "mk_decode_step_static",
-    "mk_check", "mk_set_timeout_ms", "mk_set_trace", "mk_debug_read", "mk_debug_size",
+    "mk_check", "mk_selftest_timeout", "mk_set_timeout_ms", "mk_set_trace", "mk_debug_read",
+    "mk_debug_size",
     "mk_plan_schedule", "mk_strerror", "mk_destroy",
 )
 
@@ -76,6 +77,7 @@ def _load():
         "mk_decode_step_unfused": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_decode_step_static": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_check": (c_int, [c_void_p, P(c_int32), P(c_int32)]),
+        "mk_selftest_timeout": (c_int, [c_void_p, c_int32, P(c_int32), P(c_int32)]),
         "mk_set_timeout_ms": (c_int, [c_void_p, c_int32]),
         "mk_set_trace": (c_int, [c_void_p, c_int32]),
         "mk_debug_read": (c_int, [c_void_p, c_int, c_void_p, c_size_t]),

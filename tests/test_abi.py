@@ -36,4 +36,5 @@ def test_strerror_and_argument_validation_without_gpu():
     assert mk.lib.mk_decode_step(None, None, None, None, None, None, None) == mk.MK_ERR_INVALID
     assert mk.lib.mk_decode_step_static(None, None, None, None, None, None,
                                         None) == mk.MK_ERR_INVALID
+    assert mk.lib.mk_selftest_timeout(None, 10, None, None) == mk.MK_ERR_INVALID
     mk.lib.mk_destroy(None)
