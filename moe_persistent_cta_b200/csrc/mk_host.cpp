@@ -50,6 +50,7 @@ struct mk_ctx {
   uint32_t* d_counters = nullptr;
   int counters_cap = 0;
   DevBuf desc, phase_desc;
+  bool phases_uploaded = false;
   DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, route, expert_a, afrag,
       moe_part, trace;
   DevBuf selftest;   // one descriptor + two counters for mk_selftest_timeout
@@ -326,7 +327,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   MK_CUDA(cudaDeviceSynchronize());
   c->have_schedule = false;
   Plan plan;
-  MK_TRY((mk_status)mk::plan_schedule(s, c->n_sms, batch, seq_lens, plan_len, true, &plan));
+  MK_TRY((mk_status)mk::plan_schedule(s, c->n_sms, batch, seq_lens, plan_len, false, &plan));
   SmemLayout sl;
   {
     int rc = mk::smem_layout(s, batch, plan.max_chunks, &sl);
@@ -369,7 +370,6 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   ENSURE(afrag, (size_t)L * S * afrag_bytes);
   ENSURE(moe_part, (size_t)L * s.k * B * d * 4);
   ENSURE(desc, (size_t)plan.n_tasks * mk::kDescWords * 4);
-  ENSURE(phase_desc, (size_t)plan.n_tasks * mk::kDescWords * 4);
 #undef ENSURE
   if (plan.n_counters > c->counters_cap) {
     cudaFree(c->d_counters);
@@ -383,10 +383,9 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
     return fail(MK_ERR_CUDA);
   if (cudaMemset(c->route.ptr, 0, c->route.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
   if (cudaMemcpy(c->desc.ptr, plan.desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
-                 cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(c->phase_desc.ptr, plan.phase_desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
                  cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(MK_ERR_CUDA);
+  c->phases_uploaded = false;   // the unfused path builds its phase lists on first use
 
   Params& p = c->base;
   std::memset(&p, 0, sizeof(p));
@@ -484,6 +483,15 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
     p.grab = c->plan.grab;
     e = mk::launch_interp(p, c->plan.n_ctas, st);
   } else {
+    if (!c->phases_uploaded) {
+      // the same tasks grouped by phase, each group in list order
+      const size_t bytes = (size_t)c->plan.n_tasks * mk::kDescWords * 4;
+      std::vector<int32_t> h((size_t)c->plan.n_tasks * mk::kDescWords);
+      mk::group_by_phase(c->plan, h.data());
+      MK_TRY(ensure(c->phase_desc, bytes));
+      MK_CUDA(cudaMemcpy(c->phase_desc.ptr, h.data(), bytes, cudaMemcpyHostToDevice));
+      c->phases_uploaded = true;
+    }
     for (int ph = 0; ph < c->plan.n_phases && e == cudaSuccess; ++ph) {
       const int n = c->plan.phase_off[ph + 1] - c->plan.phase_off[ph];
       if (n == 0) continue;

@@ -262,6 +262,7 @@ int validate_shape(const Shape& s);
 // Validates the shape and builds the plan; returns 0 or an mk_status code.
 int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
                   const int32_t* plan_len, bool with_phases, Plan* out);
+void group_by_phase(const Plan& plan, int32_t* out);
 
 // GEMV tile geometry shared by planner and host (rows per tile for a K).
 int gemv_rows_for(int K, int n_mat);

@@ -693,6 +693,17 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   return MK_OK;
 }
 
+// The unfused launcher's lists: the plan's tasks grouped by phase (phase ph
+// at [phase_off[ph], phase_off[ph + 1]) of `out`), each group in list order.
+void group_by_phase(const Plan& plan, int32_t* out) {
+  std::vector<int> fill(plan.phase_off, plan.phase_off + plan.n_phases);
+  for (int i = 0; i < plan.n_tasks; ++i) {
+    const int32_t* w = plan.desc + (size_t)i * kDescWords;
+    const int pos = fill[w[D_PHASE]]++;
+    std::memcpy(out + (size_t)pos * kDescWords, w, sizeof(int32_t) * kDescWords);
+  }
+}
+
 }  // namespace mk
 
 extern "C" mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batch,
