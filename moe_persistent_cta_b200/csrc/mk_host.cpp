@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -51,7 +52,7 @@ struct mk_ctx {
   int counters_cap = 0;
   DevBuf desc, phase_desc;
   bool phases_uploaded = false;
-  DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, route, expert_a, afrag,
+  DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, rpart, route, expert_a, afrag,
       moe_part, trace;
   DevBuf selftest;   // one descriptor + two counters for mk_selftest_timeout
   bool tracing = false;
@@ -169,7 +170,7 @@ void mk_destroy(mk_ctx* c) {
   cudaFree(c->d_counters);
   for (DevBuf* b : {&c->desc, &c->phase_desc, &c->x, &c->actA,
                     &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
-                    &c->rlogits, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
+                    &c->rlogits, &c->rpart, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
                     &c->trace, &c->selftest})
     release(*b);
   c->plan.release();
@@ -234,7 +235,9 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
       return fail(st);
     if ((st = encode_3d(m + 1, t->w_o[l], (uint64_t)s.Hq * s.hd, s.d, 64, 2)) != MK_OK)
       return fail(st);
-    if ((st = encode_3d(m + 2, t->w_router[l], s.d, s.E, c->r_qkv, ch_qkv)) != MK_OK)
+    // router: one 64-column chunk of up to 128 expert rows per copy
+    if ((st = encode_3d(m + mk::kMapRouter, t->w_router[l], s.d, s.E,
+                        (uint32_t)std::min(s.E, mk::kRouterRowsPerStage), 1)) != MK_OK)
       return fail(st);
     if ((st = encode_3d(m + 3, t->w_gate[l], s.d, (uint64_t)s.E * s.F, c->r_ff, ch_ff)) != MK_OK)
       return fail(st);
@@ -365,6 +368,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   ENSURE(ofrag, (size_t)L * s.Hkv * ofrag_bytes);
   ENSURE(o_part, (size_t)L * s.Hkv * B * d * 4);
   ENSURE(rlogits, (size_t)L * B * s.E * 4);
+  ENSURE(rpart, (size_t)L * NR * B * s.E * 4);
   ENSURE(route, (size_t)L * rwords * 4);
   ENSURE(expert_a, (size_t)L * S * B * s.F * 4);
   ENSURE(afrag, (size_t)L * S * afrag_bytes);
@@ -419,6 +423,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.ofrag = static_cast<uint8_t*>(c->ofrag.ptr);
   p.o_part = static_cast<float*>(c->o_part.ptr);
   p.rlogits = static_cast<float*>(c->rlogits.ptr);
+  p.rpart = static_cast<float*>(c->rpart.ptr);
   p.route = static_cast<int32_t*>(c->route.ptr);
   p.expert_a = static_cast<float*>(c->expert_a.ptr);
   p.afrag = static_cast<uint8_t*>(c->afrag.ptr);
@@ -435,6 +440,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.actB_bytes = sl.actB_bytes;
   p.off_ring = sl.off_ring;
   p.off_epi = sl.off_epi;
+  p.off_ptrs = sl.off_ptrs;
   p.part_cols = sl.part_cols;
   p.smem_bytes = sl.dyn_bytes;
 
@@ -640,6 +646,7 @@ size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) 
   uint8_t* ofrag = take(L * b.Hkv * (size_t)b.ofrag_bytes);
   uint8_t* o_part = take(L * b.Hkv * B * d * 4);
   uint8_t* rlogits = take(L * B * b.E * 4);
+  uint8_t* rpart = take(L * b.NR * B * b.E * 4);
   uint8_t* expert_a = take(L * b.S * B * b.F * 4);
   uint8_t* afrag = take(L * b.S * (size_t)b.afrag_bytes);
   uint8_t* moe_part = take(L * b.k * B * d * 4);
@@ -655,6 +662,7 @@ size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) 
     p->ofrag = ofrag;
     p->o_part = reinterpret_cast<float*>(o_part);
     p->rlogits = reinterpret_cast<float*>(rlogits);
+    p->rpart = reinterpret_cast<float*>(rpart);
     p->expert_a = reinterpret_cast<float*>(expert_a);
     p->afrag = afrag;
     p->moe_part = reinterpret_cast<float*>(moe_part);

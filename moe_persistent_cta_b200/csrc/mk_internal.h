@@ -33,15 +33,22 @@ constexpr int kFirstConsumerWarp = 3;
 constexpr int kEpilogueWarp = kFirstConsumerWarp + kConsumerWarps;   // 11
 constexpr int kThreads = (kEpilogueWarp + 1) * 32;                    // 384
 constexpr int kRstdRing = 4;         // per-level 1/rms slots (levels in flight)
-constexpr int kTopkScratch = 2048;   // epilogue warp scratch: top-k join (1.5 KB), router bias (512 B)
 constexpr int kMaxParts = 1 + 16 + kMaxTopK;   // residual + O-proj groups + expert ranks
 constexpr int kFifo = 16;            // task entries in flight per CTA
 constexpr int kFifoEntryWords = 64;  // 32 descriptor words + 32 resolved words
 constexpr int kMapsPerLayer = 8;     // qkv, o, router, gate, up, down, kpool, vpool
+constexpr int kMapRouter = 2;
 // Activation rows are padded by 8 floats so that the 8 columns a warp reads
 // at one k land in different shared-memory banks.
 constexpr int kActPad = 8;
 constexpr int kRnStage = 4096;       // floats of residual partials staged per round
+constexpr int kRouterRowsPerStage = 128;   // router weight rows (x 64 columns) per ring stage
+constexpr int kTopkLogitsOff = 2048; // top-k scratch: selection state, then logits [B][E]
+// Per-layer pointer table in shared memory: norm weights of levels 0..L (the
+// final norm last), then router bias, K pool and V pool of layers 0..L-1.  A
+// task reads its layer's pointers from there, so its first global loads need
+// no dependent pointer load.
+MK_HD constexpr int ptr_table_words(int L) { return 4 * L + 1; }
 constexpr int kTraceWords = 18;      // per task: see TraceField
 
 // Per-task trace words: globaltimer stamps (low 32 bits, ns) and the CTA
@@ -72,7 +79,7 @@ enum Op : int32_t {
   OP_NONE = 0,
   OP_RN = 1,        // fused residual add + RMSNorm statistics for one 64-row tile
   OP_QKV = 2,       // QKV projection tile (RoPE/append happen in OP_ATTN)
-  OP_ROUTER = 3,    // router logits tile
+  OP_ROUTER = 3,    // (unused: the norm tiles produce the router logits)
   OP_TOPK = 4,      // top-k + softmax + expert-slot compaction
   OP_ATTN = 5,      // paged GQA decode attention over one KV chunk (+RoPE, append)
   OP_COMBINE = 6,   // log-sum-exp merge of the chunk partials of (b, g)
@@ -183,6 +190,7 @@ struct Params {
   uint8_t* ofrag;    // [L][Hkv][ofrag_bytes]
   float* o_part;     // [L][Hkv][B][d]
   float* rlogits;    // [L][B][E]
+  float* rpart;      // [L][NR][B][E] router logits per 64-column tile (before 1/rms)
   int32_t* route;    // [L][route_words]
   float* expert_a;   // [L][S][B][F]
   uint8_t* afrag;    // [L][S][afrag_bytes]
@@ -194,8 +202,8 @@ struct Params {
   int n_stages, nA, actA_stride;
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, actB_bytes, off_ring;
   int off_epi;       // GEMV partials [2][kConsumerWarps][16][part_cols], then the
-                     // per-level 1/rms ring [kRstdRing][kMaxBatch], then the
-                     // epilogue warp's top-k scratch (kTopkScratch bytes)
+                     // per-level 1/rms ring [kRstdRing][kMaxBatch]
+  int off_ptrs;      // per-layer pointer table, copied in at launch (see PtrTable)
   int part_cols;     // token columns per partial row: B for B <= 2, else 8
   int smem_bytes;
 };
@@ -249,7 +257,7 @@ struct SmemLayout {
   int actB_bytes;     // bytes per small-activation buffer (two of them)
   int scratch_bytes;
   int n_stages;       // ring stages of kStageBytes
-  int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring, off_epi;
+  int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring, off_epi, off_ptrs;
   int part_cols;
   int total;          // bytes from the 1024-aligned base
   int dyn_bytes;      // dynamic shared memory to request (total + alignment slack)

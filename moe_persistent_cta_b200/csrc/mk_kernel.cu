@@ -227,6 +227,7 @@ struct Smem {
   uint8_t* actA;
   uint8_t* actB;
   uint8_t* epi;
+  const void* const* ptrs;   // per-layer pointer table
   int32_t* fifo;
   uint32_t bars;  // shared-window address of barrier 0
   int NS;
@@ -245,6 +246,20 @@ struct Smem {
   __device__ uint32_t pempty(int i) const { return bar(2 * NS + 4 * kFifo + 10 + i); }
 };
 
+// Entries of the shared-memory pointer table.
+__device__ __forceinline__ const uint16_t* norm_w(const Smem& sm, int lv) {
+  return static_cast<const uint16_t*>(sm.ptrs[lv]);   // lv == L: the final norm
+}
+__device__ __forceinline__ const float* router_b(const Params& p, const Smem& sm, int l) {
+  return static_cast<const float*>(sm.ptrs[p.L + 1 + l]);
+}
+__device__ __forceinline__ uint16_t* kpool_of(const Params& p, const Smem& sm, int l) {
+  return static_cast<uint16_t*>(const_cast<void*>(sm.ptrs[2 * p.L + 1 + l]));
+}
+__device__ __forceinline__ uint16_t* vpool_of(const Params& p, const Smem& sm, int l) {
+  return static_cast<uint16_t*>(const_cast<void*>(sm.ptrs[3 * p.L + 1 + l]));
+}
+
 __device__ __forceinline__ Smem smem_view(const Params& p) {
   Smem s;
   const uint32_t raw = saddr(g_smem);
@@ -255,6 +270,7 @@ __device__ __forceinline__ Smem smem_view(const Params& p) {
   s.actA = base + p.off_actA;
   s.actB = base + p.off_actB;
   s.epi = base + p.off_epi;
+  s.ptrs = reinterpret_cast<const void* const*>(base + p.off_ptrs);
   s.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
   s.bars = raw + pad + (uint32_t)p.off_bars;
   s.NS = p.n_stages;
@@ -539,6 +555,27 @@ __device__ __noinline__ void producer_loop(const Params& p) {
           const int y = (phys * p.Hkv + g) * kPage;
           const void* m = (s & 1) ? mv_ : mk_;
           tma_3d(dst, m, 0, y, 0, fb, pol);   // [hd/64 chunks][64 tokens][128 B]
+        }
+        __syncwarp();
+        ring_next();
+      }
+      if (fail) break;
+    } else if (op == OP_RN && nstage > 0) {
+      // the tile's router weights: rows [128 s, 128 s + 128) of its 64-column
+      // chunk; rows past E land as zeros
+      const int r = __shfl_sync(FULL, dw, D_A);
+      const void* m0 = tmap(p, map0);
+      const uint32_t box_bytes = (uint32_t)min(p.E, kRouterRowsPerStage) * 128u;
+      for (int s = 0; s < nstage; ++s) {
+        if (!warp_wait(p, sm.empty(slot), phase ^ 1, 103)) {
+          fail = true;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = sm.full(slot);
+          mbar_expect_tx(fb, box_bytes);
+          const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
+          tma_3d(dst, m0, 0, kRouterRowsPerStage * s, r, fb, pol);
         }
         __syncwarp();
         ring_next();
@@ -942,8 +979,7 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
 // the operation's outputs.  `rs` is the level's 1/rms per token (A-input
 // operations).
 __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* ent,
-                                              const float* part, const float* rs,
-                                              const float* bias_s) {
+                                              const float* part, const float* rs) {
   const int lane = threadIdx.x & 31;
   const int op = ent[D_OP], layer = ent[D_LAYER];
   const int nm = ent[D_NMAT], R = ent[D_R], row0 = ent[D_ROW0];
@@ -965,9 +1001,6 @@ __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* en
     switch (op) {
       case OP_QKV:
         p.qkv[((size_t)layer * p.B + n) * p.qkvR + row] = s0 * rs[n];
-        break;
-      case OP_ROUTER:
-        if (row < p.E) p.rlogits[((size_t)layer * p.B + n) * p.E + row] = s0 * rs[n] + bias_s[r];
         break;
       case OP_LMHEAD:
         if (row < p.V) p.logits[(size_t)n * p.V + row] = s0 * rs[n];
@@ -1000,7 +1033,7 @@ __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* en
 }
 
 __device__ __forceinline__ bool is_gemv(int op) {
-  return op == OP_QKV || op == OP_ROUTER || op == OP_OPROJ || op == OP_GATEUP ||
+  return op == OP_QKV || op == OP_OPROJ || op == OP_GATEUP ||
          op == OP_DOWN || op == OP_LMHEAD;
 }
 
@@ -1058,8 +1091,8 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     vn[i] = __bfloat162float(vb);
     if (flags & F_LAST_CHUNK) {
       const size_t off = (((size_t)phys_new * p.Hkv + g) * kPage + (seqlen % kPage)) * HD + i;
-      reinterpret_cast<__nv_bfloat16*>(p.k_pool[layer])[off] = kb;
-      reinterpret_cast<__nv_bfloat16*>(p.v_pool[layer])[off] = vb;
+      reinterpret_cast<__nv_bfloat16*>(kpool_of(p, sm, layer))[off] = kb;
+      reinterpret_cast<__nv_bfloat16*>(vpool_of(p, sm, layer))[off] = vb;
     }
   }
   cbar();
@@ -1320,10 +1353,19 @@ __device__ __noinline__ void rope_table(const Params& p, int task) {
 // Fused residual add + RMSNorm statistics for one 64-column tile of level l:
 // x_l = x_{l-1} + sum_g o_part[g] + sum_j moe_part[j] (fixed order), the
 // gamma-scaled rows the next projections read, and the tile's sum of squares
-// per token (1/rms is applied in the consumers' epilogues).  The partials are
-// staged through shared memory in rounds so that all loads of a round are in
-// flight at once.
-__device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
+// per token (1/rms is applied by the readers).  The partials are staged
+// through shared memory in rounds so that all loads of a round are in flight
+// at once.
+//
+// A level that feeds a layer also gets the tile's share of that layer's
+// router logits: rpart[l][r][b][e] = sum over the tile's 64 columns c of
+// W_r[e][c] (gamma x)[b][c].  The producer streams the tile's router columns
+// into the ring when it hands the task out (128 expert rows of 128 bytes per
+// stage, 128-byte swizzled), so they are resident before the inputs are.
+// Unit u = 8 e + ch covers columns 8 ch .. 8 ch + 7 of expert row e (one
+// 16-byte shared load); the eight lanes of a row reduce by shuffles and lane
+// ch stores token ch.  Returns the advanced ring counter.
+__device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int l = ent[D_LAYER], r = ent[D_A];
@@ -1331,47 +1373,88 @@ __device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
   float* xs = reinterpret_cast<float*>(sm.scratch);  // [B][64]
   float* stage = xs + kMaxBatch * 64;                 // [kRnStage] staged partials
   const int nparts = (l == 0) ? 1 : 1 + p.Hkv + p.k;
-  const int per_round = kRnStage / per;
-  const int per4 = per / 4;   // float4 units (4 consecutive columns) per part
-  for (int j0 = 0; j0 < nparts; j0 += per_round) {
-    const int nj = min(per_round, nparts - j0);
-    // every load of the round is issued before any is used (one L2 round trip)
-#pragma unroll 4
-    for (int t4 = ct; t4 < nj * per4; t4 += 256) {
-      const int j = j0 + t4 / per4, e4 = t4 % per4, b = e4 >> 4, col = r * 64 + 4 * (e4 & 15);
-      float4 v;
-      if (l == 0) {
-        int tok = __ldg(p.tokens + b);
-        if (tok < 0 || tok >= p.V) {
-          if ((e4 & 15) == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
-          tok = 0;
-        }
-        const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.embed + (size_t)tok * d + col));
-        v = make_float4(lo_bf16(w.x), hi_bf16(w.x), lo_bf16(w.y), hi_bf16(w.y));
-      } else {
-        const float* src =
-            j == 0 ? p.x + (size_t)(l - 1) * B * d
-            : j <= p.Hkv ? p.o_part + ((size_t)(l - 1) * p.Hkv + (j - 1)) * B * d
-                         : p.moe_part + ((size_t)(l - 1) * p.k + (j - 1 - p.Hkv)) * B * d;
-        v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * d + col));
-      }
-      reinterpret_cast<float4*>(stage)[t4] = v;
-    }
-    cbar();
+  const int nst = ent[32 + R_NSTAGE];   // router stages (0 for the final norm)
+  // this thread's gamma column (every element it owns is column ct % 64)
+  const float gam =
+      __uint_as_float((uint32_t)__ldg(norm_w(sm, l) + r * 64 + (ct & 63)) << 16);
+  if (l == 0) {
+    // the embedding rows of this step's tokens
+#pragma unroll 1
     for (int e = ct; e < per; e += 256) {
-      float x = j0 == 0 ? 0.f : xs[e];
-      for (int j = 0; j < nj; ++j) x += stage[j * per + e];
-      xs[e] = x;
+      const int b = e >> 6;
+      int tok = __ldg(p.tokens + b);
+      if (tok < 0 || tok >= p.V) {
+        if ((e & 63) == 0) raise_error(p, MK_ERR_DEVICE, ent[32 + R_TASK], OP_RN, -1, tok, p.V, 4);
+        tok = 0;
+      }
+      xs[e] = __uint_as_float((uint32_t)__ldg(p.embed + (size_t)tok * d + r * 64 + (e & 63)) << 16);
+    }
+  } else {
+    // part j of the sum (x_{l-1}, then the O-proj partial of each KV group,
+    // then the expert partial of each rank), at this tile's first column
+    const float** pp = reinterpret_cast<const float**>(stage + kRnStage) - kMaxParts;
+    if (ct < nparts) {
+      const int j = ct;
+      const size_t lb = (size_t)(l - 1);
+      const float* src = j == 0 ? p.x + lb * B * d
+                         : j <= p.Hkv ? p.o_part + (lb * p.Hkv + (j - 1)) * B * d
+                                      : p.moe_part + (lb * p.k + (j - 1 - p.Hkv)) * B * d;
+      pp[j] = src + r * 64;
     }
     cbar();
+    // thread (group jg, float4 column e4) sums parts jg, jg + nJ, ... with
+    // eight loads in flight; the groups' sums are then added in jg order
+    const int per4 = B * 16, nJ = 256 / per4;
+    float4* grp = reinterpret_cast<float4*>(stage);   // [nJ][per4]
+    if (ct < nJ * per4) {
+      const int jg = ct / per4, e4 = ct - jg * per4;
+      const size_t off = (size_t)(e4 >> 4) * d + 4 * (e4 & 15);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int j0 = jg; j0 < nparts; j0 += 8 * nJ) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = j0 + i * nJ;
+          v[i] = j < nparts ? __ldcg(reinterpret_cast<const float4*>(pp[j] + off))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc.x += v[i].x;
+          acc.y += v[i].y;
+          acc.z += v[i].z;
+          acc.w += v[i].w;
+        }
+      }
+      grp[jg * per4 + e4] = acc;
+    }
+    cbar();
+#pragma unroll 1
+    for (int e4 = ct; e4 < per4; e4 += 256) {
+      float4 x = grp[e4];
+#pragma unroll 1
+      for (int g = 1; g < nJ; ++g) {
+        const float4 v = grp[g * per4 + e4];
+        x.x += v.x;
+        x.y += v.y;
+        x.z += v.z;
+        x.w += v.w;
+      }
+      reinterpret_cast<float4*>(xs)[e4] = x;
+    }
   }
+  cbar();
   float* rows = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes);
-  const uint16_t* gam = (l < p.L) ? p.attn_norm[l] : p.final_norm;
+  float* gxs = stage;   // [B][64] gamma x of the tile (the staging area is free)
+#pragma unroll 1
   for (int e = ct; e < per; e += 256) {
     const int b = e >> 6, col = r * 64 + (e & 63);
     const float x = xs[e];
+    const float gx = x * gam;
     p.x[((size_t)l * B + b) * d + col] = x;
-    rows[(size_t)b * (d + kActPad) + col] = x * __uint_as_float((uint32_t)__ldg(gam + col) << 16);
+    rows[(size_t)b * (d + kActPad) + col] = gx;
+    gxs[e] = gx;
   }
   if (cw < B) {
     const float x0 = xs[cw * 64 + lane], x1 = xs[cw * 64 + 32 + lane];
@@ -1381,25 +1464,137 @@ __device__ __forceinline__ void rn_task(const Params& p, const int32_t* ent) {
       reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_rows_bytes)[r * B + cw] = ss;
   }
   if (l == 0 && r == 0) rope_table(p, ent[32 + R_TASK]);
+  if (nst == 0) return stage_ctr;
+  cbar();
+  float* out = p.rpart + ((size_t)l * p.NR + r) * B * p.E;
+  auto unit = [&](int e, int ch, bool valid, const uint4 w) {
+    const float wf[8] = {lo_bf16(w.x), hi_bf16(w.x), lo_bf16(w.y), hi_bf16(w.y),
+                         lo_bf16(w.z), hi_bf16(w.z), lo_bf16(w.w), hi_bf16(w.w)};
+    float mine = 0.f;
+#pragma unroll 1
+    for (int b = 0; b < B; ++b) {   // uniform: every lane takes part in the shuffles
+      const float4 g0 = reinterpret_cast<const float4*>(gxs + b * 64 + ch * 8)[0];
+      const float4 g1 = reinterpret_cast<const float4*>(gxs + b * 64 + ch * 8)[1];
+      float a = wf[0] * g0.x;
+      a = fmaf(wf[1], g0.y, a);
+      a = fmaf(wf[2], g0.z, a);
+      a = fmaf(wf[3], g0.w, a);
+      a = fmaf(wf[4], g1.x, a);
+      a = fmaf(wf[5], g1.y, a);
+      a = fmaf(wf[6], g1.z, a);
+      a = fmaf(wf[7], g1.w, a);
+      a += __shfl_xor_sync(FULL, a, 4);
+      a += __shfl_xor_sync(FULL, a, 2);
+      a += __shfl_xor_sync(FULL, a, 1);
+      if (b == ch) mine = a;
+    }
+    if (valid && ch < B) out[(size_t)ch * p.E + e] = mine;
+  };
+#pragma unroll 1
+  for (int s = 0; s < nst; ++s) {
+    const uint32_t slot = stage_ctr % (uint32_t)sm.NS, ph = (stage_ctr / (uint32_t)sm.NS) & 1u;
+    wait_bar(p, sm.full(slot), ph, 404);
+    const uint8_t* wt = sm.ring + (size_t)slot * kStageBytes;
+    const int e0 = kRouterRowsPerStage * s;
+    const int nu = min(kRouterRowsPerStage, p.E - e0) * 8;   // units in this stage
+#pragma unroll 1
+    for (int u0 = 0; u0 < nu; u0 += 256) {                    // uniform trip count
+      const int u = u0 + ct, el = u >> 3, ch = u & 7;
+      const bool valid = u < nu;
+      const uint4 w = valid ? *reinterpret_cast<const uint4*>(wt + el * 128 + ((ch ^ (el & 7)) << 4))
+                            : make_uint4(0u, 0u, 0u, 0u);
+      unit(e0 + el, ch, valid, w);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(slot));
+    ++stage_ctr;
+  }
+  return stage_ctr;
 }
 
-// top-k (logit desc, index asc) + softmax over the selected + slot compaction
-
-__device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
+// Router logits of layer l from the norm tiles' shares, then top-k (logit
+// desc, index asc) + softmax over the selected + slot compaction.
+// logits[b][e] = (1/rms_b) * sum_r rpart[l][r][b][e] + bias[e], the shares
+// summed in ascending r: thread group g of nG sums r = g, g + nG, ... of one
+// float4 column, and the groups' sums are added in g order.
+__device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int l = ent[D_LAYER];
-  const int B = p.B, E = p.E, K = p.k, S = p.S;
+  const int B = p.B, E = p.E, K = p.k, S = p.S, NR = p.NR;
   int32_t* rt = p.route + (size_t)l * p.route_words;
   int* sel = reinterpret_cast<int*>(sm.scratch);               // [B][8]
   float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [B][8]
   int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8); // [E]
   uint32_t* used = reinterpret_cast<uint32_t*>(slot_of + 256); // [8]
+  float* rstd_s = reinterpret_cast<float*>(used + 8);          // [B]
+  float* lgs = reinterpret_cast<float*>(sm.scratch + kTopkLogitsOff);   // [B][E]
+  float4* grp = reinterpret_cast<float4*>(lgs + kMaxBatch * 256);       // [nG][C4]
+  const int C4 = B * E / 4;
+  const int span = min(C4, 256), nG = 256 / span;
+  const float* bias = router_b(p, sm, l);
+  const float bv = (bias && ct < E) ? __ldg(bias + ct) : 0.f;   // expert ct's bias
+  {
+    const float4* rp = reinterpret_cast<const float4*>(p.rpart + (size_t)l * NR * B * E);
+    if (ct < nG * span) {
+      const int g = ct / span;
+#pragma unroll 1
+      for (int c4 = ct - g * span; c4 < C4; c4 += 256) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        // eight independent loads in flight, then added in r order
+#pragma unroll 1
+        for (int rr0 = g; rr0 < NR; rr0 += 8 * nG) {
+          float4 v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int rr = rr0 + j * nG;
+            v[j] = rr < NR ? __ldcg(rp + (size_t)rr * C4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            a.x += v[j].x;
+            a.y += v[j].y;
+            a.z += v[j].z;
+            a.w += v[j].w;
+          }
+        }
+        if (nG == 1)
+          reinterpret_cast<float4*>(lgs)[c4] = a;
+        else
+          grp[g * C4 + c4] = a;
+      }
+    }
+  }
   if (ct < 8) used[ct] = 0u;
+  if (cw < B) {
+    // 1/rms of token cw from the level's sum-of-squares partials
+    const float* ss = reinterpret_cast<const float*>(p.actA + (size_t)l * p.actA_bytes +
+                                                     p.actA_rows_bytes);
+    float acc = 0.f;
+#pragma unroll 1
+    for (int rr = lane; rr < NR; rr += 32) acc += __ldcg(ss + rr * B + cw);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+    if (lane == 0) rstd_s[cw] = frsqrt(acc / (float)p.d + p.eps);
+  }
+  cbar();
+  // thread e finishes expert e of every token
+  if (ct < E) {
+    const float* gs = reinterpret_cast<const float*>(grp);
+#pragma unroll 1
+    for (int bb = 0; bb < B; ++bb) {
+      const int i = bb * E + ct;
+      float v = nG == 1 ? lgs[i] : 0.f;
+#pragma unroll 1
+      for (int g = 0; g < (nG == 1 ? 0 : nG); ++g) v += gs[g * 4 * C4 + i];
+      v = v * rstd_s[bb] + bv;
+      lgs[i] = v;
+      p.rlogits[(size_t)l * B * E + i] = v;
+    }
+  }
   cbar();
   const int b = cw;
   if (b < B) {
-    const float* lg = p.rlogits + ((size_t)l * B + b) * E;
+    const float* lg = lgs + b * E;
     // order-preserving unsigned keys of the logits; 0 marks taken / absent
     uint32_t key[8];
 #pragma unroll
@@ -1407,12 +1602,12 @@ __device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
       const int e = lane + 32 * t;
       uint32_t k = 0u;
       if (e < E) {
-        const uint32_t u = __float_as_uint(__ldcg(lg + e));
+        const uint32_t u = __float_as_uint(lg[e]);
         k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
       }
       key[t] = k;
     }
-    float selv[8];
+#pragma unroll 1
     for (int j = 0; j < K; ++j) {
       uint32_t bk = 0u;
       int bi = 0x7fffffff;
@@ -1428,36 +1623,42 @@ __device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
 #pragma unroll
       for (int t = 0; t < 8; ++t)
         if (lane + 32 * t == wi) key[t] = 0u;
-      const uint32_t u = (mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk;
-      selv[j] = __uint_as_float(u);
-      if (lane == 0) sel[b * 8 + j] = wi;
+      if (lane == 0) {
+        sel[b * 8 + j] = wi;
+        wsel[b * 8 + j] = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk);
+      }
     }
-    if (lane == 0) {
-      float ws[8], sum = 0.f;
-      for (int j = 0; j < K; ++j) {
-        ws[j] = fexp(selv[j] - selv[0]);
-        sum += ws[j];
-      }
-      for (int j = 0; j < K; ++j) {
-        const float w = ws[j] * frcp(sum);
-        wsel[b * 8 + j] = w;
-        rt[route_topk_idx(B, K) + b * K + j] = sel[b * 8 + j];
-        reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + j] = w;
-        atomicOr(&used[sel[b * 8 + j] >> 5], 1u << (sel[b * 8 + j] & 31));
-      }
+    __syncwarp();
+    // softmax over the selected logits: lane j < K takes rank j
+    const float v0 = wsel[b * 8];
+    float w = lane < K ? fexp(wsel[b * 8 + (lane & 7)] - v0) : 0.f;
+    float sum = w;
+    for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+    __syncwarp();
+    if (lane < K) {
+      w *= frcp(sum);
+      const int e = sel[b * 8 + lane];
+      wsel[b * 8 + lane] = w;
+      rt[route_topk_idx(B, K) + b * K + lane] = e;
+      reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + lane] = w;
+      atomicOr(&used[e >> 5], 1u << (e & 31));
     }
   }
   cbar();
   // slot of each used expert = number of used experts below it
+#pragma unroll 1
   for (int e = ct; e < E; e += 256) {
     int cnt = 0;
+#pragma unroll 1
     for (int w = 0; w < (e >> 5); ++w) cnt += __popc(used[w]);
     cnt += __popc(used[e >> 5] & ((1u << (e & 31)) - 1u));
     slot_of[e] = ((used[e >> 5] >> (e & 31)) & 1u) ? cnt : -1;
   }
   cbar();
   int n_used = 0;
+#pragma unroll
   for (int w = 0; w < 8; ++w) n_used += __popc(used[w]);
+#pragma unroll 1
   for (int s = ct; s < S; s += 256) {
     if (s >= n_used) {
       rt[route_slot_expert(B, K) + s] = -1;
@@ -1471,14 +1672,18 @@ __device__ __forceinline__ void topk_task(const Params& p, const int32_t* ent) {
     const int e = sel[bb * 8 + j];
     const int s = slot_of[e];
     int pos = 0;
+#pragma unroll 1
     for (int b2 = 0; b2 < bb; ++b2)
+#pragma unroll 1
       for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
     rt[route_slot_tok(B, K, S) + s * 8 + pos] = bb;
     rt[route_slot_rank(B, K, S) + s * 8 + pos] = j;
     reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s * 8 + pos] = wsel[bb * 8 + j];
     if (pos == 0) {
       int cnt = 0;
+#pragma unroll 1
       for (int b2 = 0; b2 < B; ++b2)
+#pragma unroll 1
         for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
       rt[route_slot_expert(B, K) + s] = e;
       rt[route_slot_ntok(B, K, S) + s] = cnt;
@@ -1588,7 +1793,7 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
 
     switch (op) {
       case OP_RN:
-        rn_task(p, ent);
+        stage_ctr = rn_task(p, ent, stage_ctr);
         break;
       case OP_TOPK:
         topk_task(p, ent);
@@ -1627,207 +1832,6 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
   }
 }
 
-// ========================================================== last arriver ==
-// A group of tasks that feeds one join (the 64-column norm tile, the layer's
-// top-k, the (b, g) attention merge) counts its arrivals on a counter; the
-// task whose arrival completes this step's count does the join.  The arrival
-// is an acquire-release add by one thread after a barrier of the writers:
-// release publishes this task's outputs (the barrier orders the other
-// writers' stores before it), acquire makes the earlier arrivals' outputs
-// visible to the last one, which reads them through L2.
-__device__ __forceinline__ bool warp_arrive_last(const Params& p, int ctr, int arrivals) {
-  __syncwarp();
-  uint32_t old = 0;
-  if ((threadIdx.x & 31) == 0) old = atom_add_acq_rel(p.counters + ctr, 1u);
-  old = __shfl_sync(FULL, old, 0);
-  return old + 1u == p.epoch * (uint32_t)arrivals;
-}
-__device__ __forceinline__ void warp_signal(const Params& p, int ctr) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) red_release_add(p.counters + ctr, 1u);
-}
-__device__ __forceinline__ float4 ldcg4(const float* a) {
-  return __ldcg(reinterpret_cast<const float4*>(a));
-}
-
-// Residual add + RMSNorm statistics of the 64 columns [64 r, 64 r + 64) for
-// level lv >= 1, by one warp: x_lv = x_{lv-1} + the O-proj partials of every
-// KV group + the expert partials of every rank (in that order), written to x;
-// gamma * x into the level's activation rows; and per token the tile's sum of
-// squares, from which every reader of the level forms 1/rms.  Half-warp h
-// takes tokens h, h + 2, ...; lane q of a half its 4 columns.
-__device__ __noinline__ void fused_norm(const Params& p, int lv, int r) {
-  const int lane = threadIdx.x & 31;
-  const int B = p.B, d = p.d, Hkv = p.Hkv, K = p.k;
-  const int q = lane & 15, col = r * 64 + 4 * q;
-  const int l = lv - 1;
-  const uint16_t* gam = (lv < p.L) ? p.attn_norm[lv] : p.final_norm;
-  const uint2 gw = __ldg(reinterpret_cast<const uint2*>(gam + col));
-  const float g0 = lo_bf16(gw.x), g1 = hi_bf16(gw.x), g2 = lo_bf16(gw.y), g3 = hi_bf16(gw.y);
-  float* rows = reinterpret_cast<float*>(p.actA + (size_t)lv * p.actA_bytes);
-  float* ssp = reinterpret_cast<float*>(p.actA + (size_t)lv * p.actA_bytes + p.actA_rows_bytes);
-  const int nparts = 1 + Hkv + K;
-  for (int b0 = 0; b0 < B; b0 += 2) {
-    const int b = b0 + (lane >> 4);
-    float ss = 0.f;
-    if (b < B) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j0 = 0; j0 < nparts; j0 += 8) {   // 8 loads in flight per round
-        float4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u;
-          if (j < nparts) {
-            const float* src =
-                j == 0 ? p.x + (size_t)l * B * d
-                : j <= Hkv ? p.o_part + ((size_t)l * Hkv + (j - 1)) * B * d
-                           : p.moe_part + ((size_t)l * K + (j - 1 - Hkv)) * B * d;
-            v[u] = ldcg4(src + (size_t)b * d + col);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (j0 + u < nparts) {
-            x.x += v[u].x;
-            x.y += v[u].y;
-            x.z += v[u].z;
-            x.w += v[u].w;
-          }
-        }
-      }
-      *reinterpret_cast<float4*>(p.x + ((size_t)lv * B + b) * d + col) = x;
-      *reinterpret_cast<float4*>(rows + (size_t)b * (d + kActPad) + col) =
-          make_float4(x.x * g0, x.y * g1, x.z * g2, x.w * g3);
-      ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-    }
-    for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);   // within the half
-    if (q == 0 && b < B) ssp[r * B + b] = ss;
-  }
-}
-
-// Top-k + softmax + expert-slot compaction of layer l (one warp), from the
-// router logits: per token the k largest logits by (value descending, expert
-// ascending), weights softmax over the selected logits; the experts any token
-// selected get slots in ascending expert order, each slot listing its tokens
-// (ascending) with their rank and weight; unused slots are marked empty.
-__device__ __noinline__ void fused_topk(const Params& p, int l) {
-  const Smem sm = smem_view(p);
-  const int lane = threadIdx.x & 31;
-  const int B = p.B, E = p.E, K = p.k, S = p.S;
-  int32_t* rt = p.route + (size_t)l * p.route_words;
-  int* sel = reinterpret_cast<int*>(sm.epi + 2 * kConsumerWarps * 16 * p.part_cols * 4 +
-                                    kRstdRing * kMaxBatch * 4);   // [8][8]
-  float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [8][8] logits, then weights
-  int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8);  // [256]
-  uint32_t used = 0u;   // lane w < 8: bit e of experts 32 w + e selected by any token
-  for (int b = 0; b < B; ++b) {
-    const float* lg = p.rlogits + ((size_t)l * B + b) * E;
-    uint32_t key[8];   // order-preserving unsigned keys; 0 marks taken / absent
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int e = lane + 32 * t;
-      uint32_t k = 0u;
-      if (e < E) {
-        const uint32_t u = __float_as_uint(__ldcg(lg + e));
-        k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-      }
-      key[t] = k;
-    }
-#pragma unroll 1
-    for (int j = 0; j < K; ++j) {
-      uint32_t bk = 0u;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (key[t] > bk) {   // ascending e within a lane: first max has the smallest e
-          bk = key[t];
-          bi = lane + 32 * t;
-        }
-      }
-      const uint32_t mk = __reduce_max_sync(FULL, bk);
-      const int wi = __reduce_min_sync(FULL, bk == mk ? bi : 0x7fffffff);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-        if (lane + 32 * t == wi) key[t] = 0u;
-      if (lane == (wi >> 5)) used |= 1u << (wi & 31);
-      if (lane == 0) {
-        sel[b * 8 + j] = wi;
-        wsel[b * 8 + j] = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) {
-      // softmax over the selected logits (in place)
-      const float m0 = wsel[b * 8];
-      float sum = 0.f;
-      for (int j = 0; j < K; ++j) {
-        const float w = fexp(wsel[b * 8 + j] - m0);
-        wsel[b * 8 + j] = w;
-        sum += w;
-      }
-      const float inv = frcp(sum);
-      for (int j = 0; j < K; ++j) {
-        const float w = wsel[b * 8 + j] * inv;
-        wsel[b * 8 + j] = w;
-        rt[route_topk_idx(B, K) + b * K + j] = sel[b * 8 + j];
-        reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + j] = w;
-      }
-    }
-    __syncwarp();
-  }
-  // slot of each used expert = number of used experts below it (every lane
-  // takes all 8 words first; the per-expert loop below only reads them)
-  uint32_t words[8];
-  int below[8], n_used = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    words[w] = __shfl_sync(FULL, used, w);
-    below[w] = n_used;
-    n_used += __popc(words[w]);
-  }
-  for (int e = lane; e < E; e += 32) {
-    const int w = e >> 5;
-    uint32_t word = 0u;
-    int bw = 0;
-#pragma unroll
-    for (int w2 = 0; w2 < 8; ++w2) {
-      if (w2 == w) {
-        word = words[w2];
-        bw = below[w2];
-      }
-    }
-    const int cnt = bw + __popc(word & ((1u << (e & 31)) - 1u));
-    slot_of[e] = ((word >> (e & 31)) & 1u) ? cnt : -1;
-  }
-  for (int s2 = lane; s2 < S; s2 += 32) {
-    if (s2 >= n_used) {
-      rt[route_slot_expert(B, K) + s2] = -1;
-      rt[route_slot_ntok(B, K, S) + s2] = 0;
-    }
-  }
-  if (lane == 0) rt[0] = n_used;
-  __syncwarp();
-  // one (token, rank) pair per lane: its position in the slot's token list
-  for (int idx = lane; idx < B * K; idx += 32) {
-    const int bb = idx / K, j = idx % K;
-    const int e = sel[bb * 8 + j];
-    const int s2 = slot_of[e];
-    int pos = 0;
-    for (int b2 = 0; b2 < bb; ++b2)
-      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
-    rt[route_slot_tok(B, K, S) + s2 * 8 + pos] = bb;
-    rt[route_slot_rank(B, K, S) + s2 * 8 + pos] = j;
-    reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s2 * 8 + pos] = wsel[bb * 8 + j];
-    if (pos == 0) {
-      int cnt = 0;
-      for (int b2 = 0; b2 < B; ++b2)
-        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
-      rt[route_slot_expert(B, K) + s2] = e;
-      rt[route_slot_ntok(B, K, S) + s2] = cnt;
-    }
-  }
-}
-
 // ============================================================== epilogue ==
 // One warp follows the FIFO behind the consumers.  For a GEMV tile it waits
 // for the consumer warps' partials, reduces them, writes the outputs and
@@ -1839,10 +1843,6 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
   const int PC = p.part_cols;
   const float* part0 = reinterpret_cast<const float*>(sm.epi);
   const float* rstd_ring = part0 + 2 * kConsumerWarps * 16 * PC;
-  // router bias of the current tile: the tail of the warp's top-k scratch
-  // (the top-k join uses its first 1.5 KB)
-  float* bias_s = reinterpret_cast<float*>(sm.epi + 2 * kConsumerWarps * 16 * PC * 4 +
-                                           kRstdRing * kMaxBatch * 4 + 1536);
   uint32_t ngemv = 0;
   int nloadB = 0;
   for (int i = 0;; ++i) {
@@ -1859,30 +1859,11 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
       continue;
     }
     const int pb = (int)(ngemv & 1u);
-    if (op == OP_ROUTER) {
-      // the tile's bias values, staged while the consumers stream the tile
-      // (the pointer and the values are two dependent global loads)
-      const float* bias = p.router_bias ? p.router_bias[ent[D_LAYER]] : nullptr;
-      const int R = ent[D_R], row0 = ent[D_ROW0];
-      for (int r = lane; r < R; r += 32)
-        bias_s[r] = (bias && row0 + r < p.E) ? __ldg(bias + row0 + r) : 0.f;
-      __syncwarp();
-    }
     if (!warp_wait(p, sm.pfull(pb), (ngemv >> 1) & 1u, 601)) break;
     const int t = ent[32 + R_TASK];
     if (lane == 0) cstamp(p, t, T_K4);
     gemv_epilogue(p, ent, part0 + pb * kConsumerWarps * 16 * PC,
-                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch, bias_s);
-    const int flags = ent[D_FLAGS];
-    if (flags & (F_NORM | F_TOPK)) {
-      if (warp_arrive_last(p, ent[D_X0], ent[D_X1])) {
-        if (flags & F_NORM)
-          fused_norm(p, ent[D_LAYER] + 1, op == OP_OPROJ ? ent[D_A] : ent[D_B]);
-        else
-          fused_topk(p, ent[D_LAYER]);
-        warp_signal(p, ent[D_X2]);
-      }
-    }
+                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch);
     __syncwarp();
     if (lane == 0) {
       stamp(p, t, T_C_END);
@@ -1923,6 +1904,20 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  {
+    const Smem sm = smem_view(p);
+    const void** tab = const_cast<const void**>(sm.ptrs);
+    const int L = p.L;
+    for (int i = threadIdx.x; i < ptr_table_words(L); i += kThreads) {
+      const void* v;
+      if (i < L) v = p.attn_norm[i];
+      else if (i == L) v = p.final_norm;
+      else if (i < 2 * L + 1) v = p.router_bias ? p.router_bias[i - L - 1] : nullptr;
+      else if (i < 3 * L + 1) v = p.k_pool[i - 2 * L - 1];
+      else v = p.v_pool[i - 3 * L - 1];
+      tab[i] = v;
+    }
   }
   __syncthreads();
   if (warp == kProducerWarp) {

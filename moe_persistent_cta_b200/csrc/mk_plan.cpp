@@ -17,10 +17,11 @@
 // projection of one expert only for that expert's gate/up tiles (section
 // "Three sources of speedup", item 2).
 //
-// The order in which tasks are handed out comes from simulating the step on
-// the CTAs with a cost model (order_by_simulation): tasks are emitted when
-// the simulation would start them, preferring, among tasks whose inputs are
-// ready, the one with the longest remaining path.
+// Priority order inside a layer: the norm tiles (which also produce the
+// router logits, share by share); QKV and top-k; attention chunks (their
+// cached K/V stream before the new query exists); expert gate/up (the MoE
+// branch is the longer one); then the attention tail and the expert down
+// projections.
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
@@ -72,6 +73,7 @@ int validate_shape(const Shape& s) {
   const int r_qkv = gemv_rows_for(s.d, 1);
   if (r_qkv > s.hd || s.hd % r_qkv != 0) return MK_ERR_INVALID;
   if (s.E < 1 || s.E > 256) return MK_ERR_CAPACITY;
+  if (s.E % 4 != 0) return MK_ERR_INVALID;   // router logits summed as float4 columns
   if (s.k < 1 || s.k > kMaxTopK || s.k > s.E) return MK_ERR_INVALID;
   if (s.F < 128 || s.F % 128 != 0) return MK_ERR_INVALID;
   if (s.F % gemv_rows_for(s.d, 2) != 0) return MK_ERR_INVALID;
@@ -95,7 +97,7 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->actB_bytes = round_up(b_need, 128);
   int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
-  int sc_topk = B * s.E * 4 + B * 8 * 8 + s.E * 4 + 256;
+  int sc_topk = kTopkLogitsOff + (kMaxBatch * 256 + 1024) * 4;   // logits + group sums
   int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
   int sc_comb = 3 * max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
@@ -104,11 +106,11 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   const int max_stages = 14;
   const int bars = round_up((2 * max_stages + 4 * kFifo + 12) * 8, 1024);
   o->part_cols = B <= 2 ? B : 8;
-  const int epi = round_up(2 * kConsumerWarps * 16 * o->part_cols * 4 + kRstdRing * kMaxBatch * 4 +
-                               kTopkScratch,
+  const int epi = round_up(2 * kConsumerWarps * 16 * o->part_cols * 4 + kRstdRing * kMaxBatch * 4,
                            128);
   const int budget = 232448 - 2048;   // max per block, less alignment slack and static smem
-  int rest1 = bars + fifo + epi + o->scratch_bytes + o->actA_stride + 2 * o->actB_bytes;
+  const int ptrs = round_up(ptr_table_words(s.L) * 8, 128);
+  int rest1 = bars + fifo + epi + ptrs + o->scratch_bytes + o->actA_stride + 2 * o->actB_bytes;
   int rest2 = rest1 + o->actA_stride;
   int nA = ((budget - rest2) / kStageBytes >= 8) ? 2 : 1;
   int rest = nA == 2 ? rest2 : rest1;
@@ -123,7 +125,8 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->off_actA = o->off_scratch + o->scratch_bytes;
   o->off_actB = o->off_actA + nA * o->actA_stride;
   o->off_epi = o->off_actB + 2 * o->actB_bytes;
-  o->total = o->off_epi + epi;
+  o->off_ptrs = o->off_epi + epi;
+  o->total = o->off_ptrs + ptrs;
   o->dyn_bytes = o->total + 1024;
   return MK_OK;
 }
@@ -137,13 +140,12 @@ struct Task {
 
 struct Layout {
   int L, B, S, Hkv, NR;
-  int norm0, qkv0, rpart0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
+  int norm0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
   void build(int L_, int B_, int S_, int Hkv_, int NR_) {
     L = L_; B = B_; S = S_; Hkv = Hkv_; NR = NR_;
     int c = 0;
     norm0 = c; c += L + 1;
     qkv0 = c; c += L * Hkv;
-    rpart0 = c; c += L;
     rtr0 = c; c += L;
     attp0 = c; c += L * B * Hkv;
     atto0 = c; c += L * Hkv;
@@ -154,7 +156,6 @@ struct Layout {
   }
   int norm(int l) const { return norm0 + l; }
   int qkv(int l, int g) const { return qkv0 + l * Hkv + g; }
-  int rpart(int l) const { return rpart0 + l; }
   int rtr(int l) const { return rtr0 + l; }
   int attp(int l, int b, int g) const { return attp0 + (l * B + b) * Hkv + g; }
   int atto(int l, int g) const { return atto0 + l * Hkv + g; }
@@ -190,169 +191,9 @@ void add_signal(Task& t, int ctr) {
   t.w[D_S0 + i] = ctr;
 }
 
-// ---------------------------------------------------------------------------
-// List scheduling of the step's tasks onto n_ctas CTAs.
-//
-// The run-time dispenser hands tasks out in list order to whichever CTA asks
-// next, and each CTA runs its tasks in the order it took them, so a task
-// taken long before its inputs exist holds up everything behind it on that
-// CTA.  The list is therefore built by simulating that execution with a
-// simple cost model and emitting tasks in the order the simulation starts
-// them.  A task enters the candidate set only once every task signalling a
-// counter it waits on has been emitted, so the order is topological (the
-// condition the dispenser's deadlock freedom rests on).  Among candidates
-// whose inputs are ready when a CTA frees up, the one with the longest
-// remaining path to the end of the step goes first; if none is ready, the
-// one ready soonest.
-//
-// Cost model (microseconds): a task streams its stages at kSmGBs per SM
-// from the moment its CTA takes it (the weights do not depend on the inputs)
-// but computes only once its inputs are ready, at kComputeGBs; a fixed cost
-// per task; kHop between a signal and the waiter seeing it.
-constexpr double kSmGBs = 40.0, kComputeGBs = 80.0, kHop = 2.0;
-
-double task_bytes(const Task& t, int hd) {
-  switch (t.w[D_OP]) {
-    case OP_ATTN: return 2.0 * t.w[D_PPC] * kPage * hd * 2.0;   // K and V pages of a chunk
-    case OP_QKV: case OP_ROUTER: case OP_OPROJ: case OP_GATEUP: case OP_DOWN: case OP_LMHEAD:
-      return (double)t.w[D_NSTAGE] * kStageBytes;
-    default: return 0.0;
-  }
-}
-double task_fixed(const Task& t) {
-  switch (t.w[D_OP]) {
-    case OP_RN: return 4.5;
-    case OP_TOPK: return 4.0;
-    case OP_COMBINE: return 6.0;
-    case OP_ATTN: return 2.0;
-    default: return 1.0;
-  }
-}
-
-void order_by_simulation(std::vector<Task>& tasks, int n_counters, int n_ctas, int hd) {
-  const int n = (int)tasks.size();
-  std::vector<std::vector<int>> signallers(n_counters), waiters(n_counters);
-  auto waits_of = [&](const Task& t, int* out) {
-    int m = 0;
-    for (int w = 0; w < t.w[D_NWAIT]; ++w) out[m++] = t.w[D_W0 + 2 * w];
-    if (t.w[D_PW] >= 0) out[m++] = t.w[D_PW];
-    return m;
-  };
-  // the counters a task may signal: its signal list, and the join counter of
-  // its last-arriver group (any member may be the last)
-  auto sigs_of = [&](const Task& t, int* out) {
-    int m = 0;
-    for (int q = 0; q < t.w[D_NSIG]; ++q) out[m++] = t.w[D_S0 + q];
-    if (t.w[D_FLAGS] & (F_NORM | F_TOPK | F_COMBINE)) out[m++] = t.w[D_X2];
-    return m;
-  };
-  for (int i = 0; i < n; ++i) {
-    const Task& t = tasks[i];
-    {
-      int c[4];
-      const int m = sigs_of(t, c);
-      for (int q = 0; q < m; ++q) signallers[c[q]].push_back(i);
-    }
-    int c[4];
-    const int m = waits_of(t, c);
-    for (int q = 0; q < m; ++q) waiters[c[q]].push_back(i);
-  }
-  std::vector<double> stream(n), compute(n), fixed(n);
-  for (int i = 0; i < n; ++i) {
-    const double b = task_bytes(tasks[i], hd);
-    stream[i] = b / (kSmGBs * 1e3);
-    compute[i] = b / (kComputeGBs * 1e3);
-    fixed[i] = task_fixed(tasks[i]);
-  }
-  // remaining-path priority, from the back (the generation order is topological)
-  std::vector<double> level(n, 0.0), clevel(n_counters, 0.0);
-  for (int i = n - 1; i >= 0; --i) {
-    const Task& t = tasks[i];
-    double after = 0.0;
-    {
-      int c[4];
-      const int m = sigs_of(t, c);
-      for (int q = 0; q < m; ++q) after = std::max(after, kHop + clevel[c[q]]);
-    }
-    level[i] = stream[i] + fixed[i] + after;
-    int c[4];
-    const int m = waits_of(t, c);
-    for (int q = 0; q < m; ++q) clevel[c[q]] = std::max(clevel[c[q]], level[i]);
-  }
-  // simulation
-  std::vector<int> pending(n, 0), unsched(n_counters, 0);
-  std::vector<double> cfinish(n_counters, 0.0), ready(n, 0.0);
-  for (int c = 0; c < n_counters; ++c) unsched[c] = (int)signallers[c].size();
-  using Cand = std::pair<double, int>;
-  std::priority_queue<Cand, std::vector<Cand>, std::greater<Cand>> later;   // by ready time
-  std::priority_queue<std::pair<double, int>> now;                         // by priority
-  auto make_available = [&](int i) {
-    int c[4];
-    const int m = waits_of(tasks[i], c);
-    double r = 0.0;
-    for (int q = 0; q < m; ++q) r = std::max(r, cfinish[c[q]] + kHop);
-    ready[i] = r;
-    later.push({r, i});
-  };
-  for (int i = 0; i < n; ++i) {
-    int c[4];
-    const int m = waits_of(tasks[i], c);
-    int p = 0;
-    for (int q = 0; q < m; ++q) p += unsched[c[q]] > 0 ? 1 : 0;
-    pending[i] = p;
-    if (p == 0) make_available(i);
-  }
-  using Free = std::pair<double, int>;
-  std::priority_queue<Free, std::vector<Free>, std::greater<Free>> ctas;
-  for (int c = 0; c < n_ctas; ++c) ctas.push({0.0, c});
-  std::vector<int> order;
-  order.reserve(n);
-  while ((int)order.size() < n) {
-    const Free f = ctas.top();
-    ctas.pop();
-    const double T = f.first;
-    while (!later.empty() && later.top().first <= T) {
-      now.push({level[later.top().second], later.top().second});
-      later.pop();
-    }
-    int i;
-    if (!now.empty()) {
-      i = now.top().second;
-      now.pop();
-    } else {
-      i = later.top().second;   // nothing ready: the soonest
-      later.pop();
-    }
-    order.push_back(i);
-    const double finish = std::max(T + stream[i], ready[i] + compute[i]) + fixed[i];
-    ctas.push({finish, f.second});
-    int sc[4];
-    const int nsc = sigs_of(tasks[i], sc);
-    for (int q = 0; q < nsc; ++q) {
-      const int c = sc[q];
-      cfinish[c] = std::max(cfinish[c], finish);
-      if (--unsched[c] == 0) {
-        for (int w : waiters[c]) {
-          // one entry per listed wait, matching how pending was counted
-          if (--pending[w] == 0) make_available(w);
-        }
-      }
-    }
-  }
-  std::vector<Task> sorted;
-  sorted.reserve(n);
-  for (int i : order) sorted.push_back(tasks[i]);
-  tasks.swap(sorted);
-}
-
-// How the step's joins are scheduled and the list is ordered.
-struct PlanOptions {
-  bool fuse_norm = false;     // residual+RMSNorm in the last O-proj/down tile (else norm tasks)
-  bool fuse_topk = false;     // top-k in the last router tile (else a top-k task)
-  bool fuse_combine = true;   // attention merge in the last chunk (else combine tasks)
-  bool simulate_order = false;  // list order from order_by_simulation (else by layer, rank)
-};
-constexpr PlanOptions kPlanOptions{};
+// How the attention merge is scheduled: by the last chunk of each
+// (token, KV head) (an acquire-release arrival counter), else as combine tasks.
+constexpr bool kFuseCombine = true;
 
 }  // namespace
 
@@ -368,7 +209,6 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   const int r_qkv = gemv_rows_for(d, 1);
   const int r_ff = gemv_rows_for(d, 2);
   const int n_qkv = qkvR / r_qkv;
-  const int n_rt = (E + r_qkv - 1) / r_qkv;
   const int n_ff = F / r_ff;
   const int n_lm = (s.V + 127) / 128;
   if (r_qkv > hd || hd % r_qkv != 0) return MK_ERR_INVALID;
@@ -398,12 +238,14 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
 
 
   std::vector<Task> tasks;
-  tasks.reserve((size_t)L * (NR + n_qkv + n_rt + 1 + 2 * B * Hkv * max_chunks + NR * Hkv +
+  tasks.reserve((size_t)L * (NR + n_qkv + 1 + 2 * B * Hkv * max_chunks + NR * Hkv +
                              S * (n_ff + NR)) + NR + n_lm + 16);
   const int PH = 8;  // phases per layer
   auto map_of = [&](int l, int which) { return l * kMapsPerLayer + which; };
 
-  const PlanOptions opt = kPlanOptions;
+  // a task that also performs the join it completes: it arrives on
+  // arrive_ctr, and the last of `arrivals` arrivals runs the joined work and
+  // signals join_ctr
   auto fuse = [&](Task& t, int flag, int arrive_ctr, int arrivals, int join_ctr) {
     t.w[D_FLAGS] |= flag;
     t.w[D_X0] = arrive_ctr;
@@ -411,12 +253,18 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
     t.w[D_X2] = join_ctr;
     targets[arrive_ctr] += 1;
   };
-  // norm tiles producing level l: every level without fused norms, else the
-  // embedding level only (later levels: the last O-proj/down tile, F_NORM)
+  // residual add + RMSNorm tiles producing level l; a tile of a level that
+  // feeds a layer also computes its 64 columns' share of that layer's router
+  // logits (W_r[:, tile] . gamma x), its router columns streamed through the
+  // ring like GEMV weights: one stage per 128 experts
   auto emit_norm = [&](int l) {
     for (int r = 0; r < NR; ++r) {
       Task t = make_task(OP_RN, l, l * PH + 0);
       t.w[D_A] = r;
+      if (l < L) {
+        t.w[D_NSTAGE] = (E + kRouterRowsPerStage - 1) / kRouterRowsPerStage;
+        t.w[D_MAP0] = map_of(l, kMapRouter);
+      }
       if (l > 0) add_wait(t, lay.dt(l - 1, r), Hkv + S);
       add_signal(t, lay.norm(l));
       targets[lay.norm(l)] += 1;
@@ -425,31 +273,11 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   };
   emit_norm(0);
   for (int l = 0; l < L; ++l) {
-    if (l > 0 && !opt.fuse_norm) emit_norm(l);
-    // -- router tiles
-    for (int t_i = 0; t_i < n_rt; ++t_i) {
-      Task t = make_task(OP_ROUTER, l, l * PH + 1);
-      t.w[D_A] = t_i;
-      t.w[D_ROW0] = t_i * r_qkv;
-      t.w[D_K0] = 0;
-      t.w[D_KCH] = d / 64;
-      t.w[D_R] = r_qkv;
-      t.w[D_NMAT] = 1;
-      t.w[D_MAP0] = map_of(l, 2);
-      t.w[D_NSTAGE] = (r_qkv / 16) * (d / 64) / 8;
-      add_wait(t, lay.norm(l), NR);
-      if (opt.fuse_topk) {
-        fuse(t, F_TOPK, lay.rpart(l), n_rt, lay.rtr(l));
-      } else {
-        add_signal(t, lay.rpart(l));
-        targets[lay.rpart(l)] += 1;
-      }
-      t.w[D_ACT] = ACT_A;
-      tasks.push_back(t);
-    }
-    if (!opt.fuse_topk) {
+    if (l > 0) emit_norm(l);
+    // -- top-k over the router logits summed from the norm tiles' shares
+    {
       Task t = make_task(OP_TOPK, l, l * PH + 2);
-      add_wait(t, lay.rpart(l), n_rt);
+      add_wait(t, lay.norm(l), NR);
       add_signal(t, lay.rtr(l));
       tasks.push_back(t);
     }
@@ -497,7 +325,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
           add_wait(t, lay.qkv(l, g), (G * hd + 2 * hd) / r_qkv);
           if (nc == 1) {
             add_signal(t, lay.atto(l, g));
-          } else if (opt.fuse_combine) {
+          } else if (kFuseCombine) {
             fuse(t, F_COMBINE, lay.attp(l, b, g), nc, lay.atto(l, g));
           } else {
             add_signal(t, lay.attp(l, b, g));
@@ -511,7 +339,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         }
       }
     }
-    if (!opt.fuse_combine) {
+    if (!kFuseCombine) {
       for (int g = 0; g < Hkv; ++g) {
         for (int b = 0; b < B; ++b) {
           if (out->nc[b] <= 1) continue;
@@ -540,12 +368,8 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         t.w[D_MAP0] = map_of(l, 1);
         t.w[D_NSTAGE] = 4 * (G * hd / 64) / 8;
         add_wait(t, lay.atto(l, g), B);
-        if (opt.fuse_norm) {
-          fuse(t, F_NORM, lay.dt(l, r), Hkv + S, lay.norm(l + 1));
-        } else {
-          add_signal(t, lay.dt(l, r));
-          targets[lay.dt(l, r)] += 1;
-        }
+        add_signal(t, lay.dt(l, r));
+        targets[lay.dt(l, r)] += 1;
         t.w[D_ACT] = ACT_B;
         tasks.push_back(t);
       }
@@ -588,22 +412,14 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         t.w[D_PW] = lay.rtr(l);
         t.w[D_PWN] = 1;
         add_wait(t, lay.slot(l, j), n_ff);
-        if (opt.fuse_norm) {
-          fuse(t, F_NORM, lay.dt(l, r), Hkv + S, lay.norm(l + 1));
-        } else {
-          add_signal(t, lay.dt(l, r));
-          targets[lay.dt(l, r)] += 1;
-        }
+        add_signal(t, lay.dt(l, r));
+        targets[lay.dt(l, r)] += 1;
         t.w[D_ACT] = ACT_B;
         tasks.push_back(t);
       }
     }
   }
-  if (opt.fuse_norm) {
-    for (int l = 1; l <= L; ++l) targets[lay.norm(l)] += NR;   // one per 64-column tile
-  } else {
-    emit_norm(L);   // the final norm
-  }
+  emit_norm(L);   // the final norm
   // -- LM head
   for (int t_i = 0; t_i < n_lm; ++t_i) {
     Task t = make_task(OP_LMHEAD, L, L * PH + 1);
@@ -622,20 +438,14 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
     tasks.push_back(t);
   }
 
-  // ---- dispensing order: list scheduling over a cost model (see
-  // order_by_simulation), or by (layer, operation rank); either is a
-  // topological order of the tasks.
-  if (opt.simulate_order) {
-    order_by_simulation(tasks, lay.total, n_ctas, hd);
-  } else {
-    static const int kRank[OP_COUNT] = {
-        /*NONE*/ 99, /*RN*/ 0, /*QKV*/ 2, /*ROUTER*/ 1, /*TOPK*/ 3, /*ATTN*/ 4,
-        /*COMBINE*/ 6, /*OPROJ*/ 7, /*GATEUP*/ 5, /*DOWN*/ 8, /*LMHEAD*/ 9};
-    std::stable_sort(tasks.begin(), tasks.end(), [](const Task& x, const Task& y) {
-      if (x.w[D_LAYER] != y.w[D_LAYER]) return x.w[D_LAYER] < y.w[D_LAYER];
-      return kRank[x.w[D_OP]] < kRank[y.w[D_OP]];
-    });
-  }
+  // ---- priority order: stable sort by (layer, operation rank)
+  static const int kRank[OP_COUNT] = {
+      /*NONE*/ 99, /*RN*/ 0, /*QKV*/ 2, /*ROUTER*/ 1, /*TOPK*/ 3, /*ATTN*/ 4,
+      /*COMBINE*/ 6, /*OPROJ*/ 7, /*GATEUP*/ 5, /*DOWN*/ 8, /*LMHEAD*/ 9};
+  std::stable_sort(tasks.begin(), tasks.end(), [](const Task& x, const Task& y) {
+    if (x.w[D_LAYER] != y.w[D_LAYER]) return x.w[D_LAYER] < y.w[D_LAYER];
+    return kRank[x.w[D_OP]] < kRank[y.w[D_OP]];
+  });
   // A-slot double buffering where two buffers fit in shared memory
   SmemLayout sl;
   int slrc = smem_layout(s, B, max_chunks, &sl);

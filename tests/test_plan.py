@@ -25,8 +25,8 @@ ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 
 D_X0, D_X1, D_X2 = 29, 30, 31
-F_NORM, F_TOPK, F_COMBINE = 32, 64, 128
-FUSED = F_NORM | F_TOPK | F_COMBINE
+F_COMBINE = 128
+FUSED = F_COMBINE
 
 
 def signal_sets(desc, targets):
@@ -113,20 +113,18 @@ def test_30b_b1_plan_structure():
     L, d = shape["n_layers"], shape["d_model"]
     qkv_rows = (shape["n_q_heads"] + 2 * shape["n_kv_heads"]) * shape["head_dim"]
     assert ops[OP_QKV] == L * qkv_rows // 16
-    assert ops[OP_ROUTER] == L * shape["n_experts"] // 16
-    # each join is done one way or the other, never both: as its own tasks,
-    # or by the last-arriving producer tile of its group
-    fl = desc[:, D_FLAGS]
-
-    def all_or_none(op, flag):
-        f = fl[desc[:, D_OP] == op] & flag
-        assert np.all(f) or not np.any(f)
-        return bool(np.all(f))
-
-    fused_norm = all_or_none(OP_OPROJ, F_NORM)
-    assert all_or_none(OP_DOWN, F_NORM) == fused_norm
-    assert ops[OP_RN] == (1 if fused_norm else L + 1) * d // 64
-    assert ops[OP_TOPK] == (0 if all_or_none(OP_ROUTER, F_TOPK) else L)
+    # the norm tiles produce the router logits: no router tiles, and each
+    # layer's top-k waits for all of the layer's norm tiles
+    assert ops[OP_ROUTER] == 0
+    assert ops[OP_RN] == (L + 1) * d // 64
+    assert ops[OP_TOPK] == L
+    tk = desc[desc[:, D_OP] == OP_TOPK]
+    assert np.all(tk[:, D_NWAIT] == 1) and np.all(tk[:, D_W0N] == d // 64)
+    rn = desc[desc[:, D_OP] == OP_RN]
+    for l in (0, 5):
+        ctr = tk[tk[:, D_LAYER] == l][0, D_W0]
+        senders = rn[(rn[:, D_LAYER] == l)]
+        assert np.all(senders[:, D_S0] == ctr) and len(senders) == d // 64
     a_multi = desc[(desc[:, D_OP] == OP_ATTN) & (desc[:, D_D] > 1)]
     assert len(a_multi)
     fused_comb = bool(np.all(a_multi[:, D_FLAGS] & F_COMBINE))
@@ -143,8 +141,7 @@ def test_30b_b1_plan_structure():
     nc, ppc = a[0, D_D], a[0, D_PPC]
     assert nc * ppc * 64 >= 8192 + 64
     assert len(a) == L * shape["n_kv_heads"] * nc
-    # the dispensing order comes from a simulation, but each layer still ends
-    # with tiles feeding the next norm
+    # each layer ends with tiles feeding the next norm
     for l in (0, 3, 47):
         ops = desc[desc[:, D_LAYER] == l][:, D_OP]
         assert ops[-1] in (OP_OPROJ, OP_DOWN)
@@ -171,7 +168,7 @@ def test_activation_levels_never_decrease():
         meta, desc, targets = engine.plan_schedule(shape, 148, lens)
         a = desc[desc[:, D_ACT] == ACT_A]
         assert np.all(np.diff(a[:, D_LAYER]) >= 0)
-        assert set(desc[desc[:, D_ACT] == ACT_A][:, D_OP]) <= {OP_QKV, OP_ROUTER, OP_GATEUP, OP_LM}
+        assert set(desc[desc[:, D_ACT] == ACT_A][:, D_OP]) <= {OP_QKV, OP_GATEUP, OP_LM}
         assert set(desc[desc[:, D_ACT] == ACT_B][:, D_OP]) <= {OP_ATTN, OP_OPROJ, OP_DOWN}
 
 
@@ -180,7 +177,7 @@ def test_gemv_tiles_fill_whole_stages():
     of 2 KB, a multiple of 8 per stage."""
     for shape in (configs.TINY, configs.MOE30B):
         meta, desc, targets = engine.plan_schedule(shape, 148, [100])
-        g = desc[np.isin(desc[:, D_OP], [OP_QKV, OP_ROUTER, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM])]
+        g = desc[np.isin(desc[:, D_OP], [OP_QKV, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_LM])]
         units = g[:, D_NMAT] * (g[:, D_R] // 16) * g[:, D_KCH]
         assert np.all(units % 8 == 0)
         assert np.all(units // 8 == g[:, D_NSTAGE])
@@ -196,3 +193,5 @@ def test_invalid_shapes_rejected():
         engine.plan_schedule(configs.TINY, 148, [10] * 9)      # batch > 8
     with pytest.raises(mk.MKError):
         engine.plan_schedule(configs.TINY, 148, [-1])
+    with pytest.raises(mk.MKError):
+        engine.plan_schedule(dict(configs.TINY, n_experts=10, top_k=2), 148, [10])   # E % 4
