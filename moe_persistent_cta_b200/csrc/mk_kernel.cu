@@ -640,6 +640,11 @@ __device__ __noinline__ void loader_loop(const Params& p) {
   const int lane = threadIdx.x & 31;
   int curA = -1, nloadA = 0, nloadB = 0;
   const int nA = p.nA;
+  // lane w: the last counter its wait slot saw reach a target this step (the
+  // counters only grow within a step, so a later wait on the same counter
+  // for no more arrivals needs no load)
+  int seen_ctr = -1;
+  uint32_t seen_tgt = 0;
   for (int i = 0;; ++i) {
     const int e = i % kFifo;
     if (!warp_wait(p, sm.posted(e), (i / kFifo) & 1, 200)) break;
@@ -659,7 +664,11 @@ __device__ __noinline__ void loader_loop(const Params& p) {
     if (lane < nwait) {
       const int ctr = ent[D_W0 + 2 * lane];
       const uint32_t tgt = p.epoch * (uint32_t)ent[D_W0N + 2 * lane];
-      ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
+      if (ctr != seen_ctr || tgt > seen_tgt) {
+        ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
+        seen_ctr = ctr;
+        seen_tgt = tgt;
+      }
     }
     ok = __all_sync(FULL, ok);
     if (!ok) break;
