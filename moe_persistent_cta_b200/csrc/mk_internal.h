@@ -43,6 +43,7 @@ constexpr int kMapRouter = 2;
 constexpr int kActPad = 8;
 constexpr int kRnStage = 4096;       // floats of residual partials staged per round
 constexpr int kRouterRowsPerStage = 128;   // router weight rows (x 64 columns) per ring stage
+constexpr int kMaxAttnOut = 512;    // G x hd floats of one (token, KV head) output (G <= 4, hd <= 128)
 constexpr int kTopkLogitsOff = 2048; // top-k scratch: selection state, then logits [B][E]
 // Per-layer pointer table in shared memory: norm weights of levels 0..L (the
 // final norm last), then router bias, K pool and V pool of layers 0..L-1.  A
@@ -82,7 +83,7 @@ enum Op : int32_t {
   OP_ROUTER = 3,    // (unused: the norm tiles produce the router logits)
   OP_TOPK = 4,      // top-k + softmax + expert-slot compaction
   OP_ATTN = 5,      // paged GQA decode attention over one KV chunk (+RoPE, append)
-  OP_COMBINE = 6,   // log-sum-exp merge of the chunk partials of (b, g)
+  OP_COMBINE = 6,   // (unused: the last-arriving attention chunk of (b, g) merges)
   OP_OPROJ = 7,     // O-proj tile, split-K by KV group
   OP_GATEUP = 8,    // expert gate+up tile with SwiGLU epilogue
   OP_DOWN = 9,      // expert down tile with weighted scatter into rank slots

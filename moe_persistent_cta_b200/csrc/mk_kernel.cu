@@ -1271,10 +1271,10 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     if (single) {
       osm[idx] = O * frcp(Lsum);
     } else {
-      part[2 * G + idx] = O;
+      part[idx] = O;   // chunk record: [O (G x hd)][m (G)][l (G)]
       if (i == 0) {
-        part[h] = M;
-        part[G + h] = Lsum;
+        part[G * HD + h] = M;
+        part[G * HD + G + h] = Lsum;
       }
     }
   }
@@ -1291,16 +1291,18 @@ __device__ __forceinline__ void combine_task(const Params& p, const int32_t* ent
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], nc = ent[D_D];
-  const int G = p.G, hd = p.hd, PS = p.part_stride;
+  const int G = p.G, hd = p.hd, PS = p.part_stride, GH = G * hd;
+  // chunk records [O (G x hd)][m (G)][l (G)], PS floats apart
   const float* parts =
       p.attn_part + (((size_t)layer * p.B + b) * p.Hkv + g) * p.max_chunks * (size_t)PS;
-  float* msm = reinterpret_cast<float*>(sm.scratch);  // [nc][G] chunk maxima
-  float* lsm = msm + p.max_chunks * G;                // [nc][G] chunk sums
-  float* wsm = lsm + p.max_chunks * G;                // [nc][G] merge weights
-  float* ML = wsm + p.max_chunks * G;                 // [2][G]
-  float* osm = ML + 2 * G;                            // [G][hd]
+  float4* gsum = reinterpret_cast<float4*>(sm.scratch);   // [nCG][GH / 4] group sums
+  float* osm = reinterpret_cast<float*>(gsum + 256);      // [G][hd]
+  float* msm = osm + kMaxAttnOut;                         // [nc][G] chunk maxima
+  float* lsm = msm + p.max_chunks * G;                    // [nc][G] chunk sums
+  float* wsm = lsm + p.max_chunks * G;                    // [nc][G] merge weights
+  float* ML = wsm + p.max_chunks * G;                     // [2][G]
   for (int t = ct; t < nc * G; t += 256) {
-    const float* pp = parts + (size_t)(t / G) * PS;
+    const float* pp = parts + (size_t)(t / G) * PS + GH;
     msm[t] = __ldcg(pp + t % G);
     lsm[t] = __ldcg(pp + G + t % G);
   }
@@ -1321,21 +1323,47 @@ __device__ __forceinline__ void combine_task(const Params& p, const int32_t* ent
   cbar();
   for (int t = ct; t < nc * G; t += 256) wsm[t] = ex2(msm[t] - ML[t % G]) * ML[G + t % G];
   cbar();
-  for (int idx = ct; idx < G * hd; idx += 256) {
-    const int h = idx / hd;
-    const float* pp = parts + 2 * G + idx;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    int ch = 0;
-    for (; ch + 4 <= nc; ch += 4) {
-      const float v0 = __ldcg(pp + (size_t)ch * PS), v1 = __ldcg(pp + (size_t)(ch + 1) * PS);
-      const float v2 = __ldcg(pp + (size_t)(ch + 2) * PS), v3 = __ldcg(pp + (size_t)(ch + 3) * PS);
-      o0 += wsm[ch * G + h] * v0;
-      o1 += wsm[(ch + 1) * G + h] * v1;
-      o2 += wsm[(ch + 2) * G + h] * v2;
-      o3 += wsm[(ch + 3) * G + h] * v3;
+  // thread (group cg, float4 column c4) sums chunks cg, cg + nCG, ... of its
+  // four outputs with eight loads in flight; the groups are added in cg order
+  const int C4 = GH / 4, nCG = 256 / C4;
+  if (ct < nCG * C4) {
+    const int cg = ct / C4, c4 = ct - cg * C4, h = (4 * c4) / hd;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int ch0 = cg; ch0 < nc; ch0 += 8 * nCG) {
+      float4 v[8];
+      float w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int ch = ch0 + j * nCG;
+        const bool on = ch < nc;
+        v[j] = on ? __ldcg(reinterpret_cast<const float4*>(parts + (size_t)ch * PS) + c4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        w[j] = on ? wsm[ch * G + h] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        acc.x = fmaf(w[j], v[j].x, acc.x);
+        acc.y = fmaf(w[j], v[j].y, acc.y);
+        acc.z = fmaf(w[j], v[j].z, acc.z);
+        acc.w = fmaf(w[j], v[j].w, acc.w);
+      }
     }
-    for (; ch < nc; ++ch) o0 += wsm[ch * G + h] * __ldcg(pp + (size_t)ch * PS);
-    osm[idx] = (o0 + o1) + (o2 + o3);
+    gsum[cg * C4 + c4] = acc;
+  }
+  cbar();
+#pragma unroll 1
+  for (int c4 = ct; c4 < C4; c4 += 256) {
+    float4 o = gsum[c4];
+#pragma unroll 1
+    for (int cg = 1; cg < nCG; ++cg) {
+      const float4 v = gsum[cg * C4 + c4];
+      o.x += v.x;
+      o.y += v.y;
+      o.z += v.z;
+      o.w += v.w;
+    }
+    reinterpret_cast<float4*>(osm)[c4] = o;
   }
   cbar();
   write_attn_out(p, layer, b, g, osm);
@@ -1806,9 +1834,6 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
         break;
       case OP_TOPK:
         topk_task(p, ent);
-        break;
-      case OP_COMBINE:
-        combine_task(p, ent);
         break;
       default:  // OP_ATTN
         if (p.hd == 128)

@@ -99,7 +99,7 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
   int sc_topk = kTopkLogitsOff + (kMaxBatch * 256 + 1024) * 4;   // logits + group sums
   int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
-  int sc_comb = 3 * max_chunks * G * 4 + 2 * G * 4 + G * s.hd * 4 + 256;
+  int sc_comb = 256 * 16 + kMaxAttnOut * 4 + 3 * max_chunks * G * 4 + 2 * G * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
   o->scratch_bytes = round_up(sc, 1024);
   const int fifo = kFifo * kFifoEntryWords * 4;
@@ -191,9 +191,6 @@ void add_signal(Task& t, int ctr) {
   t.w[D_S0 + i] = ctr;
 }
 
-// How the attention merge is scheduled: by the last chunk of each
-// (token, KV head) (an acquire-release arrival counter), else as combine tasks.
-constexpr bool kFuseCombine = true;
 
 }  // namespace
 
@@ -323,32 +320,16 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
           if (c == nc - 1) t.w[D_FLAGS] |= F_LAST_CHUNK;
           if (nc == 1) t.w[D_FLAGS] |= F_SINGLE;
           add_wait(t, lay.qkv(l, g), (G * hd + 2 * hd) / r_qkv);
-          if (nc == 1) {
+          // the attention merge of (b, g) is done by the chunk whose arrival
+          // completes the (b, g) count (an acquire-release arrival counter)
+          if (nc == 1)
             add_signal(t, lay.atto(l, g));
-          } else if (kFuseCombine) {
+          else
             fuse(t, F_COMBINE, lay.attp(l, b, g), nc, lay.atto(l, g));
-          } else {
-            add_signal(t, lay.attp(l, b, g));
-            targets[lay.attp(l, b, g)] += 1;
-          }
           long p0 = (long)c * out->ppc[b];
           long pages_now = ((long)seq_lens[b] + kPage - 1) / kPage;
           long np = std::max(0L, std::min((long)out->ppc[b], pages_now - p0));
           t.w[D_ACT] = ACT_B;
-          tasks.push_back(t);
-        }
-      }
-    }
-    if (!kFuseCombine) {
-      for (int g = 0; g < Hkv; ++g) {
-        for (int b = 0; b < B; ++b) {
-          if (out->nc[b] <= 1) continue;
-          Task t = make_task(OP_COMBINE, l, l * PH + 4);
-          t.w[D_A] = b;
-          t.w[D_B] = g;
-          t.w[D_D] = out->nc[b];
-          add_wait(t, lay.attp(l, b, g), out->nc[b]);
-          add_signal(t, lay.atto(l, g));
           tasks.push_back(t);
         }
       }
