@@ -721,6 +721,8 @@ __device__ __noinline__ void loader_loop(const Params& p) {
           mbar_expect_tx(fb, (uint32_t)p.ofrag_bytes);
           bulk_g2s(dst, p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes,
                    (uint32_t)p.ofrag_bytes, fb);
+        } else if (ent[32 + R_EXPERT] < 0) {   // OP_DOWN of an empty slot: nothing to copy
+          mbar_arrive(fb);
         } else {  // OP_DOWN
           const int j = a;
           mbar_expect_tx(fb, (uint32_t)p.afrag_bytes);
@@ -996,7 +998,6 @@ __device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* en
   const int PC = p.part_cols;
   const bool expert = (op == OP_GATEUP || op == OP_DOWN);
   const int ncols = expert ? ent[32 + R_NTOK] : p.B;
-  if (expert && ent[32 + R_EXPERT] < 0) return;   // empty slot
   const int n_out = R * ncols;
   for (int idx = lane; idx < n_out; idx += 32) {
     const int n = idx / R, r = idx - n * R;   // r fastest: coalesced output rows
@@ -1795,17 +1796,16 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
     const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
 
     if (gemv) {
+      // an empty expert slot: nothing streamed or computed; the epilogue warp
+      // completes it without a partials buffer
+      if ((op == OP_GATEUP || op == OP_DOWN) && ent[32 + R_EXPERT] < 0) continue;
       const int pb = (int)(ngemv & 1u);
       const uint32_t pe_par = ((ngemv >> 1) & 1u) ^ 1u;
       float* pw = part0 + (pb * kConsumerWarps + cw) * 16 * PC;
       const float* a;
       int stride, ncols = p.B;
       const int32_t* tokmap = nullptr;
-      bool skip = false;
-      if (op == OP_GATEUP || op == OP_DOWN) {
-        ncols = ent[32 + R_NTOK];
-        skip = ent[32 + R_EXPERT] < 0;   // empty slot: nothing streamed
-      }
+      if (op == OP_GATEUP || op == OP_DOWN) ncols = ent[32 + R_NTOK];
       if (op == OP_OPROJ) {
         a = reinterpret_cast<const float*>(actB);
         stride = p.G * p.hd + kActPad;
@@ -1817,11 +1817,8 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
         stride = p.d + kActPad;
         if (op == OP_GATEUP) tokmap = ent + 32 + R_TOK;
       }
-      if (skip)
-        wait_bar(p, sm.pempty(pb), pe_par, 403);
-      else
-        stage_ctr = gemv_consume(p, ent, a, stride, tokmap, ncols, pw, sm.pempty(pb), pe_par,
-                                 stage_ctr);
+      stage_ctr = gemv_consume(p, ent, a, stride, tokmap, ncols, pw, sm.pempty(pb), pe_par,
+                               stage_ctr);
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.pfull(pb));
       ++ngemv;
@@ -1890,6 +1887,18 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
       if (act == ACT_B) ++nloadB;
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.fempty(e));
+      continue;
+    }
+    if ((op == OP_GATEUP || op == OP_DOWN) && ent[32 + R_EXPERT] < 0) {
+      // an empty expert slot (the consumers skipped it): complete the task
+      __syncwarp();
+      if (lane == 0) {
+        if (act == ACT_B) mbar_arrive(sm.aemptyB(nloadB & 1));
+        mbar_arrive(sm.done(e));
+        mbar_arrive(sm.fempty(e));
+      }
+      __syncwarp();
+      if (act == ACT_B) ++nloadB;
       continue;
     }
     const int pb = (int)(ngemv & 1u);
