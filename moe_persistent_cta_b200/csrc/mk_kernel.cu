@@ -948,6 +948,7 @@ __device__ __forceinline__ void gemv_stages_mma(const Params& p, const Smem& sm,
 // ncols read row 0 and are ignored by the epilogue.  Each warp streams its
 // own 16-row unit of every stage and leaves its partial sums in `pw`
 // ([16][part_cols]); the epilogue warp reduces the warps' partials.
+template <int NBK>
 __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t* ent,
                                                  const float* act, int stride,
                                                  const int32_t* tokmap, int ncols, float* pw,
@@ -966,10 +967,10 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
   uint32_t waitcyc = 0;
   if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K2);
   const uint64_t l0 = clock64();
-  if (p.B == 1) {
+  if constexpr (NBK == 1) {
     gemv_stages_ffma<1>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4, 0, ring, pw,
                         pe_bar, pe_par, waitcyc);
-  } else if (p.B == 2) {
+  } else if constexpr (NBK == 2) {
     gemv_stages_ffma<2>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4,
                         xbase + row_of(1) * stride * 4, ring, pw, pe_bar, pe_par, waitcyc);
   } else {
@@ -1729,6 +1730,10 @@ __device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
   }
 }
 
+// NBK: the GEMV path (1 and 2: FFMA for 1 or 2 tokens; 3: mma.sync for 3..8);
+// HD: the head dimension.  Each launch runs the instantiation of its batch and
+// shape, so its consumer code holds one GEMV path and one attention routine.
+template <int NBK, int HD>
 __device__ __noinline__ void consumer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
@@ -1817,7 +1822,7 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
         stride = p.d + kActPad;
         if (op == OP_GATEUP) tokmap = ent + 32 + R_TOK;
       }
-      stage_ctr = gemv_consume(p, ent, a, stride, tokmap, ncols, pw, sm.pempty(pb), pe_par,
+      stage_ctr = gemv_consume<NBK>(p, ent, a, stride, tokmap, ncols, pw, sm.pempty(pb), pe_par,
                                stage_ctr);
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.pfull(pb));
@@ -1833,10 +1838,7 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
         topk_task(p, ent);
         break;
       default:  // OP_ATTN
-        if (p.hd == 128)
-          stage_ctr = attn_task<128>(p, ent, actB, stage_ctr);
-        else
-          stage_ctr = attn_task<64>(p, ent, actB, stage_ctr);
+        stage_ctr = attn_task<HD>(p, ent, actB, stage_ctr);
         if (ent[D_FLAGS] & F_COMBINE) {
           // the chunk that completes (b, g) merges all its chunks' partials
           cbar();
@@ -1922,6 +1924,7 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
   }
 }
 
+template <int NBK, int HD>
 __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__ Params p) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -1972,7 +1975,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
   } else if (warp == kEpilogueWarp) {
     epilogue_loop(p);
   } else {
-    consumer_loop(p);
+    consumer_loop<NBK, HD>(p);
   }
   __syncthreads();
 }
@@ -1982,25 +1985,56 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
 // Launch one step (or one phase) of the interpreter: cooperative, so that all
 // CTAs are guaranteed co-resident (the counter waits and the dispenser rely
 // on it).
+namespace {
+// the kernel instantiation for a batch size and head dimension, and the
+// dynamic shared memory it was last configured for
+struct KernelSlot {
+  const void* fn;
+  int configured_bytes;
+};
+KernelSlot g_kernels[3][2] = {
+    {{reinterpret_cast<const void*>(mk_interp<1, 64>), -1},
+     {reinterpret_cast<const void*>(mk_interp<1, 128>), -1}},
+    {{reinterpret_cast<const void*>(mk_interp<2, 64>), -1},
+     {reinterpret_cast<const void*>(mk_interp<2, 128>), -1}},
+    {{reinterpret_cast<const void*>(mk_interp<3, 64>), -1},
+     {reinterpret_cast<const void*>(mk_interp<3, 128>), -1}}};
+KernelSlot& kernel_for(int B, int hd) {
+  return g_kernels[B <= 1 ? 0 : (B == 2 ? 1 : 2)][hd == 128 ? 1 : 0];
+}
+}  // namespace
+
 cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream) {
-  static int configured_bytes = -1;
-  if (configured_bytes != p.smem_bytes) {
+  KernelSlot& k = kernel_for(p.B, p.hd);
+  if (k.configured_bytes != p.smem_bytes) {
     cudaError_t e =
-        cudaFuncSetAttribute(mk_interp, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+        cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
-    configured_bytes = p.smem_bytes;
+    k.configured_bytes = p.smem_bytes;
   }
   void* args[] = {const_cast<Params*>(&p)};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(mk_interp), dim3(grid),
-                                     dim3(kThreads), args, (size_t)p.smem_bytes, stream);
+  return cudaLaunchCooperativeKernel(k.fn, dim3(grid), dim3(kThreads), args, (size_t)p.smem_bytes,
+                                     stream);
 }
 
+// Co-resident CTAs per SM at this shared-memory size; every instantiation is
+// checked, as each carries its own register count.
 cudaError_t max_coresident(int smem_bytes, int* blocks_per_sm) {
-  cudaError_t e =
-      cudaFuncSetAttribute(mk_interp, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-  if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, mk_interp, kThreads,
-                                                       (size_t)smem_bytes);
+  int best = 1 << 30;
+  for (auto& row : g_kernels) {
+    for (KernelSlot& k : row) {
+      cudaError_t e =
+          cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+      if (e != cudaSuccess) return e;
+      k.configured_bytes = smem_bytes;
+      int n = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k.fn, kThreads, (size_t)smem_bytes);
+      if (e != cudaSuccess) return e;
+      best = n < best ? n : best;
+    }
+  }
+  *blocks_per_sm = best;
+  return cudaSuccess;
 }
 
 }  // namespace mk
