@@ -58,7 +58,8 @@ typedef enum mk_status {
 
 /* Model shape.  Requirements (checked by mk_create): head_dim in {64, 128};
  * d_model, d_ff multiples of 64 with d_model / 64 <= 64 tiles; n_q_heads a
- * multiple of n_kv_heads; n_q_heads / n_kv_heads <= 4; n_experts <= 256;
+ * multiple of n_kv_heads; n_q_heads / n_kv_heads <= 4; n_experts <= 256 and
+ * a multiple of 4 (the router logits are summed as float4 columns);
  * top_k <= 8; page_size == 64; max_batch in [1, 8].  n_pages is the number
  * of physical pages in each layer's K and V pool.                           */
 typedef struct mk_config {
