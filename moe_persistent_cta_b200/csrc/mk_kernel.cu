@@ -1506,47 +1506,52 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
   if (nst == 0) return stage_ctr;
   cbar();
   float* out = p.rpart + ((size_t)l * p.NR + r) * B * p.E;
-  auto unit = [&](int e, int ch, bool valid, const uint4 w) {
-    const float wf[8] = {lo_bf16(w.x), hi_bf16(w.x), lo_bf16(w.y), hi_bf16(w.y),
-                         lo_bf16(w.z), hi_bf16(w.z), lo_bf16(w.w), hi_bf16(w.w)};
-    float mine = 0.f;
-#pragma unroll 1
-    for (int b = 0; b < B; ++b) {   // uniform: every lane takes part in the shuffles
-      const float4 g0 = reinterpret_cast<const float4*>(gxs + b * 64 + ch * 8)[0];
-      const float4 g1 = reinterpret_cast<const float4*>(gxs + b * 64 + ch * 8)[1];
-      float a = wf[0] * g0.x;
-      a = fmaf(wf[1], g0.y, a);
-      a = fmaf(wf[2], g0.z, a);
-      a = fmaf(wf[3], g0.w, a);
-      a = fmaf(wf[4], g1.x, a);
-      a = fmaf(wf[5], g1.y, a);
-      a = fmaf(wf[6], g1.z, a);
-      a = fmaf(wf[7], g1.w, a);
-      a += __shfl_xor_sync(FULL, a, 4);
-      a += __shfl_xor_sync(FULL, a, 2);
-      a += __shfl_xor_sync(FULL, a, 1);
-      if (b == ch) mine = a;
-    }
-    if (valid && ch < B) out[(size_t)ch * p.E + e] = mine;
-  };
+  // thread pair per expert row: half hf takes columns 32 hf .. 32 hf + 31
+  // (four 16-byte units, four independent FMA chains); the pair adds its two
+  // sums by one shuffle and half hf stores the tokens b with b % 2 == hf
 #pragma unroll 1
   for (int s = 0; s < nst; ++s) {
     const uint32_t slot = stage_ctr % (uint32_t)sm.NS, ph = (stage_ctr / (uint32_t)sm.NS) & 1u;
     wait_bar(p, sm.full(slot), ph, 404);
     const uint8_t* wt = sm.ring + (size_t)slot * kStageBytes;
     const int e0 = kRouterRowsPerStage * s;
-    const int nu = min(kRouterRowsPerStage, p.E - e0) * 8;   // units in this stage
-#pragma unroll 1
-    for (int u0 = 0; u0 < nu; u0 += 256) {                    // uniform trip count
-      const int u = u0 + ct, el = u >> 3, ch = u & 7;
-      const bool valid = u < nu;
-      const uint4 w = valid ? *reinterpret_cast<const uint4*>(wt + el * 128 + ((ch ^ (el & 7)) << 4))
+    const int rows = min(kRouterRowsPerStage, p.E - e0);   // expert rows in this stage
+    const int el = ct >> 1, hf = ct & 1;
+    const bool valid = el < rows;                          // warp-uniform when rows % 16 == 0
+    float wf[32];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = valid ? *reinterpret_cast<const uint4*>(
+                                  wt + el * 128 + (((4 * hf + k) ^ (el & 7)) << 4))
                             : make_uint4(0u, 0u, 0u, 0u);
-      unit(e0 + el, ch, valid, w);
+      wf[8 * k + 0] = lo_bf16(w.x);
+      wf[8 * k + 1] = hi_bf16(w.x);
+      wf[8 * k + 2] = lo_bf16(w.y);
+      wf[8 * k + 3] = hi_bf16(w.y);
+      wf[8 * k + 4] = lo_bf16(w.z);
+      wf[8 * k + 5] = hi_bf16(w.z);
+      wf[8 * k + 6] = lo_bf16(w.w);
+      wf[8 * k + 7] = hi_bf16(w.w);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.empty(slot));
     ++stage_ctr;
+#pragma unroll 1
+    for (int b = 0; b < B; ++b) {   // uniform: every lane takes part in the shuffle
+      const float4* g = reinterpret_cast<const float4*>(gxs + b * 64 + 32 * hf);
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 v = g[k];
+        a[k & 3] = fmaf(wf[4 * k + 0], v.x, a[k & 3]);
+        a[k & 3] = fmaf(wf[4 * k + 1], v.y, a[k & 3]);
+        a[k & 3] = fmaf(wf[4 * k + 2], v.z, a[k & 3]);
+        a[k & 3] = fmaf(wf[4 * k + 3], v.w, a[k & 3]);
+      }
+      float sum = (a[0] + a[1]) + (a[2] + a[3]);
+      sum += __shfl_xor_sync(FULL, sum, 1);
+      if (valid && (b & 1) == hf) out[(size_t)b * p.E + e0 + el] = sum;
+    }
   }
   return stage_ctr;
 }

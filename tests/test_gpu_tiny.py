@@ -125,6 +125,43 @@ def test_wide_model_batch8_single_activation_buffer():
         rig.close()
 
 
+@pytest.mark.parametrize("n_experts,top_k,lens", [(20, 4, [70, 3]), (192, 8, [40, 130, 65]),
+                                                  (256, 8, [90])])
+def test_router_stage_geometry(n_experts, top_k, lens):
+    """The norm tiles stream their router columns in ring stages of 128
+    expert rows: one partial stage (20 experts), two stages whose second runs
+    past the last expert (192), two full stages (256).  Router logits match
+    the oracle; the selection is the top-k of the kernel's own fp32 logits
+    (value descending, index ascending) and the oracle's wherever its k-th /
+    (k+1)-th gap is clear."""
+    shape = dict(configs.TINY, n_experts=n_experts, top_k=top_k)
+    rig = TinyRig(shape, lens, seed=7)
+    try:
+        got = rig.step()
+        rec = {}
+        ref = rig.oracle_step(record=rec)
+        L, B, E, K = shape["n_layers"], rig.B, n_experts, top_k
+        RL = rig.dec.debug(mk.MK_BUF_RLOGITS).reshape(L, B, E)
+        TK = rig.dec.debug(mk.MK_BUF_TOPK)
+        ids = TK[: L * B * K].reshape(L, B, K)
+        clear = True
+        for l in range(L):
+            for b in range(B):
+                r = rec[(l, b)]
+                assert np.allclose(RL[l, b], r["router_logits"], atol=1e-4, rtol=1e-4), (l, b)
+                own = sorted(range(E), key=lambda e: (-RL[l, b, e], e))[:K]
+                assert list(ids[l, b]) == own, (l, b)
+                if router_gap(r["router_logits"], K) > 1e-3:
+                    assert sorted(ids[l, b].tolist()) == sorted(r["topk_idx"].tolist()), (l, b)
+                else:
+                    clear = False
+        if clear:
+            err, rel = compare_logits(got, ref)
+            assert err <= TIGHT and rel <= REL_L2, (err, rel)
+    finally:
+        rig.close()
+
+
 def test_zipf_routing_batch8():
     lens = [100, 200, 300, 400, 500, 600, 700, 800]
     rig = TinyRig(configs.TINY, lens, seed=5, routing="zipf")

@@ -121,6 +121,11 @@ def test_30b_b1_plan_structure():
     tk = desc[desc[:, D_OP] == OP_TOPK]
     assert np.all(tk[:, D_NWAIT] == 1) and np.all(tk[:, D_W0N] == d // 64)
     rn = desc[desc[:, D_OP] == OP_RN]
+    # a norm tile of a level that feeds a layer streams its router columns:
+    # one ring stage per 128 experts; the final norm streams nothing
+    E = shape["n_experts"]
+    assert np.all(rn[rn[:, D_LAYER] < L][:, D_NSTAGE] == (E + 127) // 128)
+    assert np.all(rn[rn[:, D_LAYER] == L][:, D_NSTAGE] == 0)
     for l in (0, 5):
         ctr = tk[tk[:, D_LAYER] == l][0, D_W0]
         senders = rn[(rn[:, D_LAYER] == l)]
