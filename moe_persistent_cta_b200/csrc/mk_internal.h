@@ -126,8 +126,6 @@ enum Flags : int32_t {
   // Last-arriver work: after its own outputs, the task adds 1 to counter
   // D_X0 (D_X1 arrivals per step); the task that completes the count does the
   // join below and then signals counter D_X2.
-  F_NORM = 32,       // O-proj / down tile: residual add + RMSNorm of its 64 columns
-  F_TOPK = 64,       // router tile: top-k, softmax and expert-slot compaction
   F_COMBINE = 128    // attention chunk: log-sum-exp merge of the (b, g) chunks
 };
 
@@ -237,7 +235,7 @@ struct Shape {
 struct Plan {
   int n_ctas = 0, B = 0, S = 0, max_chunks = 1, n_counters = 0, n_tasks = 0;
   int n_phases = 0;
-  int r_qkv = 16, r_router = 16;
+  int r_qkv = 16;
   int grab = 0;                      // dispenser counter of the fused list
   int grab_phase0 = 0;               // dispenser counters of the phase lists
   int32_t* desc = nullptr;           // [n_tasks][kDescWords], fused priority order

@@ -449,7 +449,6 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   out->n_counters = n_counters;
   out->n_tasks = n_tasks;
   out->r_qkv = r_qkv;
-  out->r_router = r_qkv;
   out->n_phases = n_phases;
   out->grab = grab;
   out->grab_phase0 = grab_phase0;

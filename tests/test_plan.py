@@ -25,7 +25,7 @@ ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 
 D_X0, D_X1, D_X2 = 29, 30, 31
-F_COMBINE = 128
+F_COMBINE = 128   # the only last-arriver flag: the attention merge
 FUSED = F_COMBINE
 
 
