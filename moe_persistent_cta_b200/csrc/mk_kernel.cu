@@ -990,13 +990,41 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
 // over the column chunks that shared a row tile, in chunk order, and writes
 // the operation's outputs.  `rs` is the level's 1/rms per token (A-input
 // operations).
-__device__ __forceinline__ void gemv_epilogue(const Params& p, const int32_t* ent,
+// The launch parameters the epilogue writes through, held in registers for the
+// whole loop (an opaque move keeps the compiler from re-reading them from the
+// constant bank at every use, which after an operation switch can miss).
+template <typename T>
+__device__ __forceinline__ T in_reg(T v) {
+  static_assert(sizeof(T) == 4 || sizeof(T) == 8, "32- or 64-bit value");
+  if constexpr (sizeof(T) == 8) {
+    unsigned long long u = reinterpret_cast<const unsigned long long&>(v), r;
+    asm("mov.b64 %0, %1;" : "=l"(r) : "l"(u));
+    return reinterpret_cast<const T&>(r);
+  } else {
+    unsigned u = reinterpret_cast<const unsigned&>(v), r;
+    asm("mov.b32 %0, %1;" : "=r"(r) : "r"(u));
+    return reinterpret_cast<const T&>(r);
+  }
+}
+struct EpiParams {
+  float *qkv, *logits, *o_part, *expert_a, *moe_part;
+  uint8_t* afrag;
+  int qkvR, V, Hkv, d, S, F, afrag_bytes, k, B, PC;
+  __device__ explicit EpiParams(const Params& p)
+      : qkv(in_reg(p.qkv)), logits(in_reg(p.logits)), o_part(in_reg(p.o_part)),
+        expert_a(in_reg(p.expert_a)), moe_part(in_reg(p.moe_part)), afrag(in_reg(p.afrag)),
+        qkvR(in_reg(p.qkvR)), V(in_reg(p.V)), Hkv(in_reg(p.Hkv)), d(in_reg(p.d)), S(in_reg(p.S)),
+        F(in_reg(p.F)), afrag_bytes(in_reg(p.afrag_bytes)), k(in_reg(p.k)), B(in_reg(p.B)),
+        PC(in_reg(p.part_cols)) {}
+};
+
+__device__ __forceinline__ void gemv_epilogue(const EpiParams& p, const int32_t* ent,
                                               const float* part, const float* rs) {
   const int lane = threadIdx.x & 31;
   const int op = ent[D_OP], layer = ent[D_LAYER];
   const int nm = ent[D_NMAT], R = ent[D_R], row0 = ent[D_ROW0];
   const int MT = R / 16, MTn = nm * MT, kcps = 8 / MTn;
-  const int PC = p.part_cols;
+  const int PC = p.PC;
   const bool expert = (op == OP_GATEUP || op == OP_DOWN);
   const int ncols = expert ? ent[32 + R_NTOK] : p.B;
   const int n_out = R * ncols;
@@ -1881,6 +1909,7 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
   const int PC = p.part_cols;
   const float* part0 = reinterpret_cast<const float*>(sm.epi);
   const float* rstd_ring = part0 + 2 * kConsumerWarps * 16 * PC;
+  const EpiParams ep(p);
   uint32_t ngemv = 0;
   int nloadB = 0;
   for (int i = 0;; ++i) {
@@ -1912,7 +1941,7 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
     if (!warp_wait(p, sm.pfull(pb), (ngemv >> 1) & 1u, 601)) break;
     const int t = ent[32 + R_TASK];
     if (lane == 0) cstamp(p, t, T_K4);
-    gemv_epilogue(p, ent, part0 + pb * kConsumerWarps * 16 * PC,
+    gemv_epilogue(ep, ent, part0 + pb * kConsumerWarps * 16 * PC,
                   rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch);
     __syncwarp();
     if (lane == 0) {
