@@ -389,6 +389,23 @@ __device__ __forceinline__ void prefetch_tmap(const void* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
 
+// A launch parameter moved into a register through an opaque move: a loop
+// that uses it keeps it there instead of re-reading the constant bank at
+// every use (after switching to other code those reads can miss).
+template <typename T>
+__device__ __forceinline__ T in_reg(T v) {
+  static_assert(sizeof(T) == 4 || sizeof(T) == 8, "32- or 64-bit value");
+  if constexpr (sizeof(T) == 8) {
+    unsigned long long u = reinterpret_cast<const unsigned long long&>(v), r;
+    asm("mov.b64 %0, %1;" : "=l"(r) : "l"(u));
+    return reinterpret_cast<const T&>(r);
+  } else {
+    unsigned u = reinterpret_cast<const unsigned&>(v), r;
+    asm("mov.b32 %0, %1;" : "=r"(r) : "r"(u));
+    return reinterpret_cast<const T&>(r);
+  }
+}
+
 __device__ __noinline__ void producer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
@@ -637,6 +654,17 @@ __device__ __noinline__ void producer_loop(const Params& p) {
 // small activation into the next of the two B buffers.
 __device__ __noinline__ void loader_loop(const Params& p) {
   const Smem sm = smem_view(p);
+  // the activation sources and sizes, in registers for the whole loop
+  struct {
+    const uint8_t* actA;
+    const float *qkv, *cs;
+    const uint8_t *ofrag, *afrag;
+    int actA_bytes, actA_stride, actB_bytes, ofrag_bytes, afrag_bytes, S, Hkv, Hq, qkvR, B, hd,
+        G;
+  } const lp = {in_reg(p.actA), in_reg(p.qkv), in_reg(p.cs), in_reg(p.ofrag), in_reg(p.afrag),
+                in_reg(p.actA_bytes), in_reg(p.actA_stride), in_reg(p.actB_bytes),
+                in_reg(p.ofrag_bytes), in_reg(p.afrag_bytes), in_reg(p.S), in_reg(p.Hkv),
+                in_reg(p.Hq), in_reg(p.qkvR), in_reg(p.B), in_reg(p.hd), in_reg(p.G)};
   const int lane = threadIdx.x & 31;
   int curA = -1, nloadA = 0, nloadB = 0;
   const int nA = p.nA;
@@ -645,6 +673,8 @@ __device__ __noinline__ void loader_loop(const Params& p) {
   // for no more arrivals needs no load)
   int seen_ctr = -1;
   uint32_t seen_tgt = 0;
+  const uint32_t* const ctrs = in_reg(p.counters);
+  const uint32_t epoch = in_reg(p.epoch);
   for (int i = 0;; ++i) {
     const int e = i % kFifo;
     if (!warp_wait(p, sm.posted(e), (i / kFifo) & 1, 200)) break;
@@ -663,9 +693,9 @@ __device__ __noinline__ void loader_loop(const Params& p) {
     // lane w polls the task's w-th counter: all counters in one round trip
     if (lane < nwait) {
       const int ctr = ent[D_W0 + 2 * lane];
-      const uint32_t tgt = p.epoch * (uint32_t)ent[D_W0N + 2 * lane];
+      const uint32_t tgt = epoch * (uint32_t)ent[D_W0N + 2 * lane];
       if (ctr != seen_ctr || tgt > seen_tgt) {
-        ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
+        ok = (ld_acquire(ctrs + ctr) >= tgt || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
         seen_ctr = ctr;
         seen_tgt = tgt;
       }
@@ -691,9 +721,9 @@ __device__ __noinline__ void loader_loop(const Params& p) {
       if (lane == 0) {
         fence_proxy_async_global();
         const uint32_t fb = sm.afullA(buf);
-        mbar_expect_tx(fb, (uint32_t)p.actA_bytes);
-        bulk_g2s(saddr(sm.actA + (size_t)buf * p.actA_stride),
-                 p.actA + (size_t)layer * p.actA_bytes, (uint32_t)p.actA_bytes, fb);
+        mbar_expect_tx(fb, (uint32_t)lp.actA_bytes);
+        bulk_g2s(saddr(sm.actA + (size_t)buf * lp.actA_stride),
+                 lp.actA + (size_t)layer * lp.actA_bytes, (uint32_t)lp.actA_bytes, fb);
       }
       __syncwarp();
     }
@@ -704,30 +734,30 @@ __device__ __noinline__ void loader_loop(const Params& p) {
       if (lane == 0) {
         fence_proxy_async_global();
         const uint32_t fb = sm.afullB(buf);
-        const uint32_t dst = saddr(sm.actB + (size_t)buf * p.actB_bytes);
+        const uint32_t dst = saddr(sm.actB + (size_t)buf * lp.actB_bytes);
         const int a = ent[D_A];
         const int bb = ent[D_B];
         if (op == OP_ATTN) {
-          const int b = a, g = bb, G = p.G, hd = p.hd;
-          const float* row = p.qkv + ((size_t)layer * p.B + b) * p.qkvR;
+          const int b = a, g = bb, G = lp.G, hd = lp.hd;
+          const float* row = lp.qkv + ((size_t)layer * lp.B + b) * lp.qkvR;
           const uint32_t qb = (uint32_t)(G * hd * 4), hb = (uint32_t)(hd * 4);
           mbar_expect_tx(fb, qb + 3 * hb);
           bulk_g2s(dst, row + (size_t)g * G * hd, qb, fb);
-          bulk_g2s(dst + qb, row + (size_t)p.Hq * hd + g * hd, hb, fb);
-          bulk_g2s(dst + qb + hb, row + (size_t)(p.Hq + p.Hkv) * hd + g * hd, hb, fb);
-          bulk_g2s(dst + qb + 2 * hb, p.cs + (size_t)b * hd, hb, fb);
+          bulk_g2s(dst + qb, row + (size_t)lp.Hq * hd + g * hd, hb, fb);
+          bulk_g2s(dst + qb + hb, row + (size_t)(lp.Hq + lp.Hkv) * hd + g * hd, hb, fb);
+          bulk_g2s(dst + qb + 2 * hb, lp.cs + (size_t)b * hd, hb, fb);
         } else if (op == OP_OPROJ) {
           const int g = bb;
-          mbar_expect_tx(fb, (uint32_t)p.ofrag_bytes);
-          bulk_g2s(dst, p.ofrag + ((size_t)layer * p.Hkv + g) * p.ofrag_bytes,
-                   (uint32_t)p.ofrag_bytes, fb);
+          mbar_expect_tx(fb, (uint32_t)lp.ofrag_bytes);
+          bulk_g2s(dst, lp.ofrag + ((size_t)layer * lp.Hkv + g) * lp.ofrag_bytes,
+                   (uint32_t)lp.ofrag_bytes, fb);
         } else if (ent[32 + R_EXPERT] < 0) {   // OP_DOWN of an empty slot: nothing to copy
           mbar_arrive(fb);
         } else {  // OP_DOWN
           const int j = a;
-          mbar_expect_tx(fb, (uint32_t)p.afrag_bytes);
-          bulk_g2s(dst, p.afrag + ((size_t)layer * p.S + j) * p.afrag_bytes,
-                   (uint32_t)p.afrag_bytes, fb);
+          mbar_expect_tx(fb, (uint32_t)lp.afrag_bytes);
+          bulk_g2s(dst, lp.afrag + ((size_t)layer * lp.S + j) * lp.afrag_bytes,
+                   (uint32_t)lp.afrag_bytes, fb);
         }
       }
       __syncwarp();
@@ -749,6 +779,7 @@ __device__ __noinline__ void loader_loop(const Params& p) {
 __device__ __noinline__ void signal_loop(const Params& p) {
   const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
+  uint32_t* const ctrs = in_reg(p.counters);
   for (int i = 0;; ++i) {
     const int e = i % kFifo;
     if (!warp_wait(p, sm.done(e), (i / kFifo) & 1, 300)) break;
@@ -756,7 +787,7 @@ __device__ __noinline__ void signal_loop(const Params& p) {
     if (ent[D_OP] == OP_NONE) break;
     if (lane == 0) {
       const int nsig = ent[D_NSIG];
-      for (int s = 0; s < nsig; ++s) red_release_add(p.counters + ent[D_S0 + s], 1u);
+      for (int s = 0; s < nsig; ++s) red_release_add(ctrs + ent[D_S0 + s], 1u);
       mbar_arrive(sm.fempty(e));
     }
     __syncwarp();
@@ -991,21 +1022,7 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
 // the operation's outputs.  `rs` is the level's 1/rms per token (A-input
 // operations).
 // The launch parameters the epilogue writes through, held in registers for the
-// whole loop (an opaque move keeps the compiler from re-reading them from the
-// constant bank at every use, which after an operation switch can miss).
-template <typename T>
-__device__ __forceinline__ T in_reg(T v) {
-  static_assert(sizeof(T) == 4 || sizeof(T) == 8, "32- or 64-bit value");
-  if constexpr (sizeof(T) == 8) {
-    unsigned long long u = reinterpret_cast<const unsigned long long&>(v), r;
-    asm("mov.b64 %0, %1;" : "=l"(r) : "l"(u));
-    return reinterpret_cast<const T&>(r);
-  } else {
-    unsigned u = reinterpret_cast<const unsigned&>(v), r;
-    asm("mov.b32 %0, %1;" : "=r"(r) : "r"(u));
-    return reinterpret_cast<const T&>(r);
-  }
-}
+// whole loop (see in_reg).
 struct EpiParams {
   float *qkv, *logits, *o_part, *expert_a, *moe_part;
   uint8_t* afrag;
