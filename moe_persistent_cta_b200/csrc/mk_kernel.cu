@@ -408,19 +408,34 @@ __device__ __forceinline__ T in_reg(T v) {
 
 __device__ __noinline__ void producer_loop(const Params& p) {
   const Smem sm = smem_view(p);
+  // the values the dispense/resolve/issue path reads, in registers for the
+  // whole loop
+  struct {
+    uint32_t* counters;
+    const int32_t *desc, *route, *seq_lens, *page_table;
+    const uint8_t* tmaps;
+    uint32_t epoch;
+    int grab, n_tasks, n_ctas, route_words, B, k, S, E, F, d, max_pages, n_pages, Hkv, hd;
+  } const pp = {in_reg(p.counters), in_reg(p.desc), in_reg(p.route), in_reg(p.seq_lens),
+                in_reg(p.page_table), in_reg(static_cast<const uint8_t*>(p.tmaps)),
+                in_reg(p.epoch), in_reg(p.grab), in_reg(p.n_tasks), in_reg(p.n_ctas),
+                in_reg(p.route_words), in_reg(p.B), in_reg(p.k), in_reg(p.S), in_reg(p.E),
+                in_reg(p.F), in_reg(p.d), in_reg(p.max_pages), in_reg(p.n_pages), in_reg(p.Hkv),
+                in_reg(p.hd)};
+  auto tmap_at = [&](int idx) { return static_cast<const void*>(pp.tmaps + (size_t)idx * 128); };
   const int lane = threadIdx.x & 31;
   const int NS = sm.NS;
   uint32_t slot = 0, phase = 0;   // ring position of the next stage
-  const uint32_t base = (p.epoch - 1u) * (uint32_t)(p.n_tasks + p.n_ctas);
+  const uint32_t base = (pp.epoch - 1u) * (uint32_t)(pp.n_tasks + pp.n_ctas);
   const uint64_t pol = l2_evict_first();
-  auto valid = [&](int t) { return t >= 0 && t < p.n_tasks; };
+  auto valid = [&](int t) { return t >= 0 && t < pp.n_tasks; };
   int t_next = 0;
   int32_t dw_next = 0;
   auto take = [&]() {   // next task index and its descriptor (word `lane`)
     uint32_t raw = 0;
-    if (lane == 0) raw = atomicAdd(p.counters + p.grab, 1u);
+    if (lane == 0) raw = atomicAdd(pp.counters + pp.grab, 1u);
     t_next = __shfl_sync(FULL, (int)(raw - base), 0);
-    dw_next = valid(t_next) ? __ldg(p.desc + (size_t)t_next * kDescWords + lane) : 0;
+    dw_next = valid(t_next) ? __ldg(pp.desc + (size_t)t_next * kDescWords + lane) : 0;
   };
   int pw_done_ctr = -1;          // producer wait already seen satisfied (this step)
   uint32_t pw_done_tgt = 0;
@@ -448,8 +463,8 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
     const int map0 = __shfl_sync(FULL, dw, D_MAP0), map1 = __shfl_sync(FULL, dw, D_MAP1);
     if (lane == 0 && (nstage > 0 || op == OP_ATTN)) {
-      prefetch_tmap(tmap(p, map0));
-      if (op == OP_GATEUP || op == OP_ATTN) prefetch_tmap(tmap(p, map1));
+      prefetch_tmap(tmap_at(map0));
+      if (op == OP_GATEUP || op == OP_ATTN) prefetch_tmap(tmap_at(map1));
     }
     int32_t rw = 0;  // resolved word `lane`
     uint32_t pwait = 0;
@@ -457,10 +472,10 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     bool fail = false;
     if (op == OP_GATEUP || op == OP_DOWN) {
       const int ctr = __shfl_sync(FULL, dw, D_PW);
-      const uint32_t tgt = p.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
+      const uint32_t tgt = pp.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
       if (ctr != pw_done_ctr || tgt > pw_done_tgt) {
         int ok = 1;
-        if (lane == 0) ok = wait_counter(p, ctr, tgt, t, op) ? 1 : 0;
+        if (lane == 0) ok = (ld_acquire(pp.counters + ctr) >= tgt || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
         ok = __shfl_sync(FULL, ok, 0);
         if (!ok) break;
         pw_done_ctr = ctr;
@@ -470,8 +485,8 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       // expert, R_NTOK the token count, R_TOK/R_RANK/R_W + n token n's id,
       // rank and weight (words past the count are read and then dropped)
       const int j = __shfl_sync(FULL, dw, D_A);
-      const int32_t* rt = p.route + (size_t)layer * p.route_words;
-      const int B = p.B, K = p.k, S = p.S;
+      const int32_t* rt = pp.route + (size_t)layer * pp.route_words;
+      const int B = pp.B, K = pp.k, S = pp.S;
       int idx = -1;
       if (lane == R_EXPERT) idx = route_slot_expert(B, K) + j;
       else if (lane == R_NTOK) idx = route_slot_ntok(B, K, S) + j;
@@ -482,7 +497,7 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       const int32_t v = idx >= 0 ? __ldcg(rt + idx) : 0;
       expert = __shfl_sync(FULL, v, R_EXPERT);
       ntok = __shfl_sync(FULL, v, R_NTOK);
-      if (expert >= p.E || ntok < 0 || ntok > B) {
+      if (expert >= pp.E || ntok < 0 || ntok > B) {
         if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, expert, ntok, 1);
         set_abort();
         break;
@@ -498,21 +513,21 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       const int c = __shfl_sync(FULL, dw, D_C);
       const int nc = __shfl_sync(FULL, dw, D_D);
       const int ppc = __shfl_sync(FULL, dw, D_PPC);
-      seqlen = __ldg(p.seq_lens + b);
+      seqlen = __ldg(pp.seq_lens + b);
       const int pages_now = (seqlen + kPage - 1) / kPage;
       p0 = c * ppc;
       int np = min(ppc, pages_now - p0);
       if (np < 0) np = 0;
       const bool last = (c == nc - 1);
-      if (seqlen < 0 || (last && p0 + ppc < pages_now) || (seqlen / kPage) >= p.max_pages) {
+      if (seqlen < 0 || (last && p0 + ppc < pages_now) || (seqlen / kPage) >= pp.max_pages) {
         if (lane == 0) raise_error(p, MK_ERR_STATE, t, op, -1, seqlen, pages_now, b);
         set_abort();
         fail = true;
       }
       if (!fail && last) {
-        phys_new = __ldg(p.page_table + (size_t)b * p.max_pages + seqlen / kPage);
-        if (phys_new < 0 || phys_new >= p.n_pages) {
-          if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, phys_new, p.n_pages, 2);
+        phys_new = __ldg(pp.page_table + (size_t)b * pp.max_pages + seqlen / kPage);
+        if (phys_new < 0 || phys_new >= pp.n_pages) {
+          if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, phys_new, pp.n_pages, 2);
           set_abort();
           fail = true;
         }
@@ -541,17 +556,17 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     if (op == OP_ATTN) {
       const int b = __shfl_sync(FULL, dw, D_A);
       const int g = __shfl_sync(FULL, dw, D_B);
-      const void* mk_ = tmap(p, map0);
-      const void* mv_ = tmap(p, map1);
+      const void* mk_ = tmap_at(map0);
+      const void* mv_ = tmap_at(map1);
       const int np = ntok;
       int pg = -1;
-      const int* pt = p.page_table + (size_t)b * p.max_pages;
+      const int* pt = pp.page_table + (size_t)b * pp.max_pages;
       for (int s = 0; s < nstage; ++s) {
         const int pi = s >> 1;
         if ((pi & 31) == 0 && (s & 1) == 0) {
           int idx = p0 + pi + lane;
           pg = (pi + lane < np) ? __ldg(pt + idx) : 0;
-          int bad = (pi + lane < np) && (pg < 0 || pg >= p.n_pages);
+          int bad = (pi + lane < np) && (pg < 0 || pg >= pp.n_pages);
           if (__any_sync(FULL, bad)) {
             if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, 0, 0, 3);
             set_abort();
@@ -565,11 +580,11 @@ __device__ __noinline__ void producer_loop(const Params& p) {
           break;
         }
         if (lane == 0) {
-          const uint32_t bytes = (uint32_t)p.hd * kPage * 2;
+          const uint32_t bytes = (uint32_t)pp.hd * kPage * 2;
           const uint32_t fb = sm.full(slot);
           mbar_expect_tx(fb, bytes);
           const uint32_t dst = saddr(sm.ring + (size_t)slot * kStageBytes);
-          const int y = (phys * p.Hkv + g) * kPage;
+          const int y = (phys * pp.Hkv + g) * kPage;
           const void* m = (s & 1) ? mv_ : mk_;
           tma_3d(dst, m, 0, y, 0, fb, pol);   // [hd/64 chunks][64 tokens][128 B]
         }
@@ -581,8 +596,8 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       // the tile's router weights: rows [128 s, 128 s + 128) of its 64-column
       // chunk; rows past E land as zeros
       const int r = __shfl_sync(FULL, dw, D_A);
-      const void* m0 = tmap(p, map0);
-      const uint32_t box_bytes = (uint32_t)min(p.E, kRouterRowsPerStage) * 128u;
+      const void* m0 = tmap_at(map0);
+      const uint32_t box_bytes = (uint32_t)min(pp.E, kRouterRowsPerStage) * 128u;
       for (int s = 0; s < nstage; ++s) {
         if (!warp_wait(p, sm.empty(slot), phase ^ 1, 103)) {
           fail = true;
@@ -604,10 +619,10 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       const int MT = R / 16, kcps = 8 / (nm * MT);
       const int k0 = __shfl_sync(FULL, dw, D_K0);
       int row0 = __shfl_sync(FULL, dw, D_ROW0);
-      if (op == OP_GATEUP) row0 += expert * p.F;
-      if (op == OP_DOWN) row0 += expert * p.d;
-      const void* m0 = tmap(p, map0);
-      const void* m1 = nm > 1 ? tmap(p, map1) : m0;
+      if (op == OP_GATEUP) row0 += expert * pp.F;
+      if (op == OP_DOWN) row0 += expert * pp.d;
+      const void* m0 = tmap_at(map0);
+      const void* m1 = nm > 1 ? tmap_at(map1) : m0;
       for (int s = 0; s < nstage; ++s) {
         const uint64_t w0 = clock64();
         if (!warp_wait(p, sm.empty(slot), phase ^ 1, 102)) {
