@@ -35,10 +35,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "b7cd4d6dd7d6b75eddae2cae091e28b17715e7e146b48e34986be55e3bb3258b",
+    "kernel_sha256": "e57f8b901c55b30d73ad9714fd0faeb0cad450a25d95e8974e09c0badd907821",
     "workload": "moe30b_b1",
-    "fixed_bytes": 622.71e6,
-    "per_layer_bytes": 114.37e6,
+    "fixed_bytes": 623.44e6,
+    "per_layer_bytes": 114.15e6,
 }
 
 
