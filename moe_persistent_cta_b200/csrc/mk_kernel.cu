@@ -2054,17 +2054,25 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
 namespace {
 // the kernel instantiation for a batch size and head dimension, and the
 // dynamic shared memory it was last configured for
+// (the attribute is per device: the cache holds one entry per device ordinal)
+constexpr int kMaxDevices = 64;
 struct KernelSlot {
   const void* fn;
-  int configured_bytes;
+  int configured_bytes[kMaxDevices];   // 0: not configured on that device yet
 };
 KernelSlot g_kernels[3][2] = {
-    {{reinterpret_cast<const void*>(mk_interp<1, 64>), -1},
-     {reinterpret_cast<const void*>(mk_interp<1, 128>), -1}},
-    {{reinterpret_cast<const void*>(mk_interp<2, 64>), -1},
-     {reinterpret_cast<const void*>(mk_interp<2, 128>), -1}},
-    {{reinterpret_cast<const void*>(mk_interp<3, 64>), -1},
-     {reinterpret_cast<const void*>(mk_interp<3, 128>), -1}}};
+    {{reinterpret_cast<const void*>(mk_interp<1, 64>), {}},
+     {reinterpret_cast<const void*>(mk_interp<1, 128>), {}}},
+    {{reinterpret_cast<const void*>(mk_interp<2, 64>), {}},
+     {reinterpret_cast<const void*>(mk_interp<2, 128>), {}}},
+    {{reinterpret_cast<const void*>(mk_interp<3, 64>), {}},
+     {reinterpret_cast<const void*>(mk_interp<3, 128>), {}}}};
+// the cache entry of the current device, or null past kMaxDevices
+int* configured_entry(KernelSlot& k) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return &k.configured_bytes[dev];
+}
 KernelSlot& kernel_for(int B, int hd) {
   return g_kernels[B <= 1 ? 0 : (B == 2 ? 1 : 2)][hd == 128 ? 1 : 0];
 }
@@ -2072,11 +2080,12 @@ KernelSlot& kernel_for(int B, int hd) {
 
 cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream) {
   KernelSlot& k = kernel_for(p.B, p.hd);
-  if (k.configured_bytes != p.smem_bytes) {
+  int* conf = configured_entry(k);
+  if (!conf || *conf != p.smem_bytes) {
     cudaError_t e =
         cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
-    k.configured_bytes = p.smem_bytes;
+    if (conf) *conf = p.smem_bytes;
   }
   void* args[] = {const_cast<Params*>(&p)};
   return cudaLaunchCooperativeKernel(k.fn, dim3(grid), dim3(kThreads), args, (size_t)p.smem_bytes,
@@ -2092,7 +2101,7 @@ cudaError_t max_coresident(int smem_bytes, int* blocks_per_sm) {
       cudaError_t e =
           cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
       if (e != cudaSuccess) return e;
-      k.configured_bytes = smem_bytes;
+      if (int* conf = configured_entry(k)) *conf = smem_bytes;
       int n = 0;
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k.fn, kThreads, (size_t)smem_bytes);
       if (e != cudaSuccess) return e;
