@@ -126,6 +126,10 @@ def test_30b_b1_plan_structure():
     E = shape["n_experts"]
     assert np.all(rn[rn[:, D_LAYER] < L][:, D_NSTAGE] == (E + 127) // 128)
     assert np.all(rn[rn[:, D_LAYER] == L][:, D_NSTAGE] == 0)
+    # ... through its own layer's router tensor map (8 maps per layer, router third)
+    D_MAP0 = 23
+    lv = rn[rn[:, D_LAYER] < L]
+    assert np.all(lv[:, D_MAP0] == lv[:, D_LAYER] * 8 + 2)
     for l in (0, 5):
         ctr = tk[tk[:, D_LAYER] == l][0, D_W0]
         senders = rn[(rn[:, D_LAYER] == l)]
