@@ -24,14 +24,20 @@ D_OP, D_LAYER, D_A, D_B = 0, 1, 2, 3
 
 
 def _times(stamps: np.ndarray) -> np.ndarray:
-    """uint32 ns stamps -> float64 us relative to the earliest stamp."""
+    """uint32 ns stamps -> float64 us relative to the earliest stamp.
+
+    The stamps are the low 32 bits of a nanosecond timer, which wraps every
+    ~4.3 s; a step is far shorter, so stamps that span more than half the
+    range straddle one wrap, and the small (post-wrap) values are lifted by
+    2^32 before the earliest stamp is taken."""
     st = stamps[:, :T_CTA].astype(np.int64)
-    valid = st[st != 0]
-    base = int(valid.min()) if valid.size else 0
-    out = st - base
-    out[out < 0] += 1 << 32           # one wrap of the 32-bit counter
-    out = out.astype(np.float64) / 1e3
-    out[st == 0] = np.nan
+    present = st != 0
+    v = st.copy()
+    if present.any() and st[present].max() - st[present].min() > (1 << 31):
+        v[present & (st < (1 << 31))] += 1 << 32
+    base = int(v[present].min()) if present.any() else 0
+    out = (v - base).astype(np.float64) / 1e3
+    out[~present] = np.nan
     return out
 
 
