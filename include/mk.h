@@ -167,15 +167,16 @@ mk_status mk_decode_step_unfused(mk_ctx* ctx, const int32_t* tokens,
  *
  * The step's scratch (counters, routing words, activations, attention and
  * expert partials) lives in one file-scope device array of
- * MK_STATIC_SCRATCH_MAX_BYTES (32 MiB) instead of the context's buffers;
- * the array is reserved on every device that loads the library until the
- * process exits.  The call itself allocates nothing.  The context (from
+ * MK_STATIC_SCRATCH_MAX_BYTES (32 MiB) instead of the context's buffers.
+ * mk_create looks up the array's device address (cudaGetSymbolAddress, with
+ * the device current), which loads the array on that device if it is not
+ * loaded yet; it then stays reserved there until the process exits.  This
+ * call itself loads nothing and allocates nothing.  The context (from
  * mk_create and mk_build_schedule, which do allocate) supplies the schedule,
  * tensor maps and status word; arguments and device inputs are those of
  * mk_decode_step.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - Returns MK_ERR_CUDA, before any launch, if mk_create could not resolve
+ *    the array on this device (for example when no room was left for it).
  *  - Every call, from every context, shares the one array and leaves its
  *    contents in place; each call clears the counters and routing words on
  *    `stream` before the launch.  Calls that overlap on the GPU (other
@@ -190,7 +191,8 @@ mk_status mk_decode_step_static(mk_ctx* ctx, const int32_t* tokens, const int32_
                                 const int32_t* page_table, const int32_t* seq_lens,
                                 float* logits, void* stream);
 
-/* Synchronize the context's last stream and read the device status word.
+/* Synchronize the stream of the context's last step (the whole device when no
+ * step has been launched yet) and read the device status word.
  * device_status (may be NULL) receives MK_OK or the latched device error;
  * detail (may be NULL) receives int32[8]: {code, cta, task, opcode, counter,
  * observed, target, aux}.  Returns MK_OK if the device status is clean, else

@@ -18,6 +18,7 @@
 namespace mk {
 cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream);
 cudaError_t max_coresident(int smem_bytes, int* blocks_per_sm);
+mk_status static_scratch_setup(int device);
 }  // namespace mk
 
 using mk::Params;
@@ -33,6 +34,7 @@ struct DevBuf {
 struct mk_ctx {
   int device = 0;
   int n_sms = 0;
+  int clock_khz = 0;   // peak SM clock: converts wait deadlines to clock64 cycles
   mk_config cfg{};
   Shape shape{};
   int r_qkv = 16, r_ff = 16;
@@ -65,6 +67,7 @@ struct mk_ctx {
   uint32_t epoch = 0;
   unsigned long long timeout_ns = 2000ull * 1000ull * 1000ull;
   cudaStream_t last_stream = nullptr;
+  bool launched = false;   // a step was launched on last_stream
   Params base{};
 };
 
@@ -137,6 +140,12 @@ mk_status encode_3d(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows,
 
 
 int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// A wait limit in ns as SM clock cycles at the device's peak clock: at any
+// lower clock the same cycle count takes longer, so the limit only grows.
+unsigned long long deadline_cycles(const mk_ctx* c, unsigned long long ns) {
+  return ns * (unsigned long long)c->clock_khz / 1000000ull;
+}
 
 }  // namespace
 
@@ -218,6 +227,9 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
   };
   if (cudaDeviceGetAttribute(&c->n_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
     return fail(MK_ERR_CUDA);
+  if (cudaDeviceGetAttribute(&c->clock_khz, cudaDevAttrClockRate, device) != cudaSuccess ||
+      c->clock_khz <= 0)
+    c->clock_khz = 2000000;   // not reported: assume 2 GHz
 
   // tensor maps
   const int nmaps = L * mk::kMapsPerLayer + 1;
@@ -271,8 +283,8 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
     vp[l] = t->v_pool[l];
   }
   auto upload_ptrs = [&](void*** dst, std::vector<void*>& src) -> mk_status {
-    MK_CUDA(cudaMalloc(reinterpret_cast<void**>(dst), sizeof(void*) * L));
-    MK_CUDA(cudaMemcpy(*dst, src.data(), sizeof(void*) * L, cudaMemcpyHostToDevice));
+    MK_CUDA(cudaMalloc(reinterpret_cast<void**>(dst), sizeof(void*) * src.size()));
+    MK_CUDA(cudaMemcpy(*dst, src.data(), sizeof(void*) * src.size(), cudaMemcpyHostToDevice));
     return MK_OK;
   };
   {
@@ -293,6 +305,10 @@ mk_status mk_create(const mk_config* cfg, const mk_tensors* t, int device, mk_ct
     return fail(MK_ERR_CUDA);
   if (cudaMalloc(&c->d_status, sizeof(int32_t) * 16) != cudaSuccess) return fail(MK_ERR_OOM);
   if (cudaMemset(c->d_status, 0, sizeof(int32_t) * 16) != cudaSuccess) return fail(MK_ERR_CUDA);
+  // The fixed scratch array of mk_decode_step_static is resolved (and so
+  // loaded) here, not on that call's first use.  If it cannot be, the context
+  // still serves every other entry point; mk_decode_step_static then fails.
+  (void)mk::static_scratch_setup(device);
   const char* env = std::getenv("MK_TIMEOUT_MS");
   if (env) {
     long ms = std::atol(env);
@@ -471,9 +487,7 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   p.logits = logits;
-  // deadlines count SM cycles: 2 per ns bounds the wall time from below at
-  // any clock up to 2 GHz (a slower clock only lengthens the deadline)
-  p.timeout_cycles = c->timeout_ns * 2ull;
+  p.timeout_cycles = deadline_cycles(c, c->timeout_ns);
   p.epoch = c->epoch + 1;
   cudaError_t e = cudaSuccess;
   p.n_ctas = c->plan.n_ctas;
@@ -511,6 +525,7 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
   if (e != cudaSuccess) return from_cuda(e);
   c->epoch += 1;
   c->last_stream = st;
+  c->launched = true;
   return MK_OK;
 }
 
@@ -529,7 +544,10 @@ mk_status mk_decode_step_unfused(mk_ctx* c, const int32_t* tokens, const int32_t
 mk_status mk_check(mk_ctx* c, int32_t* device_status, int32_t* detail) {
   if (!c) return MK_ERR_INVALID;
   MK_CUDA(cudaSetDevice(c->device));
-  MK_CUDA(cudaDeviceSynchronize());
+  if (c->launched)
+    MK_CUDA(cudaStreamSynchronize(c->last_stream));
+  else
+    MK_CUDA(cudaDeviceSynchronize());
   int32_t st[16];
   MK_CUDA(cudaMemcpy(st, c->d_status, sizeof(st), cudaMemcpyDeviceToHost));
   if (device_status) *device_status = st[mk::ST_CODE];
@@ -690,12 +708,14 @@ mk_status launch_step_in(mk_ctx* c, const int32_t* tokens, const int32_t* positi
   carve_scratch(c->base, c->plan.n_counters, static_cast<uint8_t*>(scratch), &p);
   const size_t zero_bytes = reinterpret_cast<uint8_t*>(p.x) - static_cast<uint8_t*>(scratch);
   MK_CUDA(cudaMemsetAsync(scratch, 0, zero_bytes, st));   // counters + routing words
+  c->last_stream = st;
+  c->launched = true;
   p.tokens = tokens;
   p.positions = positions;
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   p.logits = logits;
-  p.timeout_cycles = c->timeout_ns * 2ull;
+  p.timeout_cycles = deadline_cycles(c, c->timeout_ns);
   p.epoch = 1;
   p.trace = nullptr;
   p.n_ctas = c->plan.n_ctas;
@@ -745,7 +765,7 @@ mk_status mk_selftest_timeout(mk_ctx* c, int32_t timeout_ms, int32_t* device_sta
   p.n_ctas = c->plan.n_ctas;
   p.epoch = 1;
   p.trace = nullptr;
-  p.timeout_cycles = (unsigned long long)timeout_ms * 2000000ull;
+  p.timeout_cycles = deadline_cycles(c, (unsigned long long)timeout_ms * 1000000ull);
   // step inputs are never read (the task does not run); any device address
   int32_t* d0 = static_cast<int32_t*>(c->selftest.ptr);
   p.tokens = d0;

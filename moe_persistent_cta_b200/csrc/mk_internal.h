@@ -81,7 +81,7 @@ enum Op : int32_t {
   OP_RN = 1,        // fused residual add + RMSNorm statistics for one 64-row tile
   OP_QKV = 2,       // QKV projection tile (RoPE/append happen in OP_ATTN)
   OP_ROUTER = 3,    // (unused: the norm tiles produce the router logits)
-  OP_TOPK = 4,      // top-k + softmax + expert-slot compaction
+  OP_TOPK = 4,      // (unused: the last-arriving norm tile of a level runs the top-k)
   OP_ATTN = 5,      // paged GQA decode attention over one KV chunk (+RoPE, append)
   OP_COMBINE = 6,   // (unused: the last-arriving attention chunk of (b, g) merges)
   OP_OPROJ = 7,     // O-proj tile, split-K by KV group
@@ -126,7 +126,9 @@ enum Flags : int32_t {
   // Last-arriver work: after its own outputs, the task adds 1 to counter
   // D_X0 (D_X1 arrivals per step); the task that completes the count does the
   // join below and then signals counter D_X2.
-  F_COMBINE = 128    // attention chunk: log-sum-exp merge of the (b, g) chunks
+  F_COMBINE = 128,   // attention chunk: log-sum-exp merge of the (b, g) chunks
+  F_TOPK = 256       // norm tile: router logits, top-k, softmax and slot compaction
+                     // of the layer the level feeds
 };
 
 // ------------------------------------------------- resolved entry words ---
@@ -206,6 +208,15 @@ struct Params {
   int part_cols;     // token columns per partial row: B for B <= 2, else 8
   int smem_bytes;
 };
+
+// Counters and their targets (epoch x arrivals per step) are uint32 and wrap
+// around; they are compared by signed difference, which stays right across
+// the wrap as long as a counter never lags its target by 2^31 or more (a step
+// adds at most a few thousand arrivals to any counter).
+// reached(v, t): counter value v has reached target t.
+MK_HD inline bool reached(uint32_t v, uint32_t t) { return (int32_t)(v - t) >= 0; }
+// later(t1, t0): target t1 asks for more arrivals than target t0.
+MK_HD inline bool later(uint32_t t1, uint32_t t0) { return (int32_t)(t1 - t0) > 0; }
 
 // status word layout
 enum StatusField : int {

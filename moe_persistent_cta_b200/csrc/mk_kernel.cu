@@ -24,9 +24,10 @@
 //                      fp32 activations as the 8-column B operand split into
 //                      three bf16 terms, so the product keeps ~24 bits),
 //                      attention with an online softmax, and the epilogues.
-// Every wait is bounded by a globaltimer deadline; on expiry the CTA latches an
-// error in the status word, raises the abort flag and unwinds, waiting for its
-// own copies in flight before it exits.
+// Every wait is bounded by a deadline counted in SM clock cycles (clock64; the
+// host converts the millisecond limit at the device's peak SM clock); on expiry
+// the CTA latches an error in the status word, raises the abort flag and
+// unwinds, waiting for its own copies in flight before it exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -303,7 +304,7 @@ __device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_
   const uint64_t t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     v = ld_acquire(c);
-    if (v >= target) return true;
+    if (reached(v, target)) return true;
     if ((it & 7u) == 0) {
       if (aborted()) return false;
       if (*(volatile int*)(p.status + ST_ABORT)) {
@@ -321,7 +322,7 @@ __device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_
 
 __device__ __forceinline__ bool wait_counter(const Params& p, int ctr, uint32_t target, int task,
                                              int op) {
-  if (ld_acquire(p.counters + ctr) >= target) return true;
+  if (reached(ld_acquire(p.counters + ctr), target)) return true;
   return wait_counter_slow(p, ctr, target, task, op);
 }
 
@@ -473,9 +474,10 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     if (op == OP_GATEUP || op == OP_DOWN) {
       const int ctr = __shfl_sync(FULL, dw, D_PW);
       const uint32_t tgt = pp.epoch * (uint32_t)__shfl_sync(FULL, dw, D_PWN);
-      if (ctr != pw_done_ctr || tgt > pw_done_tgt) {
+      if (ctr != pw_done_ctr || later(tgt, pw_done_tgt)) {
         int ok = 1;
-        if (lane == 0) ok = (ld_acquire(pp.counters + ctr) >= tgt || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
+        if (lane == 0)
+          ok = (reached(ld_acquire(pp.counters + ctr), tgt) || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
         ok = __shfl_sync(FULL, ok, 0);
         if (!ok) break;
         pw_done_ctr = ctr;
@@ -709,8 +711,8 @@ __device__ __noinline__ void loader_loop(const Params& p) {
     if (lane < nwait) {
       const int ctr = ent[D_W0 + 2 * lane];
       const uint32_t tgt = epoch * (uint32_t)ent[D_W0N + 2 * lane];
-      if (ctr != seen_ctr || tgt > seen_tgt) {
-        ok = (ld_acquire(ctrs + ctr) >= tgt || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
+      if (ctr != seen_ctr || later(tgt, seen_tgt)) {
+        ok = (reached(ld_acquire(ctrs + ctr), tgt) || wait_counter_slow(p, ctr, tgt, t, op)) ? 1 : 0;
         seen_ctr = ctr;
         seen_tgt = tgt;
       }
@@ -1544,6 +1546,7 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
     }
   }
   cbar();
+  if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K2);   // residual rows summed
   float* rows = reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes);
   float* gxs = stage;   // [B][64] gamma x of the tile (the staging area is free)
 #pragma unroll 1
@@ -1565,6 +1568,7 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
   if (l == 0 && r == 0) rope_table(p, ent[32 + R_TASK]);
   if (nst == 0) return stage_ctr;
   cbar();
+  if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K3);   // outputs written
   float* out = p.rpart + ((size_t)l * p.NR + r) * B * p.E;
   // thread pair per expert row: half hf takes columns 32 hf .. 32 hf + 31
   // (four 16-byte units, four independent FMA chains); the pair adds its two
@@ -1613,6 +1617,7 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
       if (valid && (b & 1) == hf) out[(size_t)b * p.E + e0 + el] = sum;
     }
   }
+  if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K4);   // router shares written
   return stage_ctr;
 }
 
@@ -1621,10 +1626,9 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
 // logits[b][e] = (1/rms_b) * sum_r rpart[l][r][b][e] + bias[e], the shares
 // summed in ascending r: thread group g of nG sums r = g, g + nG, ... of one
 // float4 column, and the groups' sums are added in g order.
-__device__ __noinline__ void topk_task(const Params& p, const int32_t* ent) {
+__device__ __noinline__ void topk_task(const Params& p, int l) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
-  const int l = ent[D_LAYER];
   const int B = p.B, E = p.E, K = p.k, S = p.S, NR = p.NR;
   int32_t* rt = p.route + (size_t)l * p.route_words;
   int* sel = reinterpret_cast<int*>(sm.scratch);               // [B][8]
@@ -1898,9 +1902,28 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
     switch (op) {
       case OP_RN:
         stage_ctr = rn_task(p, ent, stage_ctr);
-        break;
-      case OP_TOPK:
-        topk_task(p, ent);
+        if (ent[D_FLAGS] & F_TOPK) {
+          // The tile is complete: its own signal goes out now (the FIFO entry
+          // is released, so its words are copied first).  The tile whose
+          // arrival completes the level has acquired every tile's router
+          // shares and sum-of-squares partials and runs the layer's top-k.
+          const int lyr = layer, x0 = ent[D_X0], x1 = ent[D_X1], x2 = ent[D_X2];
+          cbar();
+          int last = 0;
+          if (ct == 0) {
+            stamp(p, t, T_C_END);
+            cstamp(p, t, T_K5);
+            mbar_arrive(sm.done(e));
+            const uint32_t old = atom_add_acq_rel(p.counters + x0, 1u);
+            last = old + 1u == p.epoch * (uint32_t)x1;
+          }
+          if (cbar_or(last)) {
+            topk_task(p, lyr);
+            cbar();
+            if (ct == 0) red_release_add(p.counters + x2, 1u);
+          }
+          continue;
+        }
         break;
       default:  // OP_ATTN
         stage_ctr = attn_task<HD>(p, ent, actB, stage_ctr);

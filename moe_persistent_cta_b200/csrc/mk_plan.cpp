@@ -18,10 +18,10 @@
 // "Three sources of speedup", item 2).
 //
 // Priority order inside a layer: the norm tiles (which also produce the
-// router logits, share by share); QKV and top-k; attention chunks (their
-// cached K/V stream before the new query exists); expert gate/up (the MoE
-// branch is the longer one); then the attention tail and the expert down
-// projections.
+// router logits, share by share, and the last of which runs the top-k); QKV;
+// attention chunks (their cached K/V stream before the new query exists);
+// expert gate/up (the MoE branch is the longer one); then the attention tail
+// and the expert down projections.
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
@@ -140,11 +140,12 @@ struct Task {
 
 struct Layout {
   int L, B, S, Hkv, NR;
-  int norm0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
+  int norm0, narr0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
   void build(int L_, int B_, int S_, int Hkv_, int NR_) {
     L = L_; B = B_; S = S_; Hkv = Hkv_; NR = NR_;
     int c = 0;
     norm0 = c; c += L + 1;
+    narr0 = c; c += L;
     qkv0 = c; c += L * Hkv;
     rtr0 = c; c += L;
     attp0 = c; c += L * B * Hkv;
@@ -155,6 +156,7 @@ struct Layout {
     total = c;
   }
   int norm(int l) const { return norm0 + l; }
+  int narr(int l) const { return narr0 + l; }
   int qkv(int l, int g) const { return qkv0 + l * Hkv + g; }
   int rtr(int l) const { return rtr0 + l; }
   int attp(int l, int b, int g) const { return attp0 + (l * B + b) * Hkv + g; }
@@ -253,7 +255,9 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   // residual add + RMSNorm tiles producing level l; a tile of a level that
   // feeds a layer also computes its 64 columns' share of that layer's router
   // logits (W_r[:, tile] . gamma x), its router columns streamed through the
-  // ring like GEMV weights: one stage per 128 experts
+  // ring like GEMV weights: one stage per 128 experts.  The tile whose arrival
+  // completes the level then sums the shares and runs the layer's top-k,
+  // softmax and slot compaction, and signals the routing counter.
   auto emit_norm = [&](int l) {
     for (int r = 0; r < NR; ++r) {
       Task t = make_task(OP_RN, l, l * PH + 0);
@@ -261,6 +265,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
       if (l < L) {
         t.w[D_NSTAGE] = (E + kRouterRowsPerStage - 1) / kRouterRowsPerStage;
         t.w[D_MAP0] = map_of(l, kMapRouter);
+        fuse(t, F_TOPK, lay.narr(l), NR, lay.rtr(l));
       }
       if (l > 0) add_wait(t, lay.dt(l - 1, r), Hkv + S);
       add_signal(t, lay.norm(l));
@@ -271,14 +276,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   emit_norm(0);
   for (int l = 0; l < L; ++l) {
     if (l > 0) emit_norm(l);
-    // -- top-k over the router logits summed from the norm tiles' shares
-    {
-      Task t = make_task(OP_TOPK, l, l * PH + 2);
-      add_wait(t, lay.norm(l), NR);
-      add_signal(t, lay.rtr(l));
-      tasks.push_back(t);
-    }
-    targets[lay.rtr(l)] += 1;   // one top-k per layer
+    targets[lay.rtr(l)] += 1;   // one top-k per layer, by the last norm tile
     // -- QKV tiles (grouped by KV group so attention of a group starts early)
     for (int g = 0; g < Hkv; ++g) {
       auto emit_rows = [&](int row_begin, int rows) {

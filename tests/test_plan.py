@@ -25,8 +25,9 @@ ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 
 D_X0, D_X1, D_X2 = 29, 30, 31
-F_COMBINE = 128   # the only last-arriver flag: the attention merge
-FUSED = F_COMBINE
+F_COMBINE = 128   # last-arriver work: the attention merge of a (token, KV head)
+F_TOPK = 256      # last-arriver work: the top-k of the layer a norm level feeds
+FUSED = F_COMBINE | F_TOPK
 
 
 def signal_sets(desc, targets):
@@ -113,14 +114,21 @@ def test_30b_b1_plan_structure():
     L, d = shape["n_layers"], shape["d_model"]
     qkv_rows = (shape["n_q_heads"] + 2 * shape["n_kv_heads"]) * shape["head_dim"]
     assert ops[OP_QKV] == L * qkv_rows // 16
-    # the norm tiles produce the router logits: no router tiles, and each
-    # layer's top-k waits for all of the layer's norm tiles
+    # the norm tiles produce the router logits: no router tiles, no top-k
+    # tasks; the norm tile whose arrival completes a level runs the top-k of
+    # the layer it feeds and signals the counter the layer's expert tiles wait on
     assert ops[OP_ROUTER] == 0
     assert ops[OP_RN] == (L + 1) * d // 64
-    assert ops[OP_TOPK] == L
-    tk = desc[desc[:, D_OP] == OP_TOPK]
-    assert np.all(tk[:, D_NWAIT] == 1) and np.all(tk[:, D_W0N] == d // 64)
+    assert ops[OP_TOPK] == 0
     rn = desc[desc[:, D_OP] == OP_RN]
+    feeds = rn[rn[:, D_LAYER] < L]
+    assert np.all(feeds[:, D_FLAGS] & F_TOPK) and np.all(feeds[:, D_X1] == d // 64)
+    assert not np.any(rn[rn[:, D_LAYER] == L][:, D_FLAGS] & F_TOPK)
+    gu = desc[desc[:, D_OP] == OP_GATEUP]
+    for l in (0, 5, L - 1):
+        join = set(feeds[feeds[:, D_LAYER] == l][:, D_X2].tolist())
+        assert join == set(gu[gu[:, D_LAYER] == l][:, D_PW].tolist())
+        assert len(set(feeds[feeds[:, D_LAYER] == l][:, D_X0].tolist())) == 1
     # a norm tile of a level that feeds a layer streams its router columns:
     # one ring stage per 128 experts; the final norm streams nothing
     E = shape["n_experts"]
@@ -131,7 +139,8 @@ def test_30b_b1_plan_structure():
     lv = rn[rn[:, D_LAYER] < L]
     assert np.all(lv[:, D_MAP0] == lv[:, D_LAYER] * 8 + 2)
     for l in (0, 5):
-        ctr = tk[tk[:, D_LAYER] == l][0, D_W0]
+        q = desc[(desc[:, D_OP] == OP_QKV) & (desc[:, D_LAYER] == l)]
+        ctr = q[0, D_W0]
         senders = rn[(rn[:, D_LAYER] == l)]
         assert np.all(senders[:, D_S0] == ctr) and len(senders) == d // 64
     a_multi = desc[(desc[:, D_OP] == OP_ATTN) & (desc[:, D_D] > 1)]
