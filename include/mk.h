@@ -147,6 +147,30 @@ mk_status mk_decode_step(mk_ctx* ctx, const int32_t* tokens, const int32_t* posi
                          const int32_t* page_table, const int32_t* seq_lens,
                          float* logits, void* stream);
 
+/* Greedy decoding: n_steps fused steps back to back on `stream`, with no host
+ * round trip between them.  Step i reads tokens, positions and seq_lens as
+ * mk_decode_step does and writes logits; its last LM-head tile to finish also
+ * writes each sequence's greedy token (the largest logit, the lowest token id
+ * among equal ones) to out_tokens[i][b] and to tokens[b], the next step's
+ * input, and advances positions[b] and seq_lens[b] by one (once if both
+ * pointers name the same buffer).  Each LM-head tile folds its rows' best
+ * logit per sequence into a 64-bit key with one atomicMax, so the step's
+ * argmax costs no extra pass over the logits.  This is the greedy step after
+ * the LM head of the pages' serving loop (aimodeling.com, "Cohere megakernel
+ * engine: one CUDA file, 1.58x vLLM on H100", "From demo to a full serving
+ * system"), done on the device.
+ *   tokens, positions, seq_lens  int32[batch], device, read and updated
+ *   page_table  as for mk_decode_step; it must already map the page of every
+ *               token the n_steps steps append
+ *   logits      float32[batch][vocab], device: the last step's logits
+ *   out_tokens  int32[n_steps][batch], device
+ * The schedule's plan length must cover seq_lens + n_steps (else the step
+ * that outgrows it latches MK_ERR_STATE).  Asynchronous like mk_decode_step;
+ * n_steps == 0 does nothing.                                               */
+mk_status mk_decode_greedy(mk_ctx* ctx, int32_t n_steps, int32_t* tokens, int32_t* positions,
+                           const int32_t* page_table, int32_t* seq_lens, float* logits,
+                           int32_t* out_tokens, void* stream);
+
 /* Same step as mk_decode_step, but issued as one launch of the same task
  * interpreter per operation phase (about nine per layer), so kernel
  * boundaries replace the cross-SM counters.  This is the unfused per-op

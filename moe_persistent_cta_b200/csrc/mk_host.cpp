@@ -55,7 +55,7 @@ struct mk_ctx {
   DevBuf desc, phase_desc;
   bool phases_uploaded = false;
   DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, rpart, route, expert_a, afrag,
-      moe_part, trace;
+      moe_part, amax, trace;
   DevBuf selftest;   // one descriptor + two counters for mk_selftest_timeout
   bool tracing = false;
   // schedule
@@ -180,7 +180,7 @@ void mk_destroy(mk_ctx* c) {
   for (DevBuf* b : {&c->desc, &c->phase_desc, &c->x, &c->actA,
                     &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
                     &c->rlogits, &c->rpart, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
-                    &c->trace, &c->selftest})
+                    &c->amax, &c->trace, &c->selftest})
     release(*b);
   c->plan.release();
   delete c;
@@ -389,6 +389,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   ENSURE(expert_a, (size_t)L * S * B * s.F * 4);
   ENSURE(afrag, (size_t)L * S * afrag_bytes);
   ENSURE(moe_part, (size_t)L * s.k * B * d * 4);
+  ENSURE(amax, (size_t)B * 8);
   ENSURE(desc, (size_t)plan.n_tasks * mk::kDescWords * 4);
 #undef ENSURE
   if (plan.n_counters > c->counters_cap) {
@@ -402,6 +403,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   if (cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap) != cudaSuccess)
     return fail(MK_ERR_CUDA);
   if (cudaMemset(c->route.ptr, 0, c->route.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
+  if (cudaMemset(c->amax.ptr, 0, c->amax.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
   if (cudaMemcpy(c->desc.ptr, plan.desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
                  cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(MK_ERR_CUDA);
@@ -444,6 +446,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.expert_a = static_cast<float*>(c->expert_a.ptr);
   p.afrag = static_cast<uint8_t*>(c->afrag.ptr);
   p.moe_part = static_cast<float*>(c->moe_part.ptr);
+  p.amax = static_cast<unsigned long long*>(c->amax.ptr);
   p.status = c->d_status;
   p.n_stages = sl.n_stages;
   p.nA = sl.nA;
@@ -473,9 +476,17 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   return MK_OK;
 }
 
+// A greedy step's writable views of its inputs and its row of the token output.
+struct Greedy {
+  int32_t* tokens;
+  int32_t* positions;
+  int32_t* seq_lens;
+  int32_t* out;
+};
+
 static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* positions,
                              const int32_t* page_table, const int32_t* seq_lens, float* logits,
-                             void* stream, bool unfused) {
+                             void* stream, bool unfused, const Greedy* greedy = nullptr) {
   if (!c) return MK_ERR_INVALID;
   if (!c->have_schedule) return MK_ERR_STATE;
   if (!tokens || !positions || !page_table || !seq_lens || !logits) return MK_ERR_INVALID;
@@ -487,6 +498,12 @@ static mk_status launch_step(mk_ctx* c, const int32_t* tokens, const int32_t* po
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   p.logits = logits;
+  if (greedy) {
+    p.g_tok = greedy->tokens;
+    p.g_pos = greedy->positions;
+    p.g_len = greedy->seq_lens;
+    p.g_out = greedy->out;
+  }
   p.timeout_cycles = deadline_cycles(c, c->timeout_ns);
   p.epoch = c->epoch + 1;
   cudaError_t e = cudaSuccess;
@@ -541,6 +558,18 @@ mk_status mk_decode_step_unfused(mk_ctx* c, const int32_t* tokens, const int32_t
   return launch_step(c, tokens, positions, page_table, seq_lens, logits, stream, true);
 }
 
+mk_status mk_decode_greedy(mk_ctx* c, int32_t n_steps, int32_t* tokens, int32_t* positions,
+                           const int32_t* page_table, int32_t* seq_lens, float* logits,
+                           int32_t* out_tokens, void* stream) {
+  if (!c) return MK_ERR_INVALID;
+  if (n_steps < 0 || (n_steps > 0 && !out_tokens)) return MK_ERR_INVALID;
+  for (int32_t i = 0; i < n_steps; ++i) {
+    const Greedy g{tokens, positions, seq_lens, out_tokens + (size_t)i * c->B};
+    MK_TRY(launch_step(c, tokens, positions, page_table, seq_lens, logits, stream, false, &g));
+  }
+  return MK_OK;
+}
+
 mk_status mk_check(mk_ctx* c, int32_t* device_status, int32_t* detail) {
   if (!c) return MK_ERR_INVALID;
   MK_CUDA(cudaSetDevice(c->device));
@@ -559,6 +588,7 @@ mk_status mk_check(mk_ctx* c, int32_t* device_status, int32_t* detail) {
     MK_CUDA(cudaMemset(c->d_status, 0, sizeof(st)));
     if (c->d_counters)
       MK_CUDA(cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap));
+    if (c->amax.ptr) MK_CUDA(cudaMemset(c->amax.ptr, 0, c->amax.bytes));
     c->epoch = 0;
     return st[mk::ST_CODE] != 0 ? (mk_status)st[mk::ST_CODE] : MK_ERR_DEVICE;
   }
@@ -718,6 +748,7 @@ mk_status launch_step_in(mk_ctx* c, const int32_t* tokens, const int32_t* positi
   p.timeout_cycles = deadline_cycles(c, c->timeout_ns);
   p.epoch = 1;
   p.trace = nullptr;
+  p.g_tok = p.g_pos = p.g_len = p.g_out = nullptr;
   p.n_ctas = c->plan.n_ctas;
   p.desc = static_cast<const int32_t*>(c->desc.ptr);
   p.n_tasks = c->plan.n_tasks;

@@ -127,8 +127,9 @@ enum Flags : int32_t {
   // D_X0 (D_X1 arrivals per step); the task that completes the count does the
   // join below and then signals counter D_X2.
   F_COMBINE = 128,   // attention chunk: log-sum-exp merge of the (b, g) chunks
-  F_TOPK = 256       // norm tile: router logits, top-k, softmax and slot compaction
+  F_TOPK = 256,      // norm tile: router logits, top-k, softmax and slot compaction
                      // of the layer the level feeds
+  F_ARGMAX = 512     // LM-head tile: in a greedy step, the tokens of the step
 };
 
 // ------------------------------------------------- resolved entry words ---
@@ -181,6 +182,14 @@ struct Params {
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* logits;
+  // greedy steps (null otherwise): the step's token ids (read by the
+  // embedding, overwritten with the greedy tokens), positions and lengths
+  // (advanced by one), and this step's row of the caller's token output
+  int32_t* g_tok;
+  int32_t* g_pos;
+  int32_t* g_len;
+  int32_t* g_out;
+  unsigned long long* amax;   // [B] best (logit, lowest row) keys, zero between steps
   // context buffers
   float* x;          // [L+1][B][d]
   uint8_t* actA;     // [L+1][actA_bytes]

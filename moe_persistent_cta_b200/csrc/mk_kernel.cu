@@ -1052,6 +1052,76 @@ struct EpiParams {
         PC(in_reg(p.part_cols)) {}
 };
 
+// Order-preserving key of a float: a larger float gives a larger unsigned key.
+__device__ __forceinline__ uint32_t ordered_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// LM-head tile epilogue: the logits of the tile's rows for every token, and in
+// a greedy step each token's best logit of the tile with its lowest row,
+// folded into amax[n] as the 64-bit key (ordered logit << 32 | ~row), whose
+// maximum over all tiles is the largest logit at the lowest row.
+__device__ __forceinline__ void lm_epilogue(const EpiParams& p, const Params& pr,
+                                            const int32_t* ent, const float* part,
+                                            const float* rs) {
+  const int lane = threadIdx.x & 31;
+  const int R = ent[D_R], row0 = ent[D_ROW0];
+  const int MT = R / 16, kcps = 8 / MT;
+  const int PC = p.PC;
+  unsigned long long* const amax = pr.g_tok ? pr.amax : nullptr;
+  for (int n = 0; n < p.B; ++n) {
+    uint32_t bk = 0u;
+    int brow = 0x7fffffff;
+    for (int r = lane; r < R; r += 32) {   // rows ascend per lane: the first max is kept
+      const int mt = r >> 4, r16 = r & 15;
+      float s0 = 0.f;
+      for (int kc = 0; kc < kcps; ++kc) s0 += part[((kc * MT + mt) * 16 + r16) * PC + n];
+      const int row = row0 + r;
+      if (row < p.V) {
+        const float v = s0 * rs[n];
+        p.logits[(size_t)n * p.V + row] = v;
+        const uint32_t key = ordered_key(v);
+        if (key > bk) {
+          bk = key;
+          brow = row;
+        }
+      }
+    }
+    if (amax) {
+      const uint32_t mk_ = __reduce_max_sync(FULL, bk);
+      const int mrow = __reduce_min_sync(FULL, bk == mk_ ? brow : 0x7fffffff);
+      if (lane == 0 && mrow != 0x7fffffff)
+        atomicMax(amax + n, ((unsigned long long)mk_ << 32) | (unsigned long long)(~(uint32_t)mrow));
+    }
+  }
+}
+
+// After an LM-head tile: its arrival; the tile that completes the step's
+// count (it has acquired every tile's keys) takes each token's key (resetting
+// it to zero for the next step) and, in a greedy step, writes the token, feeds
+// it to the next step and advances the position and length by one.
+__device__ __noinline__ void lm_finish(const Params& p, const int32_t* ent) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    const uint32_t old = atom_add_acq_rel(p.counters + ent[D_X0], 1u);
+    last = old + 1u == p.epoch * (uint32_t)ent[D_X1];
+  }
+  if (!__shfl_sync(FULL, last, 0)) return;
+  if (p.g_tok && lane < p.B) {
+    const unsigned long long key = atomicExch(p.amax + lane, 0ull);
+    const int tok = (int)~(uint32_t)key;
+    p.g_out[lane] = tok;
+    p.g_tok[lane] = tok;
+    p.g_pos[lane] += 1;
+    if (p.g_len != p.g_pos) p.g_len[lane] += 1;   // one buffer may serve as both
+  }
+  __syncwarp();
+  if (lane == 0) red_release_add(p.counters + ent[D_X2], 1u);
+}
+
 __device__ __forceinline__ void gemv_epilogue(const EpiParams& p, const int32_t* ent,
                                               const float* part, const float* rs) {
   const int lane = threadIdx.x & 31;
@@ -1074,9 +1144,6 @@ __device__ __forceinline__ void gemv_epilogue(const EpiParams& p, const int32_t*
     switch (op) {
       case OP_QKV:
         p.qkv[((size_t)layer * p.B + n) * p.qkvR + row] = s0 * rs[n];
-        break;
-      case OP_LMHEAD:
-        if (row < p.V) p.logits[(size_t)n * p.V + row] = s0 * rs[n];
         break;
       case OP_OPROJ: {
         const int g = ent[D_B];
@@ -1996,8 +2063,14 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
     if (!warp_wait(p, sm.pfull(pb), (ngemv >> 1) & 1u, 601)) break;
     const int t = ent[32 + R_TASK];
     if (lane == 0) cstamp(p, t, T_K4);
-    gemv_epilogue(ep, ent, part0 + pb * kConsumerWarps * 16 * PC,
-                  rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch);
+    const float* part = part0 + pb * kConsumerWarps * 16 * PC;
+    const float* rs = rstd_ring + (ent[D_LAYER] & (kRstdRing - 1)) * kMaxBatch;
+    if (op == OP_LMHEAD) {
+      lm_epilogue(ep, p, ent, part, rs);
+      if (ent[D_FLAGS] & F_ARGMAX) lm_finish(p, ent);
+    } else {
+      gemv_epilogue(ep, ent, part, rs);
+    }
     __syncwarp();
     if (lane == 0) {
       stamp(p, t, T_C_END);

@@ -140,7 +140,7 @@ struct Task {
 
 struct Layout {
   int L, B, S, Hkv, NR;
-  int norm0, narr0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmdone, total;
+  int norm0, narr0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmarr, lmdone, total;
   void build(int L_, int B_, int S_, int Hkv_, int NR_) {
     L = L_; B = B_; S = S_; Hkv = Hkv_; NR = NR_;
     int c = 0;
@@ -152,6 +152,7 @@ struct Layout {
     atto0 = c; c += L * Hkv;
     slot0 = c; c += L * S;
     dt0 = c; c += L * NR;
+    lmarr = c; c += 1;
     lmdone = c; c += 1;
     total = c;
   }
@@ -411,11 +412,12 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
     t.w[D_MAP0] = L * kMapsPerLayer;
     t.w[D_NSTAGE] = 8 * (d / 64) / 8;
     add_wait(t, lay.norm(L), NR);
-    add_signal(t, lay.lmdone);
-    targets[lay.lmdone] += 1;
+    // the last LM-head tile to finish completes a greedy step's tokens
+    fuse(t, F_ARGMAX, lay.lmarr, n_lm, lay.lmdone);
     t.w[D_ACT] = ACT_A;
     tasks.push_back(t);
   }
+  targets[lay.lmdone] += 1;
 
   // ---- priority order: stable sort by (layer, operation rank)
   static const int kRank[OP_COUNT] = {

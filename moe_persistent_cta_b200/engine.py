@@ -91,6 +91,27 @@ class Decoder:
                 _ptr(logits), c_void_p(s.cuda_stream))
         mk.check_status(st, "mk_decode_step")
 
+    def greedy(self, n_steps: int, tokens: torch.Tensor, positions: torch.Tensor,
+               page_table: torch.Tensor, seq_lens: torch.Tensor, logits: torch.Tensor,
+               out_tokens: torch.Tensor, stream=None) -> None:
+        """n_steps greedy steps on the device (mk_decode_greedy): tokens,
+        positions and seq_lens are updated in place, out_tokens[i] receives
+        step i's tokens.  Asynchronous."""
+        for t in (tokens, positions, page_table, seq_lens, out_tokens):
+            if t.dtype != torch.int32 or not t.is_cuda:
+                raise TypeError("greedy inputs and outputs must be int32 CUDA tensors")
+        if logits.dtype != torch.float32 or not logits.is_cuda:
+            raise TypeError("logits must be a float32 CUDA tensor")
+        if page_table.shape[-1] != self.max_pages:
+            raise ValueError("page_table row length differs from the schedule's")
+        if out_tokens.numel() < n_steps * self.batch:
+            raise ValueError("out_tokens holds fewer than n_steps x batch tokens")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        st = mk.lib.mk_decode_greedy(self._ctx, int(n_steps), _ptr(tokens), _ptr(positions),
+                                     _ptr(page_table), _ptr(seq_lens), _ptr(logits),
+                                     _ptr(out_tokens), c_void_p(s.cuda_stream))
+        mk.check_status(st, "mk_decode_greedy")
+
     def check(self):
         """Synchronize and return (status, detail list)."""
         st = c_int32(0)

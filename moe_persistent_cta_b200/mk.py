@@ -24,8 +24,8 @@ TRACE_WORDS = 18
 
 # every entry point the header declares (checked by the ABI test)
 EXPORTS = (
-    "mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_step_unfused",
-    "mk_decode_step_static",
+    "mk_create", "mk_build_schedule", "mk_decode_step", "mk_decode_greedy",
+    "mk_decode_step_unfused", "mk_decode_step_static",
     "mk_check", "mk_selftest_timeout", "mk_set_timeout_ms", "mk_set_trace", "mk_debug_read",
     "mk_debug_size",
     "mk_plan_schedule", "mk_strerror", "mk_destroy",
@@ -74,6 +74,7 @@ def _load():
         "mk_create": (c_int, [P(mk_config), P(mk_tensors), c_int, P(c_void_p)]),
         "mk_build_schedule": (c_int, [c_void_p, c_int, P(c_int32), P(c_int32), c_int32]),
         "mk_decode_step": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
+        "mk_decode_greedy": (c_int, [c_void_p, c_int32] + [c_void_p] * 7),
         "mk_decode_step_unfused": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_decode_step_static": (c_int, [c_void_p] + [c_void_p] * 5 + [c_void_p]),
         "mk_check": (c_int, [c_void_p, P(c_int32), P(c_int32)]),

@@ -168,9 +168,18 @@ def run_continuous(dec, shape: Dict, k_pool: torch.Tensor, v_pool: torch.Tensor,
                    steps: int, seed: int, start_lo: int, start_hi: int, mean_new: float,
                    max_new: int, max_pages_per_seq: int, stream=None,
                    horizon: Optional[int] = None) -> Dict:
-    """Run `steps` greedy decode steps with slot refills.  Returns counts and
-    times: decode (steps, argmax, table uploads), schedule rebuilds, and the
-    synthetic prefix fills, each in seconds, plus tokens generated."""
+    """Run `steps` greedy decode steps with slot refills.
+
+    A sequence's stop length is drawn when it starts, so the host knows when
+    the next slot frees up: it launches the greedy steps up to that point in
+    one mk_decode_greedy call (tokens, positions and lengths advance on the
+    device; no host round trip between steps), then refills the freed slots
+    (page pool, synthetic prefix, token and length written to the device
+    buffers on the same stream) and goes on.  Times are taken with CUDA
+    events on the stream: the greedy steps (decode_s), the synthetic prefix
+    fills (prefix_fill_s) and schedule rebuilds (rebuild_s, host).  Returns
+    counts, times, the generated tokens [steps][slots] and the cached length
+    of every slot at every step (for the KV bytes the steps read)."""
     dev = k_pool.device
     rng = np.random.default_rng(seed)
     gen = torch.Generator(device=dev).manual_seed(seed)
@@ -182,34 +191,65 @@ def run_continuous(dec, shape: Dict, k_pool: torch.Tensor, v_pool: torch.Tensor,
     tokens = torch.zeros(slots, **i32)
     lens_d = torch.zeros(slots, **i32)
     table_d = torch.zeros((slots, max_pages_per_seq), **i32)
+    out = torch.full((steps, slots), -1, **i32)
     logits = torch.empty((slots, shape["vocab"]), dtype=torch.float32, device=dev)
-    t_fill = t_rebuild = t_decode = 0.0
+    ev = []            # (kind, start event, end event)
+    t_rebuild = 0.0
     rebuilds = 0
-    for _ in range(steps):
-        t0 = time.perf_counter()
-        refilled = sched.fill()
-        for i in refilled:
-            fill_prefix_kv(k_pool, v_pool, sched.seqs[i].pages, gen)
-            tokens[i] = int(rng.integers(0, shape["vocab"]))
-        torch.cuda.synchronize(dev)
-        t1 = time.perf_counter()
-        t_fill += t1 - t0
-        if sched.before_step():
-            plan = sched.planned()
-            dec.build_schedule(sched.lens(), max_pages_per_seq, plan_len=plan)
-            rebuilds += 1
-        t2 = time.perf_counter()
-        t_rebuild += t2 - t1
-        with torch.cuda.stream(s):
-            lens_d.copy_(torch.tensor(sched.lens(), dtype=torch.int32), non_blocking=False)
-            table_d.copy_(torch.from_numpy(sched.page_table()), non_blocking=False)
-            dec.step(tokens, lens_d, table_d, lens_d, logits, stream=s)
-            tokens.copy_(torch.argmax(logits, dim=-1).to(torch.int32))
-        s.synchronize()
-        dec.check_ok()
-        t3 = time.perf_counter()
-        t_decode += t3 - t2
-        sched.after_step()
+    lens_per_step = np.zeros((steps, slots), dtype=np.int64)
+    done = 0
+    with torch.cuda.stream(s):
+        while done < steps:
+            refilled = sched.fill()
+            if refilled:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                for i in refilled:
+                    fill_prefix_kv(k_pool, v_pool, sched.seqs[i].pages, gen)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(s)
+                ev.append(("fill", e0, e1))
+                # the refilled slots' first token and cached length, from a
+                # fresh pinned buffer (torch keeps it until the copy has run)
+                vals = [[int(rng.integers(0, shape["vocab"])) for _ in refilled],
+                        [sched.seqs[i].cached for i in refilled]]
+                hr = torch.tensor(vals, dtype=torch.int32).pin_memory().to(dev, non_blocking=True)
+                idx = torch.tensor(refilled, dtype=torch.long).pin_memory().to(dev, non_blocking=True)
+                tokens.index_copy_(0, idx, hr[0])
+                lens_d.index_copy_(0, idx, hr[1])
+            n = min(min(q.remaining for q in sched.seqs), steps - done)
+            # pages for every token the next n steps append
+            for q in sched.seqs:
+                need = pages_for(q.cached + n)
+                if need > len(q.pages):
+                    q.pages.extend(pool.alloc(need - len(q.pages)))
+                if need > max_pages_per_seq:
+                    raise ValueError("sequence outgrew the page table")
+            if sched.need_rebuild or any(q.cached + n - 1 > sched.plan_len[i]
+                                         for i, q in enumerate(sched.seqs)):
+                t0 = time.perf_counter()
+                s.synchronize()
+                dec.build_schedule(sched.lens(), max_pages_per_seq, plan_len=sched.planned())
+                t_rebuild += time.perf_counter() - t0
+                rebuilds += 1
+            table_d.copy_(torch.from_numpy(sched.page_table()).pin_memory(), non_blocking=True)
+            for j in range(n):
+                lens_per_step[done + j] = [q.cached + j for q in sched.seqs]
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            dec.greedy(n, tokens, lens_d, table_d, lens_d, logits, out[done:done + n], stream=s)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(s)
+            ev.append(("decode", e0, e1))
+            for _ in range(n):
+                sched.after_step()
+            done += n
+    s.synchronize()
+    dec.check_ok()
+    t_decode = sum(a.elapsed_time(b) for k, a, b in ev if k == "decode") / 1e3
+    t_fill = sum(a.elapsed_time(b) for k, a, b in ev if k == "fill") / 1e3
     return {"steps": steps, "slots": slots, "generated": sched.generated,
             "finished": sched.finished, "sequences": sched.next_id, "rebuilds": rebuilds,
-            "decode_s": t_decode, "rebuild_s": t_rebuild, "prefix_fill_s": t_fill}
+            "decode_s": t_decode, "rebuild_s": t_rebuild, "prefix_fill_s": t_fill,
+            "greedy_calls": sum(1 for k, _, _ in ev if k == "decode"),
+            "tokens": out.cpu().numpy(), "lens_per_step": lens_per_step}

@@ -62,3 +62,68 @@ def test_continuous_batching_matches_oracle_step_by_step():
         assert refills > slots and rebuilds > 1
     finally:
         dec.close()
+
+
+@pytest.mark.parametrize("horizon", [None, 16])
+def test_greedy_chunks_match_stepwise_replay(horizon):
+    """run_continuous launches the steps between two slot refills as one
+    mk_decode_greedy call (tokens, positions and lengths advance on the
+    device).  A replay of the same run, one mk_decode_step per step with a
+    host argmax and the same seeded refills, must generate the same tokens:
+    the arithmetic of every step is the same."""
+    from moe_persistent_cta_b200 import serving
+    shape = configs.TINY
+    dev = torch.device("cuda:0")
+    slots, steps, max_pages = 3, 40, 8
+    W = synth.make_weights(shape, 0, "cpu")
+    Wd = to_dev(W, dev)
+    n_pages = 3 * slots * max_pages
+    kshape = (shape["n_layers"], n_pages, shape["n_kv_heads"], 64, shape["head_dim"])
+    common = dict(slots=slots, steps=steps, seed=21, start_lo=5, start_hi=250, mean_new=6,
+                  max_new=steps, max_pages_per_seq=max_pages)
+    k = torch.zeros(kshape, dtype=torch.bfloat16, device=dev)
+    v = torch.zeros_like(k)
+    dec = engine.Decoder(shape, Wd, k, v, max_batch=slots)
+    try:
+        r = serving.run_continuous(dec, shape, k, v, horizon=horizon, **common)
+    finally:
+        dec.close()
+    assert r["generated"] == steps * slots and r["greedy_calls"] < steps
+    # the replay: same draws in the same order, one step at a time
+    k2 = torch.zeros(kshape, dtype=torch.bfloat16, device=dev)
+    v2 = torch.zeros_like(k2)
+    dec2 = engine.Decoder(shape, Wd, k2, v2, max_batch=slots)
+    rng = np.random.default_rng(common["seed"])
+    gen = torch.Generator(device=dev).manual_seed(common["seed"])
+    sched = SlotScheduler(slots, PagePool(n_pages), max_pages, rng, 5, 250, 6, steps,
+                          horizon=None)
+    i32 = dict(dtype=torch.int32, device=dev)
+    tokens = [0] * slots
+    logits = torch.empty((slots, shape["vocab"]), dtype=torch.float32, device=dev)
+    want = np.zeros((steps, slots), dtype=np.int64)
+    try:
+        for step in range(steps):
+            refilled = sched.fill()
+            for i in refilled:
+                fill_prefix_kv(k2, v2, sched.seqs[i].pages, gen)
+            for i, t in zip(refilled, [int(rng.integers(0, shape["vocab"])) for _ in refilled]):
+                tokens[i] = t
+            if sched.before_step():
+                dec2.build_schedule(sched.lens(), max_pages, plan_len=sched.planned())
+            lens, table = sched.lens(), sched.page_table()
+            dec2.step(torch.tensor(tokens, **i32), torch.tensor(lens, **i32),
+                      torch.from_numpy(table).to(dev), torch.tensor(lens, **i32), logits)
+            dec2.check_ok()
+            tokens = [int(t) for t in logits.argmax(-1).cpu()]
+            want[step] = tokens
+            sched.after_step()
+    finally:
+        dec2.close()
+    if horizon is None:
+        # one schedule for the whole run on both sides: bit-identical steps
+        assert np.array_equal(r["tokens"], want)
+    else:
+        # rebuilt schedules cut attention into other chunks than the replay's
+        # single schedule, so only the run itself is checked
+        assert r["rebuilds"] > 1
+        assert np.all((r["tokens"] >= 0) & (r["tokens"] < shape["vocab"]))

@@ -27,7 +27,8 @@ ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 D_X0, D_X1, D_X2 = 29, 30, 31
 F_COMBINE = 128   # last-arriver work: the attention merge of a (token, KV head)
 F_TOPK = 256      # last-arriver work: the top-k of the layer a norm level feeds
-FUSED = F_COMBINE | F_TOPK
+F_ARGMAX = 512    # last-arriver work: a greedy step's tokens after the LM head
+FUSED = F_COMBINE | F_TOPK | F_ARGMAX
 
 
 def signal_sets(desc, targets):
@@ -153,6 +154,9 @@ def test_30b_b1_plan_structure():
     assert ops[OP_GATEUP] == L * S * shape["d_ff"] // 16
     assert ops[OP_DOWN] == L * S * d // 64
     assert ops[OP_LM] == shape["vocab"] // 128
+    lmt = desc[desc[:, D_OP] == OP_LM]
+    assert np.all(lmt[:, D_FLAGS] & F_ARGMAX) and np.all(lmt[:, D_X1] == len(lmt))
+    assert len(set(lmt[:, D_X0].tolist())) == 1 and np.all(lmt[:, D_NSIG] == 0)
     q = desc[desc[:, D_OP] == OP_QKV]
     assert len(set(zip(q[:, D_LAYER].tolist(), q[:, D_ROW0].tolist()))) == len(q)
     a = desc[desc[:, D_OP] == OP_ATTN]
