@@ -424,6 +424,10 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.afrag_bytes = afrag_bytes;
   p.route_words = rwords;
   p.counters = c->d_counters;
+  p.exit_ctr = plan.exit_ctr;
+  p.slot_ctr0 = plan.slot_ctr0;
+  p.dt_ctr0 = plan.dt_ctr0;
+  p.n_ff = plan.n_ff;
   p.tmaps = c->d_tmaps;
   p.embed = static_cast<const uint16_t*>(c->embed);
   p.final_norm = static_cast<const uint16_t*>(c->final_norm);
@@ -460,6 +464,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.off_ring = sl.off_ring;
   p.off_epi = sl.off_epi;
   p.off_ptrs = sl.off_ptrs;
+  p.off_rcache = sl.off_rcache;
   p.part_cols = sl.part_cols;
   p.smem_bytes = sl.dyn_bytes;
 
@@ -785,7 +790,8 @@ mk_status mk_selftest_timeout(mk_ctx* c, int32_t timeout_ms, int32_t* device_sta
   h[mk::D_MAP0] = -1;
   h[mk::D_MAP1] = -1;
   h[mk::D_ACT] = mk::ACT_NONE;
-  // words kDescWords.. : counter 0 (never signalled), counter 1 (dispenser)
+  // words kDescWords.. : counter 0 (never signalled), counter 1 (dispenser),
+  // counter 2 (producers' exit count)
   MK_CUDA(cudaMemcpy(c->selftest.ptr, h, bytes, cudaMemcpyHostToDevice));
   MK_CUDA(cudaMemset(c->d_status, 0, sizeof(int32_t) * 16));
   Params p = c->base;
@@ -793,6 +799,7 @@ mk_status mk_selftest_timeout(mk_ctx* c, int32_t timeout_ms, int32_t* device_sta
   p.counters = reinterpret_cast<uint32_t*>(static_cast<int32_t*>(c->selftest.ptr) + mk::kDescWords);
   p.n_tasks = 1;
   p.grab = 1;
+  p.exit_ctr = 2;
   p.n_ctas = c->plan.n_ctas;
   p.epoch = 1;
   p.trace = nullptr;

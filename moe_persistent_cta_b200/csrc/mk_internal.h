@@ -81,7 +81,7 @@ enum Op : int32_t {
   OP_RN = 1,        // fused residual add + RMSNorm statistics for one 64-row tile
   OP_QKV = 2,       // QKV projection tile (RoPE/append happen in OP_ATTN)
   OP_ROUTER = 3,    // (unused: the norm tiles produce the router logits)
-  OP_TOPK = 4,      // (unused: the last-arriving norm tile of a level runs the top-k)
+  OP_TOPK = 4,      // top-k + softmax + expert-slot compaction
   OP_ATTN = 5,      // paged GQA decode attention over one KV chunk (+RoPE, append)
   OP_COMBINE = 6,   // (unused: the last-arriving attention chunk of (b, g) merges)
   OP_OPROJ = 7,     // O-proj tile, split-K by KV group
@@ -97,7 +97,8 @@ enum DescField : int {
   D_LAYER = 1,
   D_A = 2,          // tile / batch index / slot
   D_B = 3,          // tile / group
-  D_C = 4,          // chunk
+  D_C = 4,          // attention: chunk; expert tiles: list index one past the
+                    // layer's last tile of the same operation (see D_A)
   D_D = 5,          // chunk count
   D_FLAGS = 6,
   D_NWAIT = 7,
@@ -127,8 +128,6 @@ enum Flags : int32_t {
   // D_X0 (D_X1 arrivals per step); the task that completes the count does the
   // join below and then signals counter D_X2.
   F_COMBINE = 128,   // attention chunk: log-sum-exp merge of the (b, g) chunks
-  F_TOPK = 256,      // norm tile: router logits, top-k, softmax and slot compaction
-                     // of the layer the level feeds
   F_ARGMAX = 512     // LM-head tile: in a greedy step, the tokens of the step
 };
 
@@ -160,11 +159,19 @@ struct Params {
   int afrag_bytes;     // per (layer, slot): B x (F + kActPad) floats
   int route_words;     // per layer
   // schedule: one list in topological priority order; CTAs take the next
-  // task with an atomic add on counters[grab]
+  // task with an atomic add on counters[grab].  The dispenser starts every
+  // launch at 0: the last producer to leave (counted on counters[exit_ctr])
+  // zeroes it, so it may also be moved forward past tasks that turn out to
+  // be empty (expert tiles of unused slots).
   const int32_t* desc;     // [n_tasks][kDescWords]
   int n_tasks;
   int n_ctas;
   int grab;                // counter index of the task dispenser
+  int exit_ctr;            // counter index of the producers' exit count
+  // counter layout the top-k needs to stand in for the unused slots' tiles:
+  // slot counters [L][S] from slot_ctr0, down-tile row counters [L][NR]
+  // from dt_ctr0 (n_ff gate/up tiles per slot)
+  int slot_ctr0, dt_ctr0, n_ff;
   uint32_t* counters;
   uint32_t epoch;
   // tensors
@@ -214,6 +221,7 @@ struct Params {
   int off_epi;       // GEMV partials [2][kConsumerWarps][16][part_cols], then the
                      // per-level 1/rms ring [kRstdRing][kMaxBatch]
   int off_ptrs;      // per-layer pointer table, copied in at launch (see PtrTable)
+  int off_rcache;    // the producer's copy of one layer's routing table (route_words)
   int part_cols;     // token columns per partial row: B for B <= 2, else 8
   int smem_bytes;
 };
@@ -258,6 +266,8 @@ struct Plan {
   int r_qkv = 16;
   int grab = 0;                      // dispenser counter of the fused list
   int grab_phase0 = 0;               // dispenser counters of the phase lists
+  int exit_ctr = 0;                  // producers' exit count (resets the dispenser)
+  int slot_ctr0 = 0, dt_ctr0 = 0, n_ff = 0;   // see Params
   int32_t* desc = nullptr;           // [n_tasks][kDescWords], fused priority order
   int32_t* targets = nullptr;        // [n_counters] arrivals per step
   // unfused launcher: the same tasks grouped by phase, phase ph being
@@ -277,6 +287,7 @@ struct SmemLayout {
   int scratch_bytes;
   int n_stages;       // ring stages of kStageBytes
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring, off_epi, off_ptrs;
+  int off_rcache;
   int part_cols;
   int total;          // bytes from the 1024-aligned base
   int dyn_bytes;      // dynamic shared memory to request (total + alignment slack)

@@ -230,6 +230,7 @@ struct Smem {
   uint8_t* epi;
   const void* const* ptrs;   // per-layer pointer table
   int32_t* fifo;
+  int32_t* rcache;           // the producer's copy of one layer's routing table
   uint32_t bars;  // shared-window address of barrier 0
   int NS;
   __device__ uint32_t bar(int i) const { return bars + 8u * (uint32_t)i; }
@@ -273,6 +274,7 @@ __device__ __forceinline__ Smem smem_view(const Params& p) {
   s.epi = base + p.off_epi;
   s.ptrs = reinterpret_cast<const void* const*>(base + p.off_ptrs);
   s.fifo = reinterpret_cast<int32_t*>(base + p.off_fifo);
+  s.rcache = reinterpret_cast<int32_t*>(base + p.off_rcache);
   s.bars = raw + pad + (uint32_t)p.off_bars;
   s.NS = p.n_stages;
   return s;
@@ -381,11 +383,11 @@ __device__ __forceinline__ const void* tmap(const Params& p, int idx) {
 
 // ============================================================== producer ==
 // The producer takes tasks of the step's list from the dispenser (an atomic
-// add on a counter that advances by n_tasks + n_ctas per step), posts each in
-// the CTA's task FIFO, and streams its tiles.  A taken index past the end
-// posts a stop entry.  The next task is taken only once the current task's
-// last stage is issued: taking it earlier holds it on this CTA while other
-// CTAs could already run it, which measured slower.
+// add on a counter that every launch starts at 0), posts each in the CTA's
+// task FIFO, and streams its tiles.  A taken index past the end
+// posts a stop entry.  The next task is taken as soon as the current one is
+// posted, so the dispenser's round trip overlaps the current task's stage
+// issue (one task of lookahead per CTA).
 __device__ __forceinline__ void prefetch_tmap(const void* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
@@ -427,7 +429,6 @@ __device__ __noinline__ void producer_loop(const Params& p) {
   const int lane = threadIdx.x & 31;
   const int NS = sm.NS;
   uint32_t slot = 0, phase = 0;   // ring position of the next stage
-  const uint32_t base = (pp.epoch - 1u) * (uint32_t)(pp.n_tasks + pp.n_ctas);
   const uint64_t pol = l2_evict_first();
   auto valid = [&](int t) { return t >= 0 && t < pp.n_tasks; };
   int t_next = 0;
@@ -435,11 +436,21 @@ __device__ __noinline__ void producer_loop(const Params& p) {
   auto take = [&]() {   // next task index and its descriptor (word `lane`)
     uint32_t raw = 0;
     if (lane == 0) raw = atomicAdd(pp.counters + pp.grab, 1u);
-    t_next = __shfl_sync(FULL, (int)(raw - base), 0);
+    t_next = __shfl_sync(FULL, (int)raw, 0);
     dw_next = valid(t_next) ? __ldg(pp.desc + (size_t)t_next * kDescWords + lane) : 0;
+  };
+  // an expert tile of an unused slot: the rest of its layer's tiles of that
+  // operation are unused too (slots fill in ascending order, tiles are
+  // slot-major); move the dispenser past them and take the next task
+  auto skip_unused = [&](int32_t dw) {
+    const int end = __shfl_sync(FULL, dw, D_C);
+    if (lane == 0) atomicMax(pp.counters + pp.grab, (uint32_t)end);
+    take();
   };
   int pw_done_ctr = -1;          // producer wait already seen satisfied (this step)
   uint32_t pw_done_tgt = 0;
+  int nu_layer = -1, n_used = 0;  // slots used in layer nu_layer (known after its top-k)
+  int rc_layer = -1;              // layer whose routing table sm.rcache holds
   auto ring_next = [&]() {
     if (++slot == (uint32_t)NS) {
       slot = 0;
@@ -461,6 +472,12 @@ __device__ __noinline__ void producer_loop(const Params& p) {
     }
     const int op = __shfl_sync(FULL, dw, D_OP);
     const int layer = __shfl_sync(FULL, dw, D_LAYER);
+    if ((op == OP_GATEUP || op == OP_DOWN) && layer == nu_layer &&
+        __shfl_sync(FULL, dw, D_A) >= n_used) {
+      skip_unused(dw);   // this FIFO entry stays free for the next task
+      --i;
+      continue;
+    }
     int nstage = __shfl_sync(FULL, dw, D_NSTAGE);
     const int map0 = __shfl_sync(FULL, dw, D_MAP0), map1 = __shfl_sync(FULL, dw, D_MAP1);
     if (lane == 0 && (nstage > 0 || op == OP_ATTN)) {
@@ -483,11 +500,32 @@ __device__ __noinline__ void producer_loop(const Params& p) {
         pw_done_ctr = ctr;
         pw_done_tgt = tgt;
       }
-      // every routing word of the slot in one round trip: lane R_EXPERT the
-      // expert, R_NTOK the token count, R_TOK/R_RANK/R_W + n token n's id,
-      // rank and weight (words past the count are read and then dropped)
+      // The layer's routing table is copied into shared memory once (its
+      // words are final once the top-k has signalled), so the layer's other
+      // expert tiles on this CTA resolve without a global round trip.
+      if (rc_layer != layer) {
+        const int32_t* rt = pp.route + (size_t)layer * pp.route_words;
+        for (int w0 = 0; w0 < pp.route_words; w0 += 32 * 16) {
+          int32_t v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int w = w0 + u * 32 + lane;
+            v[u] = w < pp.route_words ? __ldcg(rt + w) : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int w = w0 + u * 32 + lane;
+            if (w < pp.route_words) sm.rcache[w] = v[u];
+          }
+        }
+        __syncwarp();
+        rc_layer = layer;
+      }
+      // every routing word of the slot: lane R_EXPERT the expert, R_NTOK the
+      // token count, R_TOK/R_RANK/R_W + n token n's id, rank and weight
+      // (words past the count are read and then dropped)
       const int j = __shfl_sync(FULL, dw, D_A);
-      const int32_t* rt = pp.route + (size_t)layer * pp.route_words;
+      const int32_t* rt = sm.rcache;
       const int B = pp.B, K = pp.k, S = pp.S;
       int idx = -1;
       if (lane == R_EXPERT) idx = route_slot_expert(B, K) + j;
@@ -496,18 +534,22 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       else if (lane >= R_RANK && lane < R_RANK + 8)
         idx = route_slot_rank(B, K, S) + j * 8 + lane - R_RANK;
       else if (lane >= R_W && lane < R_W + 8) idx = route_slot_w(B, K, S) + j * 8 + lane - R_W;
-      const int32_t v = idx >= 0 ? __ldcg(rt + idx) : 0;
+      else if (lane == 3) idx = 0;   // slots in use
+      const int32_t v = idx >= 0 ? rt[idx] : 0;
       expert = __shfl_sync(FULL, v, R_EXPERT);
       ntok = __shfl_sync(FULL, v, R_NTOK);
-      if (expert >= pp.E || ntok < 0 || ntok > B) {
+      const int used = __shfl_sync(FULL, v, 3);
+      if (expert >= pp.E || ntok < 0 || ntok > B || used < 0 || used > S) {
         if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, expert, ntok, 1);
         set_abort();
         break;
       }
-      if (expert < 0) {
-        expert = -1;
-        ntok = 0;
-        nstage = 0;
+      nu_layer = layer;
+      n_used = used;
+      if (expert < 0) {   // an unused slot: its tiles are dropped (the top-k
+        skip_unused(dw);  // stood in for their signals)
+        --i;
+        continue;
       }
       if (lane >= R_TOK && lane < R_W + 8) rw = ((lane - R_TOK) & 7) < ntok ? v : 0;
     } else if (op == OP_ATTN) {
@@ -553,6 +595,9 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       if (p.trace) p.trace[(size_t)t * kTraceWords + T_CTA] = blockIdx.x + 1;
       mbar_arrive(sm.posted(e));
     }
+    // take the next task now: its dispenser round trip overlaps this task's
+    // stage issue
+    take();
 
     // ---- stream the task's tiles
     if (op == OP_ATTN) {
@@ -647,7 +692,6 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       }
       if (fail) break;
     }
-    take();
     if (lane == 0) {
       stamp(p, t, T_P_ISSUED);
       trace_put(p, t, T_P_WAITCYC, pwait);
@@ -660,6 +704,15 @@ __device__ __noinline__ void producer_loop(const Params& p) {
   for (int s2 = 0; s2 < NS; ++s2) {
     const uint32_t st2 = (uint32_t)s2 < slot ? phase : (phase ^ 1u);
     drain_bar(p, sm.full(s2), st2);
+  }
+  // every producer has taken its last task once all have counted out: the
+  // last one starts the next launch's dispenser at 0
+  if (lane == 0) {
+    const uint32_t old = atomicAdd(pp.counters + p.exit_ctr, 1u);
+    if (old + 1u == (uint32_t)pp.n_ctas) {
+      atomicExch(pp.counters + pp.grab, 0u);
+      atomicExch(pp.counters + p.exit_ctr, 0u);
+    }
   }
 }
 
@@ -768,8 +821,6 @@ __device__ __noinline__ void loader_loop(const Params& p) {
           mbar_expect_tx(fb, (uint32_t)lp.ofrag_bytes);
           bulk_g2s(dst, lp.ofrag + ((size_t)layer * lp.Hkv + g) * lp.ofrag_bytes,
                    (uint32_t)lp.ofrag_bytes, fb);
-        } else if (ent[32 + R_EXPERT] < 0) {   // OP_DOWN of an empty slot: nothing to copy
-          mbar_arrive(fb);
         } else {  // OP_DOWN
           const int j = a;
           mbar_expect_tx(fb, (uint32_t)lp.afrag_bytes);
@@ -1841,6 +1892,16 @@ __device__ __noinline__ void topk_task(const Params& p, int l) {
     }
   }
   if (ct == 0) rt[0] = n_used;
+  // The producers drop the tiles of unused slots; stand in for the signals
+  // those tiles would have sent: each down-tile row counter gets one per
+  // unused slot, each unused slot's counter its n_ff gate/up tiles (so every
+  // counter still gets its per-step arrival count).
+  if (n_used < S) {
+    for (int r = ct; r < NR; r += 256)
+      atomicAdd(p.counters + p.dt_ctr0 + l * NR + r, (uint32_t)(S - n_used));
+    for (int j = n_used + ct; j < S; j += 256)
+      atomicAdd(p.counters + p.slot_ctr0 + l * S + j, (uint32_t)p.n_ff);
+  }
   // one thread per (token, rank): its position in the slot's token list
   if (ct < B * K) {
     const int bb = ct / K, j = ct % K;
@@ -1937,9 +1998,6 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
     const uint8_t* actB = sm.actB + (size_t)bufB * p.actB_bytes;
 
     if (gemv) {
-      // an empty expert slot: nothing streamed or computed; the epilogue warp
-      // completes it without a partials buffer
-      if ((op == OP_GATEUP || op == OP_DOWN) && ent[32 + R_EXPERT] < 0) continue;
       const int pb = (int)(ngemv & 1u);
       const uint32_t pe_par = ((ngemv >> 1) & 1u) ^ 1u;
       float* pw = part0 + (pb * kConsumerWarps + cw) * 16 * PC;
@@ -1969,28 +2027,9 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
     switch (op) {
       case OP_RN:
         stage_ctr = rn_task(p, ent, stage_ctr);
-        if (ent[D_FLAGS] & F_TOPK) {
-          // The tile is complete: its own signal goes out now (the FIFO entry
-          // is released, so its words are copied first).  The tile whose
-          // arrival completes the level has acquired every tile's router
-          // shares and sum-of-squares partials and runs the layer's top-k.
-          const int lyr = layer, x0 = ent[D_X0], x1 = ent[D_X1], x2 = ent[D_X2];
-          cbar();
-          int last = 0;
-          if (ct == 0) {
-            stamp(p, t, T_C_END);
-            cstamp(p, t, T_K5);
-            mbar_arrive(sm.done(e));
-            const uint32_t old = atom_add_acq_rel(p.counters + x0, 1u);
-            last = old + 1u == p.epoch * (uint32_t)x1;
-          }
-          if (cbar_or(last)) {
-            topk_task(p, lyr);
-            cbar();
-            if (ct == 0) red_release_add(p.counters + x2, 1u);
-          }
-          continue;
-        }
+        break;
+      case OP_TOPK:
+        topk_task(p, layer);
         break;
       default:  // OP_ATTN
         stage_ctr = attn_task<HD>(p, ent, actB, stage_ctr);
@@ -2045,18 +2084,6 @@ __device__ __noinline__ void epilogue_loop(const Params& p) {
       if (act == ACT_B) ++nloadB;
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.fempty(e));
-      continue;
-    }
-    if ((op == OP_GATEUP || op == OP_DOWN) && ent[32 + R_EXPERT] < 0) {
-      // an empty expert slot (the consumers skipped it): complete the task
-      __syncwarp();
-      if (lane == 0) {
-        if (act == ACT_B) mbar_arrive(sm.aemptyB(nloadB & 1));
-        mbar_arrive(sm.done(e));
-        mbar_arrive(sm.fempty(e));
-      }
-      __syncwarp();
-      if (act == ACT_B) ++nloadB;
       continue;
     }
     const int pb = (int)(ngemv & 1u);

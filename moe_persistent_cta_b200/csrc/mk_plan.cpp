@@ -18,10 +18,10 @@
 // "Three sources of speedup", item 2).
 //
 // Priority order inside a layer: the norm tiles (which also produce the
-// router logits, share by share, and the last of which runs the top-k); QKV;
-// attention chunks (their cached K/V stream before the new query exists);
-// expert gate/up (the MoE branch is the longer one); then the attention tail
-// and the expert down projections.
+// router logits, share by share); QKV and top-k; attention chunks (their
+// cached K/V stream before the new query exists); expert gate/up (the MoE
+// branch is the longer one); then the attention tail and the expert down
+// projections.
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
@@ -110,7 +110,9 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
                            128);
   const int budget = 232448 - 2048;   // max per block, less alignment slack and static smem
   const int ptrs = round_up(ptr_table_words(s.L) * 8, 128);
-  int rest1 = bars + fifo + epi + ptrs + o->scratch_bytes + o->actA_stride + 2 * o->actB_bytes;
+  const int rcache = round_up(route_words(B, s.k, std::min(s.E, B * s.k)) * 4, 128);
+  int rest1 = bars + fifo + epi + ptrs + rcache + o->scratch_bytes + o->actA_stride +
+              2 * o->actB_bytes;
   int rest2 = rest1 + o->actA_stride;
   int nA = ((budget - rest2) / kStageBytes >= 8) ? 2 : 1;
   int rest = nA == 2 ? rest2 : rest1;
@@ -126,7 +128,8 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->off_actB = o->off_actA + nA * o->actA_stride;
   o->off_epi = o->off_actB + 2 * o->actB_bytes;
   o->off_ptrs = o->off_epi + epi;
-  o->total = o->off_ptrs + ptrs;
+  o->off_rcache = o->off_ptrs + ptrs;
+  o->total = o->off_rcache + rcache;
   o->dyn_bytes = o->total + 1024;
   return MK_OK;
 }
@@ -140,12 +143,11 @@ struct Task {
 
 struct Layout {
   int L, B, S, Hkv, NR;
-  int norm0, narr0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmarr, lmdone, total;
+  int norm0, qkv0, rtr0, attp0, atto0, slot0, dt0, lmarr, lmdone, total;
   void build(int L_, int B_, int S_, int Hkv_, int NR_) {
     L = L_; B = B_; S = S_; Hkv = Hkv_; NR = NR_;
     int c = 0;
     norm0 = c; c += L + 1;
-    narr0 = c; c += L;
     qkv0 = c; c += L * Hkv;
     rtr0 = c; c += L;
     attp0 = c; c += L * B * Hkv;
@@ -157,7 +159,6 @@ struct Layout {
     total = c;
   }
   int norm(int l) const { return norm0 + l; }
-  int narr(int l) const { return narr0 + l; }
   int qkv(int l, int g) const { return qkv0 + l * Hkv + g; }
   int rtr(int l) const { return rtr0 + l; }
   int attp(int l, int b, int g) const { return attp0 + (l * B + b) * Hkv + g; }
@@ -256,9 +257,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   // residual add + RMSNorm tiles producing level l; a tile of a level that
   // feeds a layer also computes its 64 columns' share of that layer's router
   // logits (W_r[:, tile] . gamma x), its router columns streamed through the
-  // ring like GEMV weights: one stage per 128 experts.  The tile whose arrival
-  // completes the level then sums the shares and runs the layer's top-k,
-  // softmax and slot compaction, and signals the routing counter.
+  // ring like GEMV weights: one stage per 128 experts
   auto emit_norm = [&](int l) {
     for (int r = 0; r < NR; ++r) {
       Task t = make_task(OP_RN, l, l * PH + 0);
@@ -266,7 +265,6 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
       if (l < L) {
         t.w[D_NSTAGE] = (E + kRouterRowsPerStage - 1) / kRouterRowsPerStage;
         t.w[D_MAP0] = map_of(l, kMapRouter);
-        fuse(t, F_TOPK, lay.narr(l), NR, lay.rtr(l));
       }
       if (l > 0) add_wait(t, lay.dt(l - 1, r), Hkv + S);
       add_signal(t, lay.norm(l));
@@ -277,7 +275,14 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   emit_norm(0);
   for (int l = 0; l < L; ++l) {
     if (l > 0) emit_norm(l);
-    targets[lay.rtr(l)] += 1;   // one top-k per layer, by the last norm tile
+    // -- top-k over the router logits summed from the norm tiles' shares
+    {
+      Task t = make_task(OP_TOPK, l, l * PH + 2);
+      add_wait(t, lay.norm(l), NR);
+      add_signal(t, lay.rtr(l));
+      tasks.push_back(t);
+    }
+    targets[lay.rtr(l)] += 1;   // one top-k per layer
     // -- QKV tiles (grouped by KV group so attention of a group starts early)
     for (int g = 0; g < Hkv; ++g) {
       auto emit_rows = [&](int row_begin, int rows) {
@@ -427,6 +432,22 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
     if (x.w[D_LAYER] != y.w[D_LAYER]) return x.w[D_LAYER] < y.w[D_LAYER];
     return kRank[x.w[D_OP]] < kRank[y.w[D_OP]];
   });
+  // expert tiles: D_C = the list index one past the layer's last tile of the
+  // same operation.  Slots are filled in ascending order at run time and the
+  // tiles are slot-major, so once a producer meets a tile of an unused slot
+  // every later tile up to that index is unused too and the dispenser jumps
+  // there.
+  for (size_t i = 0; i < tasks.size();) {
+    const int op = tasks[i].w[D_OP];
+    size_t j = i + 1;
+    if (op == OP_GATEUP || op == OP_DOWN) {
+      while (j < tasks.size() && tasks[j].w[D_OP] == op &&
+             tasks[j].w[D_LAYER] == tasks[i].w[D_LAYER])
+        ++j;
+      for (size_t q = i; q < j; ++q) tasks[q].w[D_C] = (int)j;
+    }
+    i = j;
+  }
   // A-slot double buffering where two buffers fit in shared memory
   SmemLayout sl;
   int slrc = smem_layout(s, B, max_chunks, &sl);
@@ -435,11 +456,12 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   const int n_tasks = (int)tasks.size();
   const int n_phases = L * PH + 2;
   // task dispensers: one for the fused list, one per phase list
+  // (each launch starts them at 0 and its last producer out zeroes them)
   const int grab = lay.total;
   const int grab_phase0 = lay.total + 1;
-  const int n_counters = lay.total + 1 + n_phases;
+  const int exit_ctr = lay.total + 1 + n_phases;
+  const int n_counters = lay.total + 2 + n_phases;
   targets.resize(n_counters, 0);
-  targets[grab] = n_tasks + n_ctas;
 
   out->release();
   out->n_ctas = n_ctas;
@@ -452,6 +474,10 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   out->n_phases = n_phases;
   out->grab = grab;
   out->grab_phase0 = grab_phase0;
+  out->exit_ctr = exit_ctr;
+  out->slot_ctr0 = lay.slot0;
+  out->dt_ctr0 = lay.dt0;
+  out->n_ff = n_ff;
   out->desc = (int32_t*)std::malloc((size_t)n_tasks * kDescWords * sizeof(int32_t));
   out->targets = (int32_t*)std::calloc((size_t)n_counters, sizeof(int32_t));
   out->phase_desc = with_phases
@@ -469,15 +495,8 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   for (const auto& t : tasks) per_phase[t.w[D_PHASE]]++;
   for (int ph = 0; ph < n_phases; ++ph) {
     out->phase_off[ph + 1] = out->phase_off[ph] + per_phase[ph];
-    targets[grab_phase0 + ph] = per_phase[ph] + n_ctas;
   }
-  if (with_phases) {
-    std::vector<int> fill(out->phase_off, out->phase_off + n_phases);
-    for (const auto& t : tasks) {
-      const int pos = fill[t.w[D_PHASE]]++;
-      std::memcpy(out->phase_desc + (size_t)pos * kDescWords, t.w, sizeof(int32_t) * kDescWords);
-    }
-  }
+  if (with_phases) group_by_phase(*out, out->phase_desc);
   std::memcpy(out->targets, targets.data(), sizeof(int32_t) * n_counters);
   (void)sl;
   return MK_OK;
@@ -485,12 +504,18 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
 
 // The unfused launcher's lists: the plan's tasks grouped by phase (phase ph
 // at [phase_off[ph], phase_off[ph + 1]) of `out`), each group in list order.
+// An expert phase holds one layer's tiles of one operation, so their jump
+// index (D_C) becomes the phase's own length.
 void group_by_phase(const Plan& plan, int32_t* out) {
   std::vector<int> fill(plan.phase_off, plan.phase_off + plan.n_phases);
   for (int i = 0; i < plan.n_tasks; ++i) {
     const int32_t* w = plan.desc + (size_t)i * kDescWords;
-    const int pos = fill[w[D_PHASE]]++;
-    std::memcpy(out + (size_t)pos * kDescWords, w, sizeof(int32_t) * kDescWords);
+    const int ph = w[D_PHASE];
+    const int pos = fill[ph]++;
+    int32_t* o = out + (size_t)pos * kDescWords;
+    std::memcpy(o, w, sizeof(int32_t) * kDescWords);
+    if (w[D_OP] == OP_GATEUP || w[D_OP] == OP_DOWN)
+      o[D_C] = plan.phase_off[ph + 1] - plan.phase_off[ph];
   }
 }
 

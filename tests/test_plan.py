@@ -26,9 +26,8 @@ ACT_NONE, ACT_A, ACT_B = 0, 1, 2
 
 D_X0, D_X1, D_X2 = 29, 30, 31
 F_COMBINE = 128   # last-arriver work: the attention merge of a (token, KV head)
-F_TOPK = 256      # last-arriver work: the top-k of the layer a norm level feeds
 F_ARGMAX = 512    # last-arriver work: a greedy step's tokens after the LM head
-FUSED = F_COMBINE | F_TOPK | F_ARGMAX
+FUSED = F_COMBINE | F_ARGMAX
 
 
 def signal_sets(desc, targets):
@@ -72,7 +71,7 @@ def check_order_and_targets(desc, targets, n_ctas, grab):
             assert last_sig[c] < i, f"task {i} waits on counter {c} sent later (task {last_sig[c]})"
     for c, k in count.items():
         assert targets[c] == k
-    assert targets[grab] == len(desc) + n_ctas
+    assert targets[grab] == 0      # the dispenser restarts at 0 every launch
     # greedy dynamic execution: each CTA takes the next task when it has
     # finished its previous one; a task finishes when its waits are met
     remaining = {c: len(v) for c, v in senders.items()}
@@ -115,21 +114,19 @@ def test_30b_b1_plan_structure():
     L, d = shape["n_layers"], shape["d_model"]
     qkv_rows = (shape["n_q_heads"] + 2 * shape["n_kv_heads"]) * shape["head_dim"]
     assert ops[OP_QKV] == L * qkv_rows // 16
-    # the norm tiles produce the router logits: no router tiles, no top-k
-    # tasks; the norm tile whose arrival completes a level runs the top-k of
-    # the layer it feeds and signals the counter the layer's expert tiles wait on
+    # the norm tiles produce the router logits: no router tiles, and each
+    # layer's top-k waits for all of the layer's norm tiles and signals the
+    # counter the layer's expert tiles wait on
     assert ops[OP_ROUTER] == 0
     assert ops[OP_RN] == (L + 1) * d // 64
-    assert ops[OP_TOPK] == 0
+    assert ops[OP_TOPK] == L
+    tk = desc[desc[:, D_OP] == OP_TOPK]
+    assert np.all(tk[:, D_NWAIT] == 1) and np.all(tk[:, D_W0N] == d // 64)
     rn = desc[desc[:, D_OP] == OP_RN]
-    feeds = rn[rn[:, D_LAYER] < L]
-    assert np.all(feeds[:, D_FLAGS] & F_TOPK) and np.all(feeds[:, D_X1] == d // 64)
-    assert not np.any(rn[rn[:, D_LAYER] == L][:, D_FLAGS] & F_TOPK)
     gu = desc[desc[:, D_OP] == OP_GATEUP]
     for l in (0, 5, L - 1):
-        join = set(feeds[feeds[:, D_LAYER] == l][:, D_X2].tolist())
-        assert join == set(gu[gu[:, D_LAYER] == l][:, D_PW].tolist())
-        assert len(set(feeds[feeds[:, D_LAYER] == l][:, D_X0].tolist())) == 1
+        assert set(tk[tk[:, D_LAYER] == l][:, D_S0].tolist()) == \
+            set(gu[gu[:, D_LAYER] == l][:, D_PW].tolist())
     # a norm tile of a level that feeds a layer streams its router columns:
     # one ring stage per 128 experts; the final norm streams nothing
     E = shape["n_experts"]
@@ -217,3 +214,42 @@ def test_invalid_shapes_rejected():
         engine.plan_schedule(configs.TINY, 148, [-1])
     with pytest.raises(mk.MKError):
         engine.plan_schedule(dict(configs.TINY, n_experts=10, top_k=2), 148, [10])   # E % 4
+
+
+@pytest.mark.parametrize("lens", [[8192], [100, 2000, 5, 64, 9000, 300, 40, 7]])
+def test_unused_slot_tiles_can_be_skipped(lens):
+    """Expert tiles of unused slots are dropped by the producers, which jump
+    the dispenser to D_C: one past the layer's last tile of the same
+    operation.  That is only sound if those tiles are contiguous and
+    slot-major (an unused slot is never followed by a used one), and if the
+    counters their signals would have reached are the ones the top-k stands
+    in for: the slot counter (n_ff gate/up tiles) and the down-tile row
+    counters (one signal per slot)."""
+    shape = configs.MOE30B
+    meta, desc, targets = engine.plan_schedule(shape, 148, lens)
+    S, n_ff, NR = meta[2], shape["d_ff"] // 16, shape["d_model"] // 64
+    for op, per_slot in ((OP_GATEUP, n_ff), (OP_DOWN, NR)):
+        idx = np.where(desc[:, D_OP] == op)[0]
+        for l in (0, 17, shape["n_layers"] - 1):
+            run = idx[desc[idx, D_LAYER] == l]
+            assert len(run) == S * per_slot
+            assert np.all(np.diff(run) == 1)                  # contiguous
+            assert np.all(desc[run, D_C] == run[-1] + 1)      # jump past the run
+            assert np.all(np.diff(desc[run, D_A]) >= 0)       # slot-major
+    gu = desc[desc[:, D_OP] == OP_GATEUP]
+    dn = desc[desc[:, D_OP] == OP_DOWN]
+    # each slot counter is signalled by exactly its n_ff gate/up tiles and
+    # waited on (for n_ff) by exactly its down tiles
+    for l in (0, 30):
+        for j in (0, S - 1):
+            g = gu[(gu[:, D_LAYER] == l) & (gu[:, D_A] == j)]
+            d = dn[(dn[:, D_LAYER] == l) & (dn[:, D_A] == j)]
+            c = set(g[:, D_S0].tolist())
+            assert len(c) == 1 and targets[c.pop()] == n_ff
+            assert set(d[:, D_W0].tolist()) == set(g[:, D_S0].tolist())
+            assert np.all(d[:, D_W0N] == n_ff)
+        # each down-tile row counter gets one signal per slot plus the O-proj groups
+        rows = dn[dn[:, D_LAYER] == l]
+        for r in (0, NR - 1):
+            c = set(rows[rows[:, D_B] == r][:, D_S0].tolist())
+            assert len(c) == 1 and targets[c.pop()] == S + shape["n_kv_heads"]
