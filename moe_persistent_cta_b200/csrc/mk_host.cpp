@@ -54,7 +54,7 @@ struct mk_ctx {
   int counters_cap = 0;
   DevBuf desc, phase_desc;
   bool phases_uploaded = false;
-  DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, rpart, route, expert_a, afrag,
+  DevBuf x, actA, qkv, cs, attn_part, attn_o, ofrag, o_part, rlogits, racc, ssacc, route, expert_a, afrag,
       moe_part, amax, trace;
   DevBuf selftest;   // one descriptor + two counters for mk_selftest_timeout
   bool tracing = false;
@@ -179,7 +179,7 @@ void mk_destroy(mk_ctx* c) {
   cudaFree(c->d_counters);
   for (DevBuf* b : {&c->desc, &c->phase_desc, &c->x, &c->actA,
                     &c->qkv, &c->cs, &c->attn_part, &c->attn_o, &c->ofrag, &c->o_part,
-                    &c->rlogits, &c->rpart, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
+                    &c->rlogits, &c->racc, &c->ssacc, &c->route, &c->expert_a, &c->afrag, &c->moe_part,
                     &c->amax, &c->trace, &c->selftest})
     release(*b);
   c->plan.release();
@@ -384,7 +384,8 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   ENSURE(ofrag, (size_t)L * s.Hkv * ofrag_bytes);
   ENSURE(o_part, (size_t)L * s.Hkv * B * d * 4);
   ENSURE(rlogits, (size_t)L * B * s.E * 4);
-  ENSURE(rpart, (size_t)L * NR * B * s.E * 4);
+  ENSURE(racc, (size_t)2 * L * B * s.E * 8);
+  ENSURE(ssacc, (size_t)2 * L * B * 8);
   ENSURE(route, (size_t)L * rwords * 4);
   ENSURE(expert_a, (size_t)L * S * B * s.F * 4);
   ENSURE(afrag, (size_t)L * S * afrag_bytes);
@@ -404,6 +405,8 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
     return fail(MK_ERR_CUDA);
   if (cudaMemset(c->route.ptr, 0, c->route.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
   if (cudaMemset(c->amax.ptr, 0, c->amax.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
+  if (cudaMemset(c->racc.ptr, 0, c->racc.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
+  if (cudaMemset(c->ssacc.ptr, 0, c->ssacc.bytes) != cudaSuccess) return fail(MK_ERR_CUDA);
   if (cudaMemcpy(c->desc.ptr, plan.desc, (size_t)plan.n_tasks * mk::kDescWords * 4,
                  cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(MK_ERR_CUDA);
@@ -445,7 +448,8 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.ofrag = static_cast<uint8_t*>(c->ofrag.ptr);
   p.o_part = static_cast<float*>(c->o_part.ptr);
   p.rlogits = static_cast<float*>(c->rlogits.ptr);
-  p.rpart = static_cast<float*>(c->rpart.ptr);
+  p.racc = static_cast<unsigned long long*>(c->racc.ptr);
+  p.ssacc = static_cast<unsigned long long*>(c->ssacc.ptr);
   p.route = static_cast<int32_t*>(c->route.ptr);
   p.expert_a = static_cast<float*>(c->expert_a.ptr);
   p.afrag = static_cast<uint8_t*>(c->afrag.ptr);
@@ -594,6 +598,8 @@ mk_status mk_check(mk_ctx* c, int32_t* device_status, int32_t* detail) {
     if (c->d_counters)
       MK_CUDA(cudaMemset(c->d_counters, 0, sizeof(uint32_t) * c->counters_cap));
     if (c->amax.ptr) MK_CUDA(cudaMemset(c->amax.ptr, 0, c->amax.bytes));
+    if (c->racc.ptr) MK_CUDA(cudaMemset(c->racc.ptr, 0, c->racc.bytes));
+    if (c->ssacc.ptr) MK_CUDA(cudaMemset(c->ssacc.ptr, 0, c->ssacc.bytes));
     c->epoch = 0;
     return st[mk::ST_CODE] != 0 ? (mk_status)st[mk::ST_CODE] : MK_ERR_DEVICE;
   }
@@ -690,6 +696,8 @@ size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) 
   const size_t L = b.L, B = b.B, d = b.d;
   uint8_t* counters = take(sizeof(uint32_t) * (size_t)n_counters);
   uint8_t* route = take((size_t)L * b.route_words * 4);
+  uint8_t* racc = take((size_t)2 * L * B * b.E * 8);
+  uint8_t* ssacc = take((size_t)2 * L * B * 8);
   uint8_t* x = take((L + 1) * B * d * 4);
   uint8_t* actA = take((L + 1) * (size_t)b.actA_bytes);
   uint8_t* qkv = take(L * B * b.qkvR * 4);
@@ -699,7 +707,6 @@ size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) 
   uint8_t* ofrag = take(L * b.Hkv * (size_t)b.ofrag_bytes);
   uint8_t* o_part = take(L * b.Hkv * B * d * 4);
   uint8_t* rlogits = take(L * B * b.E * 4);
-  uint8_t* rpart = take(L * b.NR * B * b.E * 4);
   uint8_t* expert_a = take(L * b.S * B * b.F * 4);
   uint8_t* afrag = take(L * b.S * (size_t)b.afrag_bytes);
   uint8_t* moe_part = take(L * b.k * B * d * 4);
@@ -715,7 +722,8 @@ size_t carve_scratch(const Params& b, int n_counters, uint8_t* base, Params* p) 
     p->ofrag = ofrag;
     p->o_part = reinterpret_cast<float*>(o_part);
     p->rlogits = reinterpret_cast<float*>(rlogits);
-    p->rpart = reinterpret_cast<float*>(rpart);
+    p->racc = reinterpret_cast<unsigned long long*>(racc);
+    p->ssacc = reinterpret_cast<unsigned long long*>(ssacc);
     p->expert_a = reinterpret_cast<float*>(expert_a);
     p->afrag = afrag;
     p->moe_part = reinterpret_cast<float*>(moe_part);
@@ -742,7 +750,8 @@ mk_status launch_step_in(mk_ctx* c, const int32_t* tokens, const int32_t* positi
   Params p = c->base;
   carve_scratch(c->base, c->plan.n_counters, static_cast<uint8_t*>(scratch), &p);
   const size_t zero_bytes = reinterpret_cast<uint8_t*>(p.x) - static_cast<uint8_t*>(scratch);
-  MK_CUDA(cudaMemsetAsync(scratch, 0, zero_bytes, st));   // counters + routing words
+  // counters, routing words and the router accumulators start at zero
+  MK_CUDA(cudaMemsetAsync(scratch, 0, zero_bytes, st));
   c->last_stream = st;
   c->launched = true;
   p.tokens = tokens;

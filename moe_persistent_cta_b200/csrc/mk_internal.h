@@ -44,7 +44,13 @@ constexpr int kActPad = 8;
 constexpr int kRnStage = 4096;       // floats of residual partials staged per round
 constexpr int kRouterRowsPerStage = 128;   // router weight rows (x 64 columns) per ring stage
 constexpr int kMaxAttnOut = 512;    // G x hd floats of one (token, KV head) output (G <= 4, hd <= 128)
-constexpr int kTopkLogitsOff = 2048; // top-k scratch: selection state, then logits [B][E]
+// Batch sizes up to which each producer computes a layer's routing table
+// itself from the norm tiles' accumulators (one warp, a few microseconds),
+// instead of waiting for the layer's top-k task and copying its table.
+constexpr int kLocalRouteMaxB = 4;
+// words of the producer's routing scratch after its copy of the routing
+// table: selections and weights [8][8] each, and an 8-word expert mask
+constexpr int kRouteTmpWords = 64 + 64 + 8;
 // Per-layer pointer table in shared memory: norm weights of levels 0..L (the
 // final norm last), then router bias, K pool and V pool of layers 0..L-1.  A
 // task reads its layer's pointers from there, so its first global loads need
@@ -207,7 +213,9 @@ struct Params {
   uint8_t* ofrag;    // [L][Hkv][ofrag_bytes]
   float* o_part;     // [L][Hkv][B][d]
   float* rlogits;    // [L][B][E]
-  float* rpart;      // [L][NR][B][E] router logits per 64-column tile (before 1/rms)
+  unsigned long long* racc;    // [2][L][B][E] router logit shares, fixed point (2^-32),
+                               // by step parity (epoch & 1)
+  unsigned long long* ssacc;   // [2][L][B] sums of squares of the layer's input, fixed point
   int32_t* route;    // [L][route_words]
   float* expert_a;   // [L][S][B][F]
   uint8_t* afrag;    // [L][S][afrag_bytes]

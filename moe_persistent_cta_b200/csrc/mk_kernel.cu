@@ -131,6 +131,20 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* a, uint32_t v) {
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// The router's logit shares and the sums of squares are accumulated across
+// the norm tiles as 64-bit fixed-point integers in units of 2^-32: integer
+// addition is associative, so a sum does not depend on the order in which
+// the tiles arrive (the step stays bit-reproducible), and one load of the
+// accumulator replaces a load per tile.
+__device__ __forceinline__ unsigned long long to_fixed(float x) {
+  return (unsigned long long)__float2ll_rn(x * 4294967296.0f);
+}
+__device__ __forceinline__ float from_fixed(unsigned long long v) {
+  return (float)((double)(long long)v * 2.3283064365386963e-10);
+}
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -381,6 +395,136 @@ __device__ __forceinline__ const void* tmap(const Params& p, int idx) {
   return static_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
 }
 
+// ================================================================ routing ==
+// Order-preserving key of a float: a larger float gives a larger unsigned key.
+__device__ __forceinline__ uint32_t ordered_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// One warp: token b's router logits in layer l from the fixed-point
+// accumulators of step parity par, logit_e = share_e * rstd + bias_e with
+// rstd = 1/sqrt(sum of squares / d + eps); its top-k (logit descending,
+// expert id ascending on ties) into sel[0..k) and the softmax over the k
+// selected logits into w[0..k) (shared memory).  logits (may be null)
+// receives the token's E logits.  Lane-parallel over experts (E <= 256).
+__device__ __noinline__ void token_route(const Params& p, const float* bias, int l, uint32_t par,
+                                         int b, int32_t* sel, float* w, float* logits) {
+  const int lane = threadIdx.x & 31;
+  const int E = p.E, K = p.k;
+  const size_t lb = (size_t)par * p.L + l;
+  const float ss = from_fixed(__ldcg(p.ssacc + lb * p.B + b));
+  const float rstd = frsqrt(ss / (float)p.d + p.eps);
+  const unsigned long long* acc = p.racc + (lb * p.B + b) * E;
+  uint32_t key[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int e = lane + 32 * t;
+    uint32_t k = 0u;   // 0: taken or absent (no finite logit has key 0)
+    if (e < E) {
+      const float v = from_fixed(__ldcg(acc + e)) * rstd + (bias ? __ldg(bias + e) : 0.f);
+      if (logits) logits[e] = v;
+      k = ordered_key(v);
+    }
+    key[t] = k;
+  }
+#pragma unroll 1
+  for (int j = 0; j < K; ++j) {
+    uint32_t bk = 0u;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (key[t] > bk) {   // ascending e within a lane: the first max has the smallest e
+        bk = key[t];
+        bi = lane + 32 * t;
+      }
+    }
+    const uint32_t mk = __reduce_max_sync(FULL, bk);
+    const int wi = __reduce_min_sync(FULL, bk == mk ? bi : 0x7fffffff);
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (lane + 32 * t == wi) key[t] = 0u;
+    if (lane == 0) {
+      sel[j] = wi;
+      w[j] = key_value(mk);
+    }
+  }
+  __syncwarp();
+  // softmax over the selected logits: lane j < K takes rank j
+  const float v0 = w[0];
+  float x = lane < K ? fexp(w[lane & 7] - v0) : 0.f;
+  float sum = x;
+  for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+  __syncwarp();
+  if (lane < K) w[lane] = x * frcp(sum);
+  __syncwarp();
+}
+
+// One warp: the layer's routing words (see route_*) from every token's
+// selection sel[b * 8 + j] and weight w[b * 8 + j] (shared memory): the
+// union of selected experts in ascending id becomes slots 0 .. n_used - 1,
+// each with its tokens in ascending order, their ranks and weights; slots
+// past n_used hold expert -1.  rt may be shared or global memory; mask is
+// 8 words of shared scratch.  Returns n_used.
+__device__ __noinline__ int compact_routes(const Params& p, const int32_t* sel, const float* w,
+                                           uint32_t* mask, int32_t* rt) {
+  const int lane = threadIdx.x & 31;
+  const int B = p.B, K = p.k, S = p.S, BK = B * K;
+  if (lane < 8) mask[lane] = 0u;
+  __syncwarp();
+  for (int q = lane; q < BK; q += 32) {
+    const int e = sel[(q / K) * 8 + q % K];
+    atomicOr(&mask[e >> 5], 1u << (e & 31));
+  }
+  __syncwarp();
+  uint32_t m[8];
+  int n_used = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    m[i] = mask[i];
+    n_used += __popc(m[i]);
+  }
+  if (lane == 0) rt[0] = n_used;
+  for (int s = n_used + lane; s < S; s += 32) {
+    rt[route_slot_expert(B, K) + s] = -1;
+    rt[route_slot_ntok(B, K, S) + s] = 0;
+  }
+  for (int q = lane; q < BK; q += 32) {
+    const int b = q / K, j = q - b * K;
+    const int e = sel[b * 8 + j];
+    const float wt = w[b * 8 + j];
+    rt[route_topk_idx(B, K) + q] = e;
+    reinterpret_cast<float*>(rt)[route_topk_w(B, K) + q] = wt;
+    // slot of e = the number of used experts below it
+    int s = __popc(m[e >> 5] & ((1u << (e & 31)) - 1u));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += (i < (e >> 5)) ? __popc(m[i]) : 0;
+    // position among the slot's tokens: earlier tokens that selected e
+    int pos = 0;
+#pragma unroll 1
+    for (int b2 = 0; b2 < b; ++b2)
+#pragma unroll 1
+      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
+    rt[route_slot_tok(B, K, S) + s * 8 + pos] = b;
+    rt[route_slot_rank(B, K, S) + s * 8 + pos] = j;
+    reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s * 8 + pos] = wt;
+    if (pos == 0) {
+      int cnt = 0;
+#pragma unroll 1
+      for (int b2 = b; b2 < B; ++b2)
+#pragma unroll 1
+        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
+      rt[route_slot_expert(B, K) + s] = e;
+      rt[route_slot_ntok(B, K, S) + s] = cnt;
+    }
+  }
+  __syncwarp();
+  return n_used;
+}
+
 // ============================================================== producer ==
 // The producer takes tasks of the step's list from the dispenser (an atomic
 // add on a counter that every launch starts at 0), posts each in the CTA's
@@ -500,10 +644,23 @@ __device__ __noinline__ void producer_loop(const Params& p) {
         pw_done_ctr = ctr;
         pw_done_tgt = tgt;
       }
-      // The layer's routing table is copied into shared memory once (its
-      // words are final once the top-k has signalled), so the layer's other
-      // expert tiles on this CTA resolve without a global round trip.
-      if (rc_layer != layer) {
+      // The layer's routing table is set up in shared memory once, so the
+      // layer's other expert tiles on this CTA resolve without a global round
+      // trip: up to kLocalRouteMaxB tokens the producer computes it from the
+      // norm tiles' accumulators (final once the norm tiles have signalled,
+      // which is what this task's producer wait covered), else it copies the
+      // top-k task's table (final once the top-k has signalled).
+      __syncwarp();   // the wait's acquire (lane 0) orders every lane's loads
+      if (rc_layer != layer && pp.B <= kLocalRouteMaxB) {
+        int32_t* tsel = sm.rcache + pp.route_words;
+        float* tw = reinterpret_cast<float*>(tsel + 64);
+        uint32_t* tmask = reinterpret_cast<uint32_t*>(tw + 64);
+        const float* bias = router_b(p, sm, layer);
+        for (int b = 0; b < pp.B; ++b)
+          token_route(p, bias, layer, pp.epoch & 1u, b, tsel + b * 8, tw + b * 8, nullptr);
+        compact_routes(p, tsel, tw, tmask, sm.rcache);
+        rc_layer = layer;
+      } else if (rc_layer != layer) {
         const int32_t* rt = pp.route + (size_t)layer * pp.route_words;
         for (int w0 = 0; w0 < pp.route_words; w0 += 32 * 16) {
           int32_t v[16];
@@ -1103,12 +1260,6 @@ struct EpiParams {
         PC(in_reg(p.part_cols)) {}
 };
 
-// Order-preserving key of a float: a larger float gives a larger unsigned key.
-__device__ __forceinline__ uint32_t ordered_key(float v) {
-  const uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // LM-head tile epilogue: the logits of the tile's rows for every token, and in
 // a greedy step each token's best logit of the tile with its lowest row,
 // folded into amax[n] as the 64-bit key (ordered logit << 32 | ~row), whose
@@ -1576,14 +1727,13 @@ __device__ __noinline__ void rope_table(const Params& p, int task) {
 // through shared memory in rounds so that all loads of a round are in flight
 // at once.
 //
-// A level that feeds a layer also gets the tile's share of that layer's
-// router logits: rpart[l][r][b][e] = sum over the tile's 64 columns c of
-// W_r[e][c] (gamma x)[b][c].  The producer streams the tile's router columns
-// into the ring when it hands the task out (128 expert rows of 128 bytes per
-// stage, 128-byte swizzled), so they are resident before the inputs are.
-// Unit u = 8 e + ch covers columns 8 ch .. 8 ch + 7 of expert row e (one
-// 16-byte shared load); the eight lanes of a row reduce by shuffles and lane
-// ch stores token ch.  Returns the advanced ring counter.
+// A level that feeds a layer also adds the tile's share of that layer's
+// router logits, sum over the tile's 64 columns c of W_r[e][c] (gamma x)[b][c],
+// and the tile's sum of squares into the layer's fixed-point accumulators
+// (racc, ssacc).  The producer streams the tile's router columns into the
+// ring when it hands the task out (128 expert rows of 128 bytes per stage,
+// 128-byte swizzled), so they are resident before the inputs are.  Returns
+// the advanced ring counter.
 __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
@@ -1680,17 +1830,20 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
     const float x0 = xs[cw * 64 + lane], x1 = xs[cw * 64 + 32 + lane];
     float ss = x0 * x0 + x1 * x1;
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-    if (lane == 0)
+    if (lane == 0) {
       reinterpret_cast<float*>(p.actA + (size_t)l * p.actA_bytes + p.actA_rows_bytes)[r * B + cw] = ss;
+      if (l < p.L) red_add_u64(p.ssacc + ((size_t)(p.epoch & 1u) * p.L + l) * B + cw, to_fixed(ss));
+    }
   }
   if (l == 0 && r == 0) rope_table(p, ent[32 + R_TASK]);
   if (nst == 0) return stage_ctr;
   cbar();
   if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K3);   // outputs written
-  float* out = p.rpart + ((size_t)l * p.NR + r) * B * p.E;
+  unsigned long long* out = p.racc + ((size_t)(p.epoch & 1u) * p.L + l) * B * p.E;
   // thread pair per expert row: half hf takes columns 32 hf .. 32 hf + 31
   // (four 16-byte units, four independent FMA chains); the pair adds its two
-  // sums by one shuffle and half hf stores the tokens b with b % 2 == hf
+  // sums by one shuffle and half hf adds the tokens b with b % 2 == hf into
+  // the layer's fixed-point logit accumulators
 #pragma unroll 1
   for (int s = 0; s < nst; ++s) {
     const uint32_t slot = stage_ctr % (uint32_t)sm.NS, ph = (stage_ctr / (uint32_t)sm.NS) & 1u;
@@ -1732,166 +1885,38 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
       }
       float sum = (a[0] + a[1]) + (a[2] + a[3]);
       sum += __shfl_xor_sync(FULL, sum, 1);
-      if (valid && (b & 1) == hf) out[(size_t)b * p.E + e0 + el] = sum;
+      if (valid && (b & 1) == hf) red_add_u64(out + (size_t)b * p.E + e0 + el, to_fixed(sum));
     }
   }
   if (ct == 0) cstamp(p, ent[32 + R_TASK], T_K4);   // router shares written
   return stage_ctr;
 }
 
-// Router logits of layer l from the norm tiles' shares, then top-k (logit
-// desc, index asc) + softmax over the selected + slot compaction.
-// logits[b][e] = (1/rms_b) * sum_r rpart[l][r][b][e] + bias[e], the shares
-// summed in ascending r: thread group g of nG sums r = g, g + nG, ... of one
-// float4 column, and the groups' sums are added in g order.
+// The top-k task of layer l: every token's router logits, top-k and softmax
+// (warp b takes token b) and the layer's routing table in global memory,
+// read by the expert tiles' producers (at batch sizes where they do not
+// route locally) and by the debug reads.  It also stands in for the signals
+// of the unused slots' tiles and zeroes the other step parity's accumulators
+// of the layer for the next step.
 __device__ __noinline__ void topk_task(const Params& p, int l) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
-  const int B = p.B, E = p.E, K = p.k, S = p.S, NR = p.NR;
-  int32_t* rt = p.route + (size_t)l * p.route_words;
-  int* sel = reinterpret_cast<int*>(sm.scratch);               // [B][8]
-  float* wsel = reinterpret_cast<float*>(sel + kMaxBatch * 8);  // [B][8]
-  int* slot_of = reinterpret_cast<int*>(wsel + kMaxBatch * 8); // [E]
-  uint32_t* used = reinterpret_cast<uint32_t*>(slot_of + 256); // [8]
-  float* rstd_s = reinterpret_cast<float*>(used + 8);          // [B]
-  float* lgs = reinterpret_cast<float*>(sm.scratch + kTopkLogitsOff);   // [B][E]
-  float4* grp = reinterpret_cast<float4*>(lgs + kMaxBatch * 256);       // [nG][C4]
-  const int C4 = B * E / 4;
-  const int span = min(C4, 256), nG = 256 / span;
-  const float* bias = router_b(p, sm, l);
-  const float bv = (bias && ct < E) ? __ldg(bias + ct) : 0.f;   // expert ct's bias
-  {
-    const float4* rp = reinterpret_cast<const float4*>(p.rpart + (size_t)l * NR * B * E);
-    if (ct < nG * span) {
-      const int g = ct / span;
-#pragma unroll 1
-      for (int c4 = ct - g * span; c4 < C4; c4 += 256) {
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        // eight independent loads in flight, then added in r order
-#pragma unroll 1
-        for (int rr0 = g; rr0 < NR; rr0 += 8 * nG) {
-          float4 v[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int rr = rr0 + j * nG;
-            v[j] = rr < NR ? __ldcg(rp + (size_t)rr * C4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            a.x += v[j].x;
-            a.y += v[j].y;
-            a.z += v[j].z;
-            a.w += v[j].w;
-          }
-        }
-        if (nG == 1)
-          reinterpret_cast<float4*>(lgs)[c4] = a;
-        else
-          grp[g * C4 + c4] = a;
-      }
-    }
-  }
-  if (ct < 8) used[ct] = 0u;
-  if (cw < B) {
-    // 1/rms of token cw from the level's sum-of-squares partials
-    const float* ss = reinterpret_cast<const float*>(p.actA + (size_t)l * p.actA_bytes +
-                                                     p.actA_rows_bytes);
-    float acc = 0.f;
-#pragma unroll 1
-    for (int rr = lane; rr < NR; rr += 32) acc += __ldcg(ss + rr * B + cw);
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if (lane == 0) rstd_s[cw] = frsqrt(acc / (float)p.d + p.eps);
+  const int B = p.B, E = p.E, S = p.S, NR = p.NR;
+  const uint32_t par = p.epoch & 1u;
+  int32_t* sel = reinterpret_cast<int32_t*>(sm.scratch);   // [8][8]
+  float* wsel = reinterpret_cast<float*>(sel + 64);          // [8][8]
+  uint32_t* mask = reinterpret_cast<uint32_t*>(wsel + 64);   // [8]
+  int* n_used_s = reinterpret_cast<int*>(mask + 8);
+  if (cw < B)
+    token_route(p, router_b(p, sm, l), l, par, cw, sel + cw * 8, wsel + cw * 8,
+                p.rlogits + ((size_t)l * B + cw) * E);
+  cbar();
+  if (cw == 0) {
+    const int nu = compact_routes(p, sel, wsel, mask, p.route + (size_t)l * p.route_words);
+    if (lane == 0) *n_used_s = nu;
   }
   cbar();
-  // thread e finishes expert e of every token
-  if (ct < E) {
-    const float* gs = reinterpret_cast<const float*>(grp);
-#pragma unroll 1
-    for (int bb = 0; bb < B; ++bb) {
-      const int i = bb * E + ct;
-      float v = nG == 1 ? lgs[i] : 0.f;
-#pragma unroll 1
-      for (int g = 0; g < (nG == 1 ? 0 : nG); ++g) v += gs[g * 4 * C4 + i];
-      v = v * rstd_s[bb] + bv;
-      lgs[i] = v;
-      p.rlogits[(size_t)l * B * E + i] = v;
-    }
-  }
-  cbar();
-  const int b = cw;
-  if (b < B) {
-    const float* lg = lgs + b * E;
-    // order-preserving unsigned keys of the logits; 0 marks taken / absent
-    uint32_t key[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int e = lane + 32 * t;
-      uint32_t k = 0u;
-      if (e < E) {
-        const uint32_t u = __float_as_uint(lg[e]);
-        k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-      }
-      key[t] = k;
-    }
-#pragma unroll 1
-    for (int j = 0; j < K; ++j) {
-      uint32_t bk = 0u;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (key[t] > bk) {   // ascending e within a lane: first max has the smallest e
-          bk = key[t];
-          bi = lane + 32 * t;
-        }
-      }
-      const uint32_t mk = __reduce_max_sync(FULL, bk);
-      const int wi = __reduce_min_sync(FULL, bk == mk ? bi : 0x7fffffff);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-        if (lane + 32 * t == wi) key[t] = 0u;
-      if (lane == 0) {
-        sel[b * 8 + j] = wi;
-        wsel[b * 8 + j] = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk);
-      }
-    }
-    __syncwarp();
-    // softmax over the selected logits: lane j < K takes rank j
-    const float v0 = wsel[b * 8];
-    float w = lane < K ? fexp(wsel[b * 8 + (lane & 7)] - v0) : 0.f;
-    float sum = w;
-    for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-    __syncwarp();
-    if (lane < K) {
-      w *= frcp(sum);
-      const int e = sel[b * 8 + lane];
-      wsel[b * 8 + lane] = w;
-      rt[route_topk_idx(B, K) + b * K + lane] = e;
-      reinterpret_cast<float*>(rt)[route_topk_w(B, K) + b * K + lane] = w;
-      atomicOr(&used[e >> 5], 1u << (e & 31));
-    }
-  }
-  cbar();
-  // slot of each used expert = number of used experts below it
-#pragma unroll 1
-  for (int e = ct; e < E; e += 256) {
-    int cnt = 0;
-#pragma unroll 1
-    for (int w = 0; w < (e >> 5); ++w) cnt += __popc(used[w]);
-    cnt += __popc(used[e >> 5] & ((1u << (e & 31)) - 1u));
-    slot_of[e] = ((used[e >> 5] >> (e & 31)) & 1u) ? cnt : -1;
-  }
-  cbar();
-  int n_used = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) n_used += __popc(used[w]);
-#pragma unroll 1
-  for (int s = ct; s < S; s += 256) {
-    if (s >= n_used) {
-      rt[route_slot_expert(B, K) + s] = -1;
-      rt[route_slot_ntok(B, K, S) + s] = 0;
-    }
-  }
-  if (ct == 0) rt[0] = n_used;
+  const int n_used = *n_used_s;
   // The producers drop the tiles of unused slots; stand in for the signals
   // those tiles would have sent: each down-tile row counter gets one per
   // unused slot, each unused slot's counter its n_ff gate/up tiles (so every
@@ -1902,29 +1927,11 @@ __device__ __noinline__ void topk_task(const Params& p, int l) {
     for (int j = n_used + ct; j < S; j += 256)
       atomicAdd(p.counters + p.slot_ctr0 + l * S + j, (uint32_t)p.n_ff);
   }
-  // one thread per (token, rank): its position in the slot's token list
-  if (ct < B * K) {
-    const int bb = ct / K, j = ct % K;
-    const int e = sel[bb * 8 + j];
-    const int s = slot_of[e];
-    int pos = 0;
-#pragma unroll 1
-    for (int b2 = 0; b2 < bb; ++b2)
-#pragma unroll 1
-      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
-    rt[route_slot_tok(B, K, S) + s * 8 + pos] = bb;
-    rt[route_slot_rank(B, K, S) + s * 8 + pos] = j;
-    reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s * 8 + pos] = wsel[bb * 8 + j];
-    if (pos == 0) {
-      int cnt = 0;
-#pragma unroll 1
-      for (int b2 = 0; b2 < B; ++b2)
-#pragma unroll 1
-        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
-      rt[route_slot_expert(B, K) + s] = e;
-      rt[route_slot_ntok(B, K, S) + s] = cnt;
-    }
-  }
+  // the next step accumulates into the other parity: start it at zero (this
+  // step's norm tiles only touch parity par)
+  const size_t lo = ((size_t)(par ^ 1u) * p.L + l) * B;
+  for (int i = ct; i < B * E; i += 256) p.racc[lo * E + i] = 0ull;
+  if (ct < B) p.ssacc[lo + ct] = 0ull;
 }
 
 // NBK: the GEMV path (1 and 2: FFMA for 1 or 2 tokens; 3: mma.sync for 3..8);

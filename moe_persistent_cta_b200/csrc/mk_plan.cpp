@@ -97,7 +97,7 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->actB_bytes = round_up(b_need, 128);
   int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
-  int sc_topk = kTopkLogitsOff + (kMaxBatch * 256 + 1024) * 4;   // logits + group sums
+  int sc_topk = (64 + 64 + 8 + 1) * 4;                            // selections, weights, mask
   int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
   int sc_comb = 256 * 16 + kMaxAttnOut * 4 + 3 * max_chunks * G * 4 + 2 * G * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
@@ -110,7 +110,8 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
                            128);
   const int budget = 232448 - 2048;   // max per block, less alignment slack and static smem
   const int ptrs = round_up(ptr_table_words(s.L) * 8, 128);
-  const int rcache = round_up(route_words(B, s.k, std::min(s.E, B * s.k)) * 4, 128);
+  const int rcache =
+      round_up((route_words(B, s.k, std::min(s.E, B * s.k)) + kRouteTmpWords) * 4, 128);
   int rest1 = bars + fifo + epi + ptrs + rcache + o->scratch_bytes + o->actA_stride +
               2 * o->actB_bytes;
   int rest2 = rest1 + o->actA_stride;
@@ -272,6 +273,18 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
       tasks.push_back(t);
     }
   };
+  // the producer of an expert tile needs the layer's routing: up to
+  // kLocalRouteMaxB tokens it computes the table itself once the layer's norm
+  // tiles are done; beyond that it waits for the layer's top-k task
+  auto set_route_wait = [&](Task& t, int l) {
+    if (B <= kLocalRouteMaxB) {
+      t.w[D_PW] = lay.norm(l);
+      t.w[D_PWN] = NR;
+    } else {
+      t.w[D_PW] = lay.rtr(l);
+      t.w[D_PWN] = 1;
+    }
+  };
   emit_norm(0);
   for (int l = 0; l < L; ++l) {
     if (l > 0) emit_norm(l);
@@ -373,8 +386,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         t.w[D_MAP0] = map_of(l, 3);
         t.w[D_MAP1] = map_of(l, 4);
         t.w[D_NSTAGE] = 2 * (r_ff / 16) * (d / 64) / 8;
-        t.w[D_PW] = lay.rtr(l);
-        t.w[D_PWN] = 1;
+        set_route_wait(t, l);
         add_wait(t, lay.norm(l), NR);
         add_signal(t, lay.slot(l, j));
         targets[lay.slot(l, j)] += 1;
@@ -394,8 +406,7 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
         t.w[D_NMAT] = 1;
         t.w[D_MAP0] = map_of(l, 5);
         t.w[D_NSTAGE] = 4 * (F / 64) / 8;
-        t.w[D_PW] = lay.rtr(l);
-        t.w[D_PWN] = 1;
+        set_route_wait(t, l);
         add_wait(t, lay.slot(l, j), n_ff);
         add_signal(t, lay.dt(l, r));
         targets[lay.dt(l, r)] += 1;

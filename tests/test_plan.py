@@ -123,10 +123,13 @@ def test_30b_b1_plan_structure():
     tk = desc[desc[:, D_OP] == OP_TOPK]
     assert np.all(tk[:, D_NWAIT] == 1) and np.all(tk[:, D_W0N] == d // 64)
     rn = desc[desc[:, D_OP] == OP_RN]
+    # at batch 1 each expert tile's producer computes the layer's routing
+    # itself once the layer's norm tiles are done: it waits on their counter
     gu = desc[desc[:, D_OP] == OP_GATEUP]
     for l in (0, 5, L - 1):
-        assert set(tk[tk[:, D_LAYER] == l][:, D_S0].tolist()) == \
-            set(gu[gu[:, D_LAYER] == l][:, D_PW].tolist())
+        norm_ctr = set(rn[rn[:, D_LAYER] == l][:, D_S0].tolist())
+        assert set(gu[gu[:, D_LAYER] == l][:, D_PW].tolist()) == norm_ctr
+        assert np.all(gu[gu[:, D_LAYER] == l][:, D_PWN] == d // 64)
     # a norm tile of a level that feeds a layer streams its router columns:
     # one ring stage per 128 experts; the final norm streams nothing
     E = shape["n_experts"]
@@ -178,6 +181,15 @@ def test_30b_b8_plan():
     meta, desc, targets = engine.plan_schedule(shape, 148, lens)
     check_order_and_targets(desc, targets, 148, meta[8])
     assert meta[2] == 64   # expert slots = min(E, B*k)
+    # at batch 8 the expert tiles' producers copy the top-k task's table:
+    # they wait on the top-k's signal
+    tk = desc[desc[:, D_OP] == OP_TOPK]
+    for op in (OP_GATEUP, OP_DOWN):
+        ex = desc[desc[:, D_OP] == op]
+        for l in (0, 20):
+            assert set(ex[ex[:, D_LAYER] == l][:, D_PW].tolist()) == \
+                set(tk[tk[:, D_LAYER] == l][:, D_S0].tolist())
+            assert np.all(ex[ex[:, D_LAYER] == l][:, D_PWN] == 1)
 
 
 def test_activation_levels_never_decrease():
