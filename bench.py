@@ -21,6 +21,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -232,6 +234,283 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+# --------------------------------------------------------------- measure --
+def step_roofline(shape, lens_mid, nslots, ms_per_step, n_layers_traffic=None, workload=None,
+                  unfused=False):
+    """HBM roofline of one step: algorithmic bytes (active weights of the
+    experts the step touched, KV read) over the step time."""
+    from moe_persistent_cta_b200 import roofline
+    sb = roofline.step_bytes(shape, lens_mid, [int(u) for u in nslots])
+    peak, peak_kind = hbm_peak()
+    achieved = sb["total"] / (ms_per_step / 1e3) / 1e9
+    traffic = None
+    if workload is not None and not unfused:
+        traffic = kernel_traffic(workload, n_layers_traffic or shape["n_layers"])
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+            "bytes_per_step": sb["total"], "weight_bytes": sb["weights"], "kv_bytes": sb["kv"],
+            "frac_of_8tbs_spec": achieved / 8000.0,
+            "experts_per_layer_mean": float(np.mean(nslots))}
+
+
+def plan_launches(dec, unfused):
+    """Kernel launches of one step: one for the fused step; one per operation
+    phase that holds tasks for the unfused path (counted from the schedule)."""
+    if not unfused:
+        return 1
+    from moe_persistent_cta_b200 import mk
+    desc = dec.debug(mk.MK_BUF_PLAN).reshape(-1, 32)
+    return int(len(set(desc[:, 28].tolist())))
+
+
+def measure_steps(name, W, dev, steps, warmup, impl="mk", dist=None, rank=0, world=1,
+                  layers=0, with_e2e=True, keep_kv=False):
+    """K timed steps of one workload (inputs staged in HBM), then the same
+    loop end to end through the public API with host buffers."""
+    import torch
+    from moe_persistent_cta_b200 import configs, engine, mk, synth
+    wl = dict(configs.WORKLOADS[name])
+    shape = dict(wl["shape"])
+    if layers > 0:
+        shape["n_layers"] = layers
+    B = wl["batch"]
+    lens = synth.seq_lengths(wl["seq_lens"], B)
+    steps_total = warmup + steps
+    table, n_pages = synth.make_page_tables(lens, wl.get("contiguous", False), wl["page_seed"],
+                                            growth=max(64, steps_total + 1))
+    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], str(dev))
+    dec = engine.Decoder(shape, W, k, v, max_batch=B, device=dev.index)
+    plan_len = [s + steps_total + 1 for s in lens]
+    dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
+    gen = torch.Generator(device="cpu").manual_seed(wl["token_seed"])
+    toks = torch.randint(0, shape["vocab"], (steps_total, B), generator=gen, dtype=torch.int32)
+    pos = torch.tensor([[s + i for s in lens] for i in range(steps_total)], dtype=torch.int32)
+    toks_d, pos_d, table_d = toks.to(dev), pos.to(dev), table.to(dev)
+    logits = torch.empty((B, shape["vocab"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    unfused = impl == "unfused"
+
+    def run(i):
+        dec.step(toks_d[i], pos_d[i], table_d, pos_d[i], logits, stream=stream, unfused=unfused)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            run(i)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(warmup, steps_total):
+        run(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    dec.check_ok()
+    nslots = dec.debug(mk.MK_BUF_NSLOTS)
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / steps
+    out = {"name": name, "shape": shape, "batch": B, "lens": lens, "steps": steps,
+           "warmup": warmup, "ms_per_step": ms_per_step,
+           "value": world * B * steps / (ms / 1e3), "clocks": clk,
+           "gpu_launches": steps * plan_launches(dec, unfused)}
+    mid = [s + warmup + steps // 2 for s in lens]
+    out["roofline"] = step_roofline(shape, mid, nslots, ms_per_step, workload=name,
+                                    unfused=unfused)
+    if with_e2e:
+        # per step: tokens, positions and the page table host->device from
+        # pinned memory, the logits device->host
+        h_toks, h_pos, h_table = toks.pin_memory(), pos.pin_memory(), table.pin_memory()
+        h_logits = torch.empty((B, shape["vocab"]), dtype=torch.float32).pin_memory()
+        d_tok = torch.empty(B, dtype=torch.int32, device=dev)
+        d_pos = torch.empty(B, dtype=torch.int32, device=dev)
+        dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(steps):
+                d_tok.copy_(h_toks[i], non_blocking=True)
+                d_pos.copy_(h_pos[i], non_blocking=True)
+                table_d.copy_(h_table, non_blocking=True)
+                dec.step(d_tok, d_pos, table_d, d_pos, logits, stream=stream, unfused=unfused)
+                h_logits.copy_(logits, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        dec.check_ok()
+        e2e_ms = e0.elapsed_time(e1)
+        if dist:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        out["e2e"] = {"value": world * B * steps / (e2e_ms / 1e3), "unit": "tok/s",
+                      "h2d_bytes_per_step": B * 4 * 2 + table.numel() * 4,
+                      "d2h_bytes_per_step": B * shape["vocab"] * 4}
+    out["wl"] = wl
+    out["toks0"] = [int(t) for t in toks[0]]
+    out["table"] = table
+    dec.close()
+    if keep_kv:
+        out["kv"] = (k, v)
+    del k, v
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_greedy(name, W, dev, steps, warmup):
+    """K greedy steps in one mk_decode_greedy call: the tokens, positions and
+    lengths advance on the device with no host round trip between steps.
+    e2e: the first step's inputs host->device and the K generated tokens back."""
+    import torch
+    from moe_persistent_cta_b200 import configs, engine, mk, synth
+    wl = configs.WORKLOADS[name]
+    shape, B = wl["shape"], wl["batch"]
+    lens = synth.seq_lengths(wl["seq_lens"], B)
+    total = warmup + 2 * steps
+    table, n_pages = synth.make_page_tables(lens, wl.get("contiguous", False), wl["page_seed"],
+                                            growth=total + 64)
+    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], str(dev))
+    dec = engine.Decoder(shape, W, k, v, max_batch=B, device=dev.index)
+    dec.build_schedule(lens, table.shape[1], plan_len=[s + total + 1 for s in lens])
+    i32 = dict(dtype=torch.int32, device=dev)
+    tok = torch.tensor(synth.make_tokens(B, shape["vocab"], wl["token_seed"]), **i32)
+    pos = torch.tensor(lens, **i32)
+    table_d = table.to(dev)
+    out = torch.empty((total, B), **i32)
+    logits = torch.empty((B, shape["vocab"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    dec.greedy(warmup, tok, pos, table_d, pos, logits, out[:warmup], stream=stream)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    dec.greedy(steps, tok, pos, table_d, pos, logits, out[warmup:warmup + steps], stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dec.check_ok()
+    ms = ev0.elapsed_time(ev1)
+    nslots = dec.debug(mk.MK_BUF_NSLOTS)
+    mid = [s + warmup + steps // 2 for s in lens]
+    res = {"metric": "decode tok/s, on-device greedy (one call, no host round trip per step)",
+           "value": B * steps / (ms / 1e3), "unit": "tok/s", "ms_per_step": ms / steps,
+           "steps": steps, "warmup": warmup, "clocks": clk, "gpu_launches": steps,
+           "roofline": step_roofline(shape, mid, nslots, ms / steps, workload=name)}
+    # e2e: host inputs of the first step in, the generated tokens out
+    h_in = torch.tensor([synth.make_tokens(B, shape["vocab"], wl["token_seed"]),
+                         [s + warmup + steps for s in lens]], dtype=torch.int32).pin_memory()
+    h_out = torch.empty((steps, B), dtype=torch.int32).pin_memory()
+    h_table = table.pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        tok.copy_(h_in[0], non_blocking=True)
+        pos.copy_(h_in[1], non_blocking=True)
+        table_d.copy_(h_table, non_blocking=True)
+        dec.greedy(steps, tok, pos, table_d, pos, logits, out[warmup + steps:], stream=stream)
+        h_out.copy_(out[warmup + steps:], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    e2e_ms = e0.elapsed_time(e1)
+    res["e2e"] = {"value": B * steps / (e2e_ms / 1e3), "unit": "tok/s",
+                  "h2d_bytes_per_step": (h_in.numel() * 4 + table.numel() * 4) / steps,
+                  "d2h_bytes_per_step": B * 4}
+    res["config"] = {"workload": workload_desc(name, wl, lens) + ", greedy tokens fed back on "
+                     "the device", "batch": B}
+    dec.close()
+    del k, v
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_continuous(W, dev, steps):
+    """Continuous batching on the 30B shape: 8 slots, sequences starting at
+    U[512, 32768] cached tokens and stopping after Geometric(mean 128) new
+    tokens, refilled as they stop, Zipf routing, greedy tokens.  The steps
+    between two refills run as one mk_decode_greedy call; value = generated
+    tokens / (decode + rebuild time); the synthetic prefix fills of refilled
+    slots (a stand-in for prefill, which runs outside the decode engine) only
+    enter e2e."""
+    import time as _time
+    import torch
+    from moe_persistent_cta_b200 import configs, engine, mk, roofline, serving
+    cfg = configs.CONTINUOUS
+    shape, slots = cfg["shape"], cfg["slots"]
+    max_pages = serving.pages_for(cfg["start_hi"] + steps + 1)
+    n_pages = slots * (max_pages + 1) + 16
+    L, Hkv, hd = shape["n_layers"], shape["n_kv_heads"], shape["head_dim"]
+    k = torch.zeros((L, n_pages, Hkv, 64, hd), dtype=torch.bfloat16, device=dev)
+    v = torch.zeros_like(k)
+    dec = engine.Decoder(shape, W, k, v, max_batch=slots, device=dev.index)
+    # new-token counts are drawn geometric with mean 128; a sequence can
+    # never outlive the run, so the run's length is the only cap
+    common = dict(slots=slots, start_lo=cfg["start_lo"], start_hi=cfg["start_hi"],
+                  mean_new=cfg["mean_new"], max_new=steps, max_pages_per_seq=max_pages)
+    serving.run_continuous(dec, shape, k, v, steps=16, seed=cfg["seed"] + 99, **common)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    t0 = _time.perf_counter()
+    r = serving.run_continuous(dec, shape, k, v, steps=steps, seed=cfg["seed"], **common)
+    wall = _time.perf_counter() - t0
+    clk = clocks.stop()
+    nslots = dec.debug(mk.MK_BUF_NSLOTS)
+    busy = r["decode_s"] + r["rebuild_s"]
+    total_bytes = sum(roofline.step_bytes(shape, [int(x) for x in r["lens_per_step"][i]],
+                                          [int(u) for u in nslots])["total"]
+                      for i in range(steps))
+    peak, peak_kind = hbm_peak()
+    achieved = total_bytes / r["decode_s"] / 1e9
+    res = {"metric": "decode tok/s, continuous batching (8 slots, 512 steps, 30B-MoE shape)",
+           "value": r["generated"] / busy, "unit": "tok/s", "steps": steps,
+           "ms_per_step": busy / steps * 1e3, "higher_is_better": True,
+           "config": {"workload": "moe30b_cb: 30B-MoE shape, 8 slots, start U[512, 32768], "
+                                  "Geometric(mean 128) new tokens, Zipf routing, 64-token "
+                                  "pages, one schedule planned at full slot capacity",
+                      "sequences": r["sequences"], "finished": r["finished"],
+                      "rebuilds": r["rebuilds"], "greedy_calls": r["greedy_calls"],
+                      "rebuild_s": round(r["rebuild_s"], 4),
+                      "prefix_fill_s": round(r["prefix_fill_s"], 4),
+                      "timing": "CUDA events on the stream around each mk_decode_greedy "
+                                "call (decode) plus host time of schedule rebuilds"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                        "bytes_per_step_mean": total_bytes / steps,
+                        "note": "KV bytes from every step's lengths; weight bytes at the "
+                                "last step's expert union per layer"},
+           "e2e": {"value": r["generated"] / (busy + r["prefix_fill_s"]), "unit": "tok/s",
+                   "h2d_bytes_per_step": None, "d2h_bytes_per_step": slots * 4,
+                   "wall_s": round(wall, 3)},
+           "gpu_launches": steps, "clocks": clk}
+    dec.close()
+    del k, v
+    torch.cuda.empty_cache()
+    return res
+
+
+def config_entry(m, impl):
+    return {"metric": METRIC + (" (unfused per-op launches)" if impl == "unfused" else ""),
+            "value": m["value"], "unit": "tok/s", "steps": m["steps"], "warmup": m["warmup"],
+            "ms_per_step": m["ms_per_step"], "roofline": m["roofline"], "e2e": m.get("e2e"),
+            "clocks": m["clocks"], "gpu_launches": m["gpu_launches"],
+            "config": {"workload": workload_desc(m["name"], m["wl"], m["lens"]),
+                       "batch": m["batch"],
+                       "impl": "unfused per-op launches" if impl == "unfused"
+                       else "fused megakernel"}}
+
+
 # ------------------------------------------------------------------- main --
 def main():
     ap = argparse.ArgumentParser()
@@ -241,6 +520,9 @@ def main():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference", "unfused"])
     ap.add_argument("--workload", default="moe30b_b1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="measure the headline workload only (no per-config lines)")
+    ap.add_argument("--cb-steps", type=int, default=512)
     ap.add_argument("--oracle-layers", type=int, default=2)
     ap.add_argument("--layers", type=int, default=0,
                     help="cut the workload's model to this many layers (small cases for "
@@ -254,12 +536,6 @@ def main():
     import torch
     from moe_persistent_cta_b200 import configs, synth
 
-    if args.workload == "moe30b_cb":
-        if args.impl != "mk":
-            print(json.dumps({"impl": args.impl, "unavailable":
-                              "continuous batching is measured for the fused step only"}))
-            return 0
-        return run_continuous_bench(args)
     wl = dict(configs.WORKLOADS[args.workload])
     if args.layers > 0:
         wl["shape"] = dict(wl["shape"], n_layers=args.layers)
@@ -284,120 +560,54 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    from moe_persistent_cta_b200 import engine, mk, roofline
-
-    steps_total = args.warmup + args.steps
-    growth = max(64, steps_total + 1)
-    table, n_pages = synth.make_page_tables(lens, wl.get("contiguous", False), wl["page_seed"],
-                                            growth=growth)
     W = synth.make_weights(shape, wl["weight_seed"], str(dev), wl.get("routing", "uniform"),
                            wl.get("zipf_s", 1.1))
-    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], str(dev))
-    dec = engine.Decoder(shape, W, k, v, max_batch=B, device=dev.index)
-    plan_len = [s + steps_total + 1 for s in lens]
-    dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
-
-    # all steps' inputs staged in HBM before timing: step s feeds a seeded
-    # token at position len + s
-    gen = torch.Generator(device="cpu").manual_seed(wl["token_seed"])
-    toks = torch.randint(0, shape["vocab"], (steps_total, B), generator=gen, dtype=torch.int32)
-    pos = torch.tensor([[s + i for s in lens] for i in range(steps_total)], dtype=torch.int32)
-    toks_d, pos_d = toks.to(dev), pos.to(dev)
-    table_d = table.to(dev)
-    logits = torch.empty((B, shape["vocab"]), dtype=torch.float32, device=dev)
-    stream = torch.cuda.Stream(device=dev)
-    unfused = args.impl == "unfused"
-
-    def run(i):
-        dec.step(toks_d[i], pos_d[i], table_d, pos_d[i], logits, stream=stream, unfused=unfused)
-
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            run(i)
-    torch.cuda.synchronize()
-    dec.check_ok()
-    nslots = dec.debug(mk.MK_BUF_NSLOTS)
-
-    clocks = ClockSampler(dev.index)
-    if rank == 0:
-        clocks.start()
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(args.warmup, steps_total):
-        run(i)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    clk = clocks.stop() if rank == 0 else None
-    dec.check_ok()
-    ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_per_step = ms / args.steps
-    tok_s = world * B * args.steps / (ms / 1e3)
-
-    # roofline of the step (the one kernel): algorithmic bytes per launch
-    mid_lens = [s + args.warmup + args.steps // 2 for s in lens]
-    sb = roofline.step_bytes(shape, mid_lens, [int(u) for u in nslots])
-    peak, peak_kind = hbm_peak()
-    achieved = sb["total"] / (ms_per_step / 1e3) / 1e9
-
-    # end to end through the public API with host buffers: per step the
-    # inputs go host->device from pinned memory and the logits come back
-    h_toks = toks.pin_memory()
-    h_pos = pos.pin_memory()
-    h_table = table.pin_memory()
-    h_logits = torch.empty((B, shape["vocab"]), dtype=torch.float32).pin_memory()
-    d_tok = torch.empty(B, dtype=torch.int32, device=dev)
-    d_pos = torch.empty(B, dtype=torch.int32, device=dev)
-    e2e_steps = args.steps
-    dec.build_schedule(lens, table.shape[1], plan_len=plan_len)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(e2e_steps):
-            d_tok.copy_(h_toks[i], non_blocking=True)
-            d_pos.copy_(h_pos[i], non_blocking=True)
-            table_d.copy_(h_table, non_blocking=True)
-            dec.step(d_tok, d_pos, table_d, d_pos, logits, stream=stream, unfused=unfused)
-            h_logits.copy_(logits, non_blocking=True)
-        e1.record(stream)
-    torch.cuda.synchronize()
-    dec.check_ok()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_tok_s = world * B * e2e_steps / (e2e_ms / 1e3)
-    h2d = (B * 4) * 2 + table.numel() * 4
-    d2h = B * shape["vocab"] * 4
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    head = measure_steps(args.workload, W, dev, args.steps, args.warmup, impl=args.impl,
+                         dist=dist, rank=rank, world=world, layers=args.layers,
+                         keep_kv=want_cpu)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(shape, W, k, v, table.numpy(), args.oracle_layers, 4096)
-        full_s, measured_s, reps = repeat_sample(smp, [int(t) for t in toks[0]], lens)
+    if want_cpu:
+        k, v = head.pop("kv")
+        smp = OracleSample(shape, W, k, v, head["table"].numpy(), args.oracle_layers, 4096)
+        del k, v
+        torch.cuda.empty_cache()
+        full_s, measured_s, reps = repeat_sample(smp, head["toks0"], lens)
         cpu = {"value": B / full_s, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
                "sample": smp.describe() + f"; repeated {reps} times, mean taken",
                "sample_seconds": round(measured_s, 2)}
 
+    per_config = None
+    if world == 1 and not args.no_configs and args.layers == 0 and args.impl == "mk" \
+            and args.workload == "moe30b_b1":
+        per_config = {}
+        Wz = dict(W)
+        Wz["w_router"], Wz["router_bias"] = synth.make_router(shape, wl["weight_seed"], str(dev),
+                                                              "zipf", 1.1)
+        b8 = measure_steps("moe30b_b8_zipf", Wz, dev, args.steps, args.warmup)
+        per_config["moe30b_b8_zipf"] = config_entry(b8, "mk")
+        lk = measure_steps("moe30b_b1_256k", W, dev, max(3, args.steps // 2), args.warmup)
+        per_config["moe30b_b1_256k"] = config_entry(lk, "mk")
+        u1 = measure_steps("moe30b_b1", W, dev, max(3, args.steps // 2), args.warmup,
+                           impl="unfused")
+        per_config["unfused_moe30b_b1"] = config_entry(u1, "unfused")
+        u8 = measure_steps("moe30b_b8_zipf", Wz, dev, max(3, args.steps // 4), args.warmup,
+                           impl="unfused")
+        per_config["unfused_moe30b_b8_zipf"] = config_entry(u8, "unfused")
+        per_config["greedy_moe30b_b1"] = measure_greedy("moe30b_b1", W, dev, args.steps,
+                                                        args.warmup)
+        per_config["continuous_moe30b_cb"] = measure_continuous(Wz, dev, args.cb_steps)
+
     if rank == 0:
         out = {
             "metric": METRIC,
-            "value": tok_s,
+            "value": head["value"],
             "unit": "tok/s",
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
-            "ms_per_step": ms_per_step,
+            "ms_per_step": head["ms_per_step"],
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
@@ -407,91 +617,21 @@ def main():
                        "global_batch": B * world,
                        "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (weights+KV streamed per step >> 126 MB)",
-                       "impl": "unfused per-op launches" if unfused else "fused megakernel",
-                       "experts_per_layer_mean": float(sum(nslots) / len(nslots))},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": (kernel_traffic(args.workload, shape["n_layers"])
-                                     if not unfused else None),
-                         "peak_kind": peak_kind,
-                         "bytes_per_step": sb["total"], "weight_bytes": sb["weights"],
-                         "kv_bytes": sb["kv"],
-                         "frac_of_8tbs_spec": achieved / 8000.0},
+                       "impl": "unfused per-op launches" if args.impl == "unfused"
+                       else "fused megakernel",
+                       "experts_per_layer_mean": head["roofline"]["experts_per_layer_mean"]},
+            "roofline": head["roofline"],
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_tok_s, "unit": "tok/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * (1 if not unfused else
-                                          sum(1 for n in dec_phase_counts(dec) if n)),
-            "clocks": clk,
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"],
+            "per_config": per_config,
         }
         print(json.dumps(out))
-    dec.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def run_continuous_bench(args):
-    """Continuous batching on the 30B shape: 8 slots, sequences starting at
-    U[512, 32768] cached tokens and stopping after Geometric(mean 128) new
-    tokens (capped at 1024), refilled as they stop, Zipf routing, greedy
-    tokens; schedules rebuilt between steps as needed.  value = generated
-    tokens / (decode + rebuild time); the synthetic prefix fills of refilled
-    slots (a stand-in for prefill, which runs outside the decode engine) are
-    timed apart and only enter e2e."""
-    import torch
-    from moe_persistent_cta_b200 import configs, engine, serving, synth
-    cfg = configs.CONTINUOUS
-    shape = cfg["shape"]
-    slots, steps = cfg["slots"], cfg["steps"]
-    max_new = 1024
-    max_pages = serving.pages_for(cfg["start_hi"] + max_new + 1)
-    n_pages = slots * max_pages + 16
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    W = synth.make_weights(shape, cfg["seed"], str(dev), cfg["routing"], cfg["zipf_s"])
-    L, Hkv, hd = shape["n_layers"], shape["n_kv_heads"], shape["head_dim"]
-    k = torch.zeros((L, n_pages, Hkv, 64, hd), dtype=torch.bfloat16, device=dev)
-    v = torch.zeros_like(k)
-    dec = engine.Decoder(shape, W, k, v, max_batch=slots)
-    common = dict(slots=slots, start_lo=cfg["start_lo"], start_hi=cfg["start_hi"],
-                  mean_new=cfg["mean_new"], max_new=max_new, max_pages_per_seq=max_pages)
-    serving.run_continuous(dec, shape, k, v, steps=max(3, args.warmup), seed=cfg["seed"] + 99,
-                           **common)
-    clocks = ClockSampler(0)
-    clocks.start()
-    r = serving.run_continuous(dec, shape, k, v, steps=steps, seed=cfg["seed"], **common)
-    clk = clocks.stop()
-    busy = r["decode_s"] + r["rebuild_s"]
-    out = {
-        "metric": "decode tok/s, continuous batching (8 slots, 512 steps, 30B-MoE shape)",
-        "value": r["generated"] / busy, "unit": "tok/s", "n_gpus": 1, "steps": steps,
-        "warmup": max(3, args.warmup), "ms_per_step": busy / steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded weights, Zipf routing, synthetic cached prefixes)",
-        "config": {"workload": "moe30b_cb: 30B-MoE shape, 8 slots, start U[512, 32768], "
-                               "Geometric(mean 128) new tokens capped at 1024, 64-token pages",
-                   "sequences": r["sequences"], "finished": r["finished"],
-                   "rebuilds": r["rebuilds"], "rebuild_s": round(r["rebuild_s"], 3),
-                   "prefix_fill_s": round(r["prefix_fill_s"], 3),
-                   "timing": "host wall clock per step (step, argmax, uploads, sync)"},
-        "roofline": None,
-        "e2e": {"value": r["generated"] / (busy + r["prefix_fill_s"]), "unit": "tok/s",
-                "h2d_bytes_per_step": slots * 4 * 2 + slots * max_pages * 4,
-                "d2h_bytes_per_step": 0},
-        "gpu_launches": steps,
-        "clocks": clk,
-    }
-    print(json.dumps(out))
-    dec.close()
-    return 0
-
-
-def dec_phase_counts(dec):
-    # phases with tasks (one launch each in the unfused path)
-    L = dec.L
-    return [1] * (8 * L + 2)
 
 
 def run_reference(args, wl, shape, lens):
@@ -506,13 +646,14 @@ def run_reference(args, wl, shape, lens):
     k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], "cuda" if torch.cuda.is_available()
                          else "cpu")
     toks = synth.make_tokens(B, shape["vocab"], wl["token_seed"])
-    times = []
+    times, measured = [], 0.0
     smp = OracleSample(shape, W, k, v, table.numpy(), 1, 2048)
     desc = smp.describe()
     for i in range(args.warmup + args.steps):
-        full_s, _ = smp.run(toks, lens)
+        full_s, m = smp.run(toks, lens)
         if i >= args.warmup:
             times.append(full_s)
+            measured += m
     mean_s = sum(times) / len(times)
     value = B / mean_s
     out = {
@@ -520,9 +661,13 @@ def run_reference(args, wl, shape, lens):
         "warmup": args.warmup, "ms_per_step": mean_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
+        # each step is a bounded sample of the full step, scaled up: ms_per_step
+        # is that projection; measured_s is the CPU time the timed steps took
+        "projected": True,
+        "measured_s": round(measured, 3),
         "config": {"workload": workload_desc(args.workload, wl, lens), "batch": B},
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": blas_threads(),
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "sample": desc, "sample_seconds": round(measured, 3)},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -52,3 +52,24 @@ def test_hbm_peak_measured_and_fallback(tmp_path, monkeypatch):
     p.write_text("{not json")
     monkeypatch.setattr(bench, "PEAKS_PATH", str(p))
     assert bench.hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+
+
+def test_step_roofline_counts_the_touched_experts_and_the_kv():
+    """The roofline's bytes are the active weights of the experts each layer
+    touched plus the KV read, and frac = bytes / time / peak."""
+    from moe_persistent_cta_b200 import configs
+    shape = configs.MOE30B
+    L = shape["n_layers"]
+    r1 = bench.step_roofline(shape, [8192], [8] * L, 2.0)
+    r8 = bench.step_roofline(shape, [8192], [16] * L, 2.0)
+    expert = 3 * shape["d_ff"] * shape["d_model"] * 2
+    assert r8["weight_bytes"] - r1["weight_bytes"] == L * 8 * expert
+    kv_tok = L * 2 * shape["n_kv_heads"] * shape["head_dim"] * 2
+    assert r1["kv_bytes"] == 8193 * kv_tok
+    assert r1["bytes_per_step"] == r1["weight_bytes"] + r1["kv_bytes"]
+    peak, _ = bench.hbm_peak()
+    assert r1["achieved"] == pytest.approx(r1["bytes_per_step"] / 2e-3 / 1e9)
+    assert r1["frac"] == pytest.approx(r1["achieved"] / peak)
+    assert r1["experts_per_layer_mean"] == 8.0
+    # the batch-1 30B step: about 6.08 GB, as the design notes state
+    assert 6.0e9 < r1["bytes_per_step"] < 6.2e9

@@ -5,8 +5,9 @@ vocab 151552), in the launch configuration bench.py times.
   the oracle (every layer, final logits), selection forced only where the
   oracle's k-th/(k+1)-th router gap is under 1e-3, plus teacher-forced
   single-layer checks (the oracle layer applied to the GPU's own layer input);
-* batch 8, ragged 1K-16K lengths, Zipf routing: teacher-forced layers for
-  every token and the whole step for sampled tokens (tokens are independent);
+* batch 8, ragged 1K-16K lengths, Zipf routing: the oracle's whole 48-layer
+  step for every token (expert selection identical at every layer outside the
+  tie band, final logits), plus teacher-forced layers 0, 24 and 47;
 * batch 1, 262144-token KV: teacher-forced layers (split-KV attention with
   ~37 chunks per KV group and the combine) and the LM head.
 """
@@ -145,7 +146,7 @@ def test_30b_b8_zipf(model):
     try:
         worst = r.teacher_forced([0, 24, 47], range(8))
         print(f"30B b8 zipf: teacher-forced layer max-abs {worst:.3e}")
-        for b in (0, 5):
+        for b in range(8):
             ref, forced = r.whole_step(b)
             got = r.logits[b].cpu().double().numpy()
             err, rel = compare_logits(got, ref)

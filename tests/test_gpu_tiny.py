@@ -5,9 +5,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from moe_persistent_cta_b200 import configs, mk
 from tests.gpu_common import (MAX_ABS, REL_L2, TinyRig, compare_logits, router_gap)
-from tests.oracle_io import array_kv
+from tests.oracle_io import array_kv, oracle_shape
 
 pytestmark = pytest.mark.gpu
 
@@ -78,20 +79,52 @@ def test_deterministic(rig):
     assert np.array_equal(a, b)
 
 
+def bf16_neighbour(bits, toward_larger):
+    """The bf16 bit pattern adjacent to `bits` in value, above or below."""
+    b = bits.astype(np.int32)
+    neg = (b & 0x8000) != 0
+    step = np.where(toward_larger ^ neg, 1, -1)     # magnitude +1 moves away from zero
+    return ((b + step) & 0xFFFF).astype(np.uint16)
+
+
 def test_kv_append_matches_oracle_bits(rig):
+    """The appended K and V are bf16 roundings of the projected (and, for K,
+    rotated) values: a quantisation, so they must match bit for bit.  Both
+    sides round to nearest even, but from different precisions (fp32 on the
+    GPU, float64 in the oracle), so where the oracle's value lies within the
+    GPU's measured projection error of the midpoint between two bf16 values
+    either neighbour is a correct rounding; everywhere else the bits must be
+    identical."""
     rec = {}
     rig.step()
     rig.oracle_step(record=rec)
+    S = oracle_shape(rig.shape)
+    L, hq, hkv, hd = S.n_layers, S.n_q_heads, S.n_kv_heads, S.head_dim
+    qkv_gpu = rig.dec.debug(mk.MK_BUF_QKV).reshape(L, rig.B, -1).astype(np.float64)
     pos = rig.lens[0]
     page = int(rig.table[0][pos // 64])
     kd = rig.kd.view(torch.int16).cpu().numpy().view(np.uint16)
     vd = rig.vd.view(torch.int16).cpu().numpy().view(np.uint16)
-    for l in range(rig.shape["n_layers"]):
-        for ours, ref in ((kd[l, page, :, pos % 64, :], rec[(l, 0)]["k_bits"]),
-                          (vd[l, page, :, pos % 64, :], rec[(l, 0)]["v_bits"])):
-            diff = np.abs(ours.astype(np.int32) - ref.astype(np.int32))
-            assert diff.max() <= 1            # at most one bf16 ulp (fp32 vs fp64 rounding)
-            assert (diff > 0).mean() < 0.02
+    cos, sin = oracle.rope_cos_sin(pos, hd, S.rope_theta)
+    n_amb = n_all = 0
+    for l in range(L):
+        r = rec[(l, 0)]
+        delta = float(np.max(np.abs(qkv_gpu[l, 0] - r["qkv"])))
+        k = r["qkv"][hq * hd:(hq + hkv) * hd].reshape(hkv, hd)
+        v = r["qkv"][(hq + hkv) * hd:].reshape(hkv, hd)
+        k_rot = oracle.apply_rope(k, cos, sin)
+        for ours, ref, x, eps in ((kd[l, page, :, pos % 64, :], r["k_bits"], k_rot, 2 * delta),
+                                  (vd[l, page, :, pos % 64, :], r["v_bits"], v, delta)):
+            assert np.array_equal(ref, oracle.f64_to_bf16_bits(x))
+            vb = oracle.bf16_bits_to_f64(ref)
+            other = np.where(x > vb, bf16_neighbour(ref, True), bf16_neighbour(ref, False))
+            mid = 0.5 * (vb + oracle.bf16_bits_to_f64(other))
+            amb = (np.abs(x - mid) <= eps) & (x != vb)
+            exact = ours == ref
+            assert np.all(exact | (amb & (ours == other))), (l, int((~exact & ~amb).sum()))
+            n_amb += int(amb.sum())
+            n_all += x.size
+    assert n_amb < 0.05 * n_all      # the band is narrow: almost every value is checked exactly
 
 
 @pytest.mark.parametrize("lens,shuffled", [([5, 64, 200], True), ([0, 1, 63, 64, 65, 127, 128, 129], True)])
