@@ -1062,8 +1062,9 @@ struct Ring {
   }
 };
 
-// CUDA-core stage loop for 1 or 2 activation columns: exact fp32 FMAs of
-// bf16 weights (widened by a shift/mask) with fp32 activations.  Lane l reads
+// CUDA-core stage loop for 1 or 2 activation columns (partial rows of pc
+// floats): exact fp32 FMAs of bf16 weights (widened by a shift/mask) with fp32
+// activations.  Lane l reads
 // 16-byte chunk (l & 7) of rows (l >> 3) + 4i of its warp's 16-row unit, so a
 // warp's 32 lanes cover the unit's 512 bytes per row group without bank
 // conflicts; partial sums are reduced over the 8 lanes of a row at the end.
@@ -1072,7 +1073,7 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
                                                  int kcps, int kl, uint32_t xaddr0,
                                                  uint32_t xaddr1, Ring& ring, float* part_w,
                                                  uint32_t pe_bar, uint32_t pe_par,
-                                                 uint32_t& waitcyc) {
+                                                 uint32_t& waitcyc, int pc) {
   MK_CONSUMER_IDS;
   const int c = lane & 7, rg = lane >> 3;
   float acc[4][NB];
@@ -1142,7 +1143,7 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int b = 0; b < NB; ++b) part_w[(rg + 4 * i) * NB + b] = acc[i][b];
+      for (int b = 0; b < NB; ++b) part_w[(rg + 4 * i) * pc + b] = acc[i][b];
   }
 }
 
@@ -1225,10 +1226,18 @@ __device__ __forceinline__ uint32_t gemv_consume(const Params& p, const int32_t*
   const uint64_t l0 = clock64();
   if constexpr (NBK == 1) {
     gemv_stages_ffma<1>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4, 0, ring, pw,
-                        pe_bar, pe_par, waitcyc);
+                        pe_bar, pe_par, waitcyc, 1);
   } else if constexpr (NBK == 2) {
     gemv_stages_ffma<2>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4,
-                        xbase + row_of(1) * stride * 4, ring, pw, pe_bar, pe_par, waitcyc);
+                        xbase + row_of(1) * stride * 4, ring, pw, pe_bar, pe_par, waitcyc, 2);
+  } else if (ncols == 1) {
+    // an expert tile of one or two tokens in a larger batch: the exact FFMA
+    // path costs fewer instructions per stage than eight mma columns
+    gemv_stages_ffma<1>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4, 0, ring, pw,
+                        pe_bar, pe_par, waitcyc, 8);
+  } else if (ncols == 2) {
+    gemv_stages_ffma<2>(p, sm, nstage, kcps, kl, xbase + row_of(0) * stride * 4,
+                        xbase + row_of(1) * stride * 4, ring, pw, pe_bar, pe_par, waitcyc, 8);
   } else {
     gemv_stages_mma(p, sm, nstage, kcps, kl, xbase + row_of(lane >> 2) * stride * 4, ring, pw,
                     pe_bar, pe_par, waitcyc);
