@@ -48,6 +48,9 @@ constexpr int kMaxAttnOut = 512;    // G x hd floats of one (token, KV head) out
 // itself from the norm tiles' accumulators (one warp, a few microseconds),
 // instead of waiting for the layer's top-k task and copying its table.
 constexpr int kLocalRouteMaxB = 4;
+// Attention chunks of up to this many pages let their CTA take its next task
+// before the chunk's stages are issued; longer chunks take it afterwards.
+constexpr int kEarlyTakeMaxPages = 32;
 // words of the producer's routing scratch after its copy of the routing
 // table: selections and weights [8][8] each, and an 8-word expert mask
 constexpr int kRouteTmpWords = 64 + 64 + 8;

@@ -530,8 +530,8 @@ __device__ __noinline__ int compact_routes(const Params& p, const int32_t* sel, 
 // add on a counter that every launch starts at 0), posts each in the CTA's
 // task FIFO, and streams its tiles.  A taken index past the end
 // posts a stop entry.  The next task is taken as soon as the current one is
-// posted, so the dispenser's round trip overlaps the current task's stage
-// issue (one task of lookahead per CTA).
+// posted (after a long attention chunk: once its stages are issued), so the
+// dispenser's round trip overlaps the current task's stage issue.
 __device__ __forceinline__ void prefetch_tmap(const void* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
@@ -752,9 +752,12 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       if (p.trace) p.trace[(size_t)t * kTraceWords + T_CTA] = blockIdx.x + 1;
       mbar_arrive(sm.posted(e));
     }
-    // take the next task now: its dispenser round trip overlaps this task's
-    // stage issue
-    take();
+    // take the next task now, so its dispenser round trip overlaps this
+    // task's stage issue -- except after a long attention chunk (at long
+    // contexts one chunk per CTA, hundreds of stages), where a task taken now
+    // would wait behind the chunk while other CTAs could run it
+    const bool early = op != OP_ATTN || __shfl_sync(FULL, dw, D_PPC) <= kEarlyTakeMaxPages;
+    if (early) take();
 
     // ---- stream the task's tiles
     if (op == OP_ATTN) {
@@ -849,6 +852,7 @@ __device__ __noinline__ void producer_loop(const Params& p) {
       }
       if (fail) break;
     }
+    if (!early) take();
     if (lane == 0) {
       stamp(p, t, T_P_ISSUED);
       trace_put(p, t, T_P_WAITCYC, pwait);
