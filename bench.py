@@ -37,10 +37,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "dcc4fdbe32d5bd2125ff58a936a103ebeaabda4e295e184041a900bfa7927630",
+    "kernel_sha256": "1c7f39e1bf21a42f09b2c9ea835884ddc50b19535999040a2f5099e808755c1d",
     "workload": "moe30b_b1",
-    "fixed_bytes": 622.74e6,
-    "per_layer_bytes": 114.36e6,
+    "fixed_bytes": 622.91e6,
+    "per_layer_bytes": 114.31e6,
 }
 
 
