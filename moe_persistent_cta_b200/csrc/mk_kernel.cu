@@ -1498,13 +1498,13 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   }
   const int key8 = 8 * cw;
   const int krow = key8 + (lane & 7);
+  Ring ring;   // K and V stages alternate; the position advances without a division
+  ring.init(stage_ctr, sm.NS);
   for (int pi = 0; pi < np; ++pi) {
     // ---- K page: scores of this warp's 8 keys for the G heads
-    uint32_t slot = stage_ctr % sm.NS;
-    uint32_t ph = (stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm.full(slot), ph, 401);
+    wait_bar(p, sm.full(ring.slot), ring.phase, 401);
     __syncwarp();
-    uint32_t kb = saddr(sm.ring + (size_t)slot * kStageBytes);
+    const uint32_t kb = saddr(sm.ring + (size_t)ring.slot * kStageBytes);
     float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t kr[HD / 32][4];
 #pragma unroll
@@ -1516,7 +1516,8 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
               kr[k2][2], kr[k2][3]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(slot));
+    if (lane == 0) mbar_arrive(sm.empty(ring.slot));
+    ring.next();
     ++stage_ctr;
 #pragma unroll
     for (int k2 = 0; k2 < HD / 32; ++k2) {
@@ -1560,11 +1561,9 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
       acc[j][1] *= my_alpha;
     }
     // ---- V page: acc += P V
-    slot = stage_ctr % sm.NS;
-    ph = (stage_ctr / sm.NS) & 1;
-    wait_bar(p, sm.full(slot), ph, 402);
+    wait_bar(p, sm.full(ring.slot), ring.phase, 402);
     __syncwarp();
-    const uint32_t vb = saddr(sm.ring + (size_t)slot * kStageBytes);
+    const uint32_t vb = saddr(sm.ring + (size_t)ring.slot * kStageBytes);
 #pragma unroll
     for (int j4 = 0; j4 < HD / 32; ++j4) {
       const int hd0 = j4 * 32;
@@ -1578,7 +1577,8 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
       mma1688(acc[4 * j4 + 3], pa, 0u, b3);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(slot));
+    if (lane == 0) mbar_arrive(sm.empty(ring.slot));
+    ring.next();
     ++stage_ctr;
   }
   if (ct == 0) stamp(p, ent[32 + R_TASK], T_C_MATH);
