@@ -51,9 +51,12 @@ constexpr int kLocalRouteMaxB = 4;
 // Attention chunks of up to this many pages let their CTA take its next task
 // before the chunk's stages are issued; longer chunks take it afterwards.
 constexpr int kEarlyTakeMaxPages = 32;
+// expert bitmasks of the routing compaction: the union (8 words, E <= 256),
+// then one per token
+constexpr int kRouteMaskWords = 8 + 8 * kMaxBatch;
 // words of the producer's routing scratch after its copy of the routing
-// table: selections and weights [8][8] each, and an 8-word expert mask
-constexpr int kRouteTmpWords = 64 + 64 + 8;
+// table: selections and weights [8][8] each, and the expert bitmasks
+constexpr int kRouteTmpWords = 64 + 64 + kRouteMaskWords;
 // Per-layer pointer table in shared memory: norm weights of levels 0..L (the
 // final norm last), then router bias, K pool and V pool of layers 0..L-1.  A
 // task reads its layer's pointers from there, so its first global loads need

@@ -468,16 +468,21 @@ __device__ __noinline__ void token_route(const Params& p, const float* bias, int
 // union of selected experts in ascending id becomes slots 0 .. n_used - 1,
 // each with its tokens in ascending order, their ranks and weights; slots
 // past n_used hold expert -1.  rt may be shared or global memory; mask is
-// 8 words of shared scratch.  Returns n_used.
+// kRouteMaskWords words of shared scratch: the union's bitmask, then each
+// token's own expert bitmask (a token's position in a slot is the number of
+// earlier tokens whose bitmask holds the expert).  Returns n_used.
 __device__ __noinline__ int compact_routes(const Params& p, const int32_t* sel, const float* w,
                                            uint32_t* mask, int32_t* rt) {
   const int lane = threadIdx.x & 31;
   const int B = p.B, K = p.k, S = p.S, BK = B * K;
-  if (lane < 8) mask[lane] = 0u;
+  uint32_t* tokmask = mask + 8;   // [B][8]
+  for (int i = lane; i < 8 + 8 * B; i += 32) mask[i] = 0u;
   __syncwarp();
   for (int q = lane; q < BK; q += 32) {
-    const int e = sel[(q / K) * 8 + q % K];
+    const int b = q / K;
+    const int e = sel[b * 8 + q - b * K];
     atomicOr(&mask[e >> 5], 1u << (e & 31));
+    atomicOr(&tokmask[b * 8 + (e >> 5)], 1u << (e & 31));
   }
   __syncwarp();
   uint32_t m[8];
@@ -502,21 +507,22 @@ __device__ __noinline__ int compact_routes(const Params& p, const int32_t* sel, 
     int s = __popc(m[e >> 5] & ((1u << (e & 31)) - 1u));
 #pragma unroll
     for (int i = 0; i < 8; ++i) s += (i < (e >> 5)) ? __popc(m[i]) : 0;
-    // position among the slot's tokens: earlier tokens that selected e
-    int pos = 0;
-#pragma unroll 1
-    for (int b2 = 0; b2 < b; ++b2)
-#pragma unroll 1
-      for (int j2 = 0; j2 < K; ++j2) pos += (sel[b2 * 8 + j2] == e);
+    // position among the slot's tokens (earlier tokens that selected e) and,
+    // for the first of them, the slot's token count
+    const uint32_t bit = 1u << (e & 31);
+    int pos = 0, cnt = 0;
+#pragma unroll
+    for (int b2 = 0; b2 < kMaxBatch; ++b2) {
+      if (b2 < B) {
+        const int hit = (tokmask[b2 * 8 + (e >> 5)] & bit) ? 1 : 0;
+        if (b2 < b) pos += hit;
+        else cnt += hit;
+      }
+    }
     rt[route_slot_tok(B, K, S) + s * 8 + pos] = b;
     rt[route_slot_rank(B, K, S) + s * 8 + pos] = j;
     reinterpret_cast<float*>(rt)[route_slot_w(B, K, S) + s * 8 + pos] = wt;
     if (pos == 0) {
-      int cnt = 0;
-#pragma unroll 1
-      for (int b2 = b; b2 < B; ++b2)
-#pragma unroll 1
-        for (int j2 = 0; j2 < K; ++j2) cnt += (sel[b2 * 8 + j2] == e);
       rt[route_slot_expert(B, K) + s] = e;
       rt[route_slot_ntok(B, K, S) + s] = cnt;
     }
@@ -1918,8 +1924,8 @@ __device__ __noinline__ void topk_task(const Params& p, int l) {
   const uint32_t par = p.epoch & 1u;
   int32_t* sel = reinterpret_cast<int32_t*>(sm.scratch);   // [8][8]
   float* wsel = reinterpret_cast<float*>(sel + 64);          // [8][8]
-  uint32_t* mask = reinterpret_cast<uint32_t*>(wsel + 64);   // [8]
-  int* n_used_s = reinterpret_cast<int*>(mask + 8);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(wsel + 64);   // [kRouteMaskWords]
+  int* n_used_s = reinterpret_cast<int*>(mask + kRouteMaskWords);
   if (cw < B)
     token_route(p, router_b(p, sm, l), l, par, cw, sel + cw * 8, wsel + cw * 8,
                 p.rlogits + ((size_t)l * B + cw) * E);

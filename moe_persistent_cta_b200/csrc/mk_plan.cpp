@@ -97,7 +97,7 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->actB_bytes = round_up(b_need, 128);
   int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
-  int sc_topk = (64 + 64 + 8 + 1) * 4;                            // selections, weights, mask
+  int sc_topk = (64 + 64 + kRouteMaskWords + 1) * 4;              // selections, weights, masks
   int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
   int sc_comb = 256 * 16 + kMaxAttnOut * 4 + 3 * max_chunks * G * 4 + 2 * G * 4 + 256;
   int sc = std::max(std::max(sc_attn, sc_gemv), std::max(std::max(sc_topk, sc_rn), sc_comb));
