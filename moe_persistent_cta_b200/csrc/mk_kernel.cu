@@ -230,6 +230,16 @@ __device__ __forceinline__ void split3(float a, float b, uint32_t& h, uint32_t& 
   l = *reinterpret_cast<uint32_t*>(&ll);
 }
 
+// Two fp32 FMAs in one instruction (sm_100 packed fp32): (c0, c1) +=
+// (a0 * b0, a1 * b1), each rounded as fma.rn.f32.
+__device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%0, %1};\n\t"
+      "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // -------------------------------------------------------------- state -----
 extern __shared__ uint8_t g_smem[];
 __shared__ int g_abort;   // this CTA's abort flag
@@ -1074,7 +1084,8 @@ struct Ring {
 
 // CUDA-core stage loop for 1 or 2 activation columns (partial rows of pc
 // floats): exact fp32 FMAs of bf16 weights (widened by a shift/mask) with fp32
-// activations.  Lane l reads
+// activations, two per instruction (ffma2): each row keeps the sums of its even
+// and odd columns, added at the end.  Lane l reads
 // 16-byte chunk (l & 7) of rows (l >> 3) + 4i of its warp's 16-row unit, so a
 // warp's 32 lanes cover the unit's 512 bytes per row group without bank
 // conflicts; partial sums are reduced over the 8 lanes of a row at the end.
@@ -1086,11 +1097,11 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
                                                  uint32_t& waitcyc, int pc) {
   MK_CONSUMER_IDS;
   const int c = lane & 7, rg = lane >> 3;
-  float acc[4][NB];
+  float acc[4][NB], acc_odd[4][NB];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int b = 0; b < NB; ++b) acc[i][b] = 0.f;
+    for (int b = 0; b < NB; ++b) acc[i][b] = acc_odd[i][b] = 0.f;
   uint32_t woff[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -1125,16 +1136,13 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
     for (int i = 0; i < 4; ++i) {
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        float a = acc[i][b];
-        a = fmaf(lo_bf16(w[i].x), xa[b].x, a);
-        a = fmaf(hi_bf16(w[i].x), xa[b].y, a);
-        a = fmaf(lo_bf16(w[i].y), xa[b].z, a);
-        a = fmaf(hi_bf16(w[i].y), xa[b].w, a);
-        a = fmaf(lo_bf16(w[i].z), xb[b].x, a);
-        a = fmaf(hi_bf16(w[i].z), xb[b].y, a);
-        a = fmaf(lo_bf16(w[i].w), xb[b].z, a);
-        a = fmaf(hi_bf16(w[i].w), xb[b].w, a);
-        acc[i][b] = a;
+        float e = acc[i][b], o = acc_odd[i][b];
+        ffma2(e, o, lo_bf16(w[i].x), hi_bf16(w[i].x), xa[b].x, xa[b].y);
+        ffma2(e, o, lo_bf16(w[i].y), hi_bf16(w[i].y), xa[b].z, xa[b].w);
+        ffma2(e, o, lo_bf16(w[i].z), hi_bf16(w[i].z), xb[b].x, xb[b].y);
+        ffma2(e, o, lo_bf16(w[i].w), hi_bf16(w[i].w), xb[b].z, xb[b].w);
+        acc[i][b] = e;
+        acc_odd[i][b] = o;
       }
     }
   }
@@ -1142,7 +1150,7 @@ __device__ __forceinline__ void gemv_stages_ffma(const Params& p, const Smem& sm
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      float a = acc[i][b];
+      float a = acc[i][b] + acc_odd[i][b];
       a += __shfl_xor_sync(FULL, a, 1);
       a += __shfl_xor_sync(FULL, a, 2);
       a += __shfl_xor_sync(FULL, a, 4);

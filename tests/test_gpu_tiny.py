@@ -214,6 +214,44 @@ def test_zipf_routing_batch8():
         rig.close()
 
 
+def test_all_tokens_share_their_experts():
+    """Every token of a batch of 8 routes to the same 8 experts (a router bias
+    of 30 on a per-layer set of 8 of 64 experts, far above the logits'
+    spread): each used slot holds all 8 tokens, the most a slot can hold, so
+    the routing compaction places tokens at positions 0..7 and counts 8 per
+    slot.  The step matches the oracle and every layer uses exactly 8 slots."""
+    from moe_persistent_cta_b200 import synth
+    shape = dict(configs.TINY, n_experts=64, top_k=8)
+    W = synth.make_weights(shape, 11, "cpu", "uniform")
+    gen = torch.Generator().manual_seed(12)
+    biased = []
+    W["router_bias"] = []
+    for _ in range(shape["n_layers"]):
+        chosen = torch.randperm(64, generator=gen)[:8]
+        b = torch.zeros(64, dtype=torch.float32)
+        b[chosen] = 30.0
+        W["router_bias"].append(b)
+        biased.append(set(chosen.tolist()))
+    lens = [100, 200, 300, 400, 500, 600, 700, 800]
+    rig = TinyRig(shape, lens, seed=11, weights=W)
+    try:
+        got = rig.step()
+        rec = {}
+        ref = rig.oracle_step(record=rec)
+        err, rel = compare_logits(got, ref)
+        assert err <= TIGHT and rel <= REL_L2, (err, rel)
+        L, B, K = shape["n_layers"], len(lens), 8
+        nslots = rig.dec.debug(mk.MK_BUF_NSLOTS)
+        ids = rig.dec.debug(mk.MK_BUF_TOPK)[: L * B * K].reshape(L, B, K)
+        for l in range(L):
+            assert nslots[l] == 8, (l, nslots[l])
+            for b in range(B):
+                assert set(ids[l, b].tolist()) == biased[l], (l, b)
+                assert set(rec[(l, b)]["topk_idx"].tolist()) == biased[l], (l, b)
+    finally:
+        rig.close()
+
+
 def test_greedy_16_steps():
     """16 greedy steps: identical tokens, logits within tolerance each step,
     the GPU appending K/V into its own pool and the oracle into its copy."""
