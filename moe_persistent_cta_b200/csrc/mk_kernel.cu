@@ -346,12 +346,6 @@ __device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_
   }
 }
 
-__device__ __forceinline__ bool wait_counter(const Params& p, int ctr, uint32_t target, int task,
-                                             int op) {
-  if (reached(ld_acquire(p.counters + ctr), target)) return true;
-  return wait_counter_slow(p, ctr, target, task, op);
-}
-
 // Bounded wait on a shared-memory mbarrier phase (every calling lane): the
 // common already-complete case inline, the spin out of line.
 __device__ __noinline__ bool wait_bar_slow(const Params& p, uint32_t bar, uint32_t parity,
@@ -399,10 +393,6 @@ __device__ __forceinline__ void trace_put(const Params& p, int task, int field, 
 }
 __device__ __forceinline__ void cstamp(const Params& p, int task, int field) {
   if (p.trace) p.trace[(size_t)task * kTraceWords + field] = (uint32_t)clock64();
-}
-
-__device__ __forceinline__ const void* tmap(const Params& p, int idx) {
-  return static_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
 }
 
 // ================================================================ routing ==
