@@ -37,10 +37,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "af2c93e479a09e76eca0b3d6cd39a72feaba36e0ce4a2133e8e8def837c66bce",
+    "kernel_sha256": "8904b5c4689deb7f8009270e05b934f0f507bfac6de61533aae43aed29ee7f79",
     "workload": "moe30b_b1",
-    "fixed_bytes": 623.04e6,
-    "per_layer_bytes": 114.31e6,
+    "fixed_bytes": 623.42e6,
+    "per_layer_bytes": 114.26e6,
 }
 
 
