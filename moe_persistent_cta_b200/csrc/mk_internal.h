@@ -29,9 +29,19 @@ constexpr int kConsumerWarps = 8;
 constexpr int kProducerWarp = 0;     // TMA weight/KV streamer + task resolver
 constexpr int kLoaderWarp = 1;       // dependency waits + activation loads
 constexpr int kSignalWarp = 2;       // completion signals (release adds)
-constexpr int kFirstConsumerWarp = 3;
-constexpr int kEpilogueWarp = kFirstConsumerWarp + kConsumerWarps;   // 11
-constexpr int kThreads = (kEpilogueWarp + 1) * 32;                    // 384
+constexpr int kEpilogueWarp = 3;     // GEMV partial reduction and outputs
+constexpr int kFirstConsumerWarp = 4;   // warps 4..11: two whole warpgroups
+constexpr int kThreads = (kFirstConsumerWarp + kConsumerWarps) * 32;   // 384
+// Registers per thread after the split (setmaxnreg) of the launch's
+// kThreads x 168 = 64,512: warpgroup 0 (the single-warp roles) keeps
+// kRoleRegs, the consumers get kConsumerRegs, 63,488 in all.  A split above
+// the launch's registers would leave the increase waiting forever.
+constexpr int kRoleRegs = 80;
+constexpr int kConsumerRegs = 208;
+static_assert(128 * kRoleRegs + 256 * kConsumerRegs <= kThreads * 168,
+              "register split exceeds the launch's registers");
+static_assert(kRoleRegs % 8 == 0 && kConsumerRegs % 8 == 0 && kConsumerRegs <= 256,
+              "setmaxnreg takes multiples of 8 up to 256");
 constexpr int kRstdRing = 4;         // per-level 1/rms slots (levels in flight)
 constexpr int kMaxParts = 1 + 16 + kMaxTopK;   // residual + O-proj groups + expert ranks
 constexpr int kFifo = 16;            // task entries in flight per CTA

@@ -19,11 +19,19 @@
 //                      vector into shared memory.
 //   warp 2 (signaler)  after the consumers finish a task, publishes it with a
 //                      release add on each of the task's counters.
-//   warps 3..10        compute: mma.sync bf16 tiles (weights as the 16-row A
+//   warp 3 (epilogue)  reduces the consumer warps' GEMV partial sums and
+//                      writes the tile's outputs.
+//   warps 4..11        compute: exact fp32 FMAs for one or two token columns,
+//                      else mma.sync bf16 tiles (weights as the 16-row A
 //                      operand read from the swizzled TMA tile with ldmatrix,
 //                      fp32 activations as the 8-column B operand split into
 //                      three bf16 terms, so the product keeps ~24 bits),
-//                      attention with an online softmax, and the epilogues.
+//                      attention with an online softmax, norm and top-k.
+// Warpgroup 0 (warps 0..3) gives registers to the two consumer warpgroups
+// (setmaxnreg: 80 and 208 per thread, from the 168 the launch holds).  Every
+// routine is inlined into the kernel so that ptxas budgets each warpgroup's
+// code on its own: an out-of-line function is compiled for the launch's 168
+// and holds every caller to it.
 // Every wait is bounded by a deadline counted in SM clock cycles (clock64; the
 // host converts the millisecond limit at the device's peak SM clock); on expiry
 // the CTA latches an error in the status word, raises the abort flag and
@@ -307,7 +315,7 @@ __device__ __forceinline__ Smem smem_view(const Params& p) {
 __device__ __forceinline__ bool aborted() { return *(volatile int*)&g_abort != 0; }
 __device__ __forceinline__ void set_abort() { *(volatile int*)&g_abort = 1; }
 
-__device__ __noinline__ void raise_error(const Params& p, int code, int task, int op, int ctr, uint32_t obs,
+__device__ __forceinline__ void raise_error(const Params& p, int code, int task, int op, int ctr, uint32_t obs,
                             uint32_t tgt, int aux) {
   if (atomicCAS(&p.status[ST_CODE], 0, code) == 0) {
     p.status[ST_CTA] = blockIdx.x;
@@ -323,7 +331,7 @@ __device__ __noinline__ void raise_error(const Params& p, int code, int task, in
 }
 
 // Bounded spin on a global counter (one lane).
-__device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_t target,
+__device__ __forceinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_t target,
                                                int task, int op) {
   const uint32_t* c = p.counters + ctr;
   uint32_t v;
@@ -347,8 +355,8 @@ __device__ __noinline__ bool wait_counter_slow(const Params& p, int ctr, uint32_
 }
 
 // Bounded wait on a shared-memory mbarrier phase (every calling lane): the
-// common already-complete case inline, the spin out of line.
-__device__ __noinline__ bool wait_bar_slow(const Params& p, uint32_t bar, uint32_t parity,
+// common already-complete case first, then the bounded spin.
+__device__ __forceinline__ bool wait_bar_slow(const Params& p, uint32_t bar, uint32_t parity,
                                            int aux) {
   const uint64_t t0 = clock64();
   for (;;) {
@@ -376,7 +384,7 @@ __device__ __forceinline__ bool warp_wait(const Params& p, uint32_t bar, uint32_
 }
 
 // Wait for a phase that is known to complete (copies in flight), bounded.
-__device__ __noinline__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void drain_bar(const Params& p, uint32_t bar, uint32_t parity) {
   const uint64_t t0 = clock64();
   while (!mbar_wait_hint(bar, parity)) {
     if ((uint64_t)clock64() - t0 > p.timeout_cycles) break;
@@ -411,7 +419,7 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // expert id ascending on ties) into sel[0..k) and the softmax over the k
 // selected logits into w[0..k) (shared memory).  logits (may be null)
 // receives the token's E logits.  Lane-parallel over experts (E <= 256).
-__device__ __noinline__ void token_route(const Params& p, const float* bias, int l, uint32_t par,
+__device__ __forceinline__ void token_route(const Params& p, const float* bias, int l, uint32_t par,
                                          int b, int32_t* sel, float* w, float* logits) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.k;
@@ -471,7 +479,7 @@ __device__ __noinline__ void token_route(const Params& p, const float* bias, int
 // kRouteMaskWords words of shared scratch: the union's bitmask, then each
 // token's own expert bitmask (a token's position in a slot is the number of
 // earlier tokens whose bitmask holds the expert).  Returns n_used.
-__device__ __noinline__ int compact_routes(const Params& p, const int32_t* sel, const float* w,
+__device__ __forceinline__ int compact_routes(const Params& p, const int32_t* sel, const float* w,
                                            uint32_t* mask, int32_t* rt) {
   const int lane = threadIdx.x & 31;
   const int B = p.B, K = p.k, S = p.S, BK = B * K;
@@ -559,7 +567,7 @@ __device__ __forceinline__ T in_reg(T v) {
   }
 }
 
-__device__ __noinline__ void producer_loop(const Params& p) {
+__device__ __forceinline__ void producer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   // the values the dispense/resolve/issue path reads, in registers for the
   // whole loop
@@ -889,7 +897,7 @@ __device__ __noinline__ void producer_loop(const Params& p) {
 // shared memory: the normalized input of a level into slot A (reused while
 // consecutive A-tasks read the same level; two buffers when they fit), a
 // small activation into the next of the two B buffers.
-__device__ __noinline__ void loader_loop(const Params& p) {
+__device__ __forceinline__ void loader_loop(const Params& p) {
   const Smem sm = smem_view(p);
   // the activation sources and sizes, in registers for the whole loop
   struct {
@@ -1011,7 +1019,7 @@ __device__ __noinline__ void loader_loop(const Params& p) {
 }
 
 // ============================================================== signaler ==
-__device__ __noinline__ void signal_loop(const Params& p) {
+__device__ __forceinline__ void signal_loop(const Params& p) {
   const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
   uint32_t* const ctrs = in_reg(p.counters);
@@ -1320,7 +1328,7 @@ __device__ __forceinline__ void lm_epilogue(const EpiParams& p, const Params& pr
 // count (it has acquired every tile's keys) takes each token's key (resetting
 // it to zero for the next step) and, in a greedy step, writes the token, feeds
 // it to the next step and advances the position and length by one.
-__device__ __noinline__ void lm_finish(const Params& p, const int32_t* ent) {
+__device__ __forceinline__ void lm_finish(const Params& p, const int32_t* ent) {
   const int lane = threadIdx.x & 31;
   __syncwarp();
   int last = 0;
@@ -1721,8 +1729,8 @@ __device__ __forceinline__ void combine_task(const Params& p, const int32_t* ent
 
 // RoPE cos/sin of this step's positions (angle in double: a 262144-token
 // position loses ~0.03 rad in fp32), plus the position check.  Runs once per
-// step, out of line.
-__device__ __noinline__ void rope_table(const Params& p, int task) {
+// step.
+__device__ __forceinline__ void rope_table(const Params& p, int task) {
   MK_CONSUMER_IDS;
   const int half = p.hd / 2;
   for (int t = ct; t < p.B * half; t += 256) {
@@ -1751,7 +1759,7 @@ __device__ __noinline__ void rope_table(const Params& p, int task) {
 // ring when it hands the task out (128 expert rows of 128 bytes per stage,
 // 128-byte swizzled), so they are resident before the inputs are.  Returns
 // the advanced ring counter.
-__device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, uint32_t stage_ctr) {
+__device__ __forceinline__ uint32_t rn_task(const Params& p, const int32_t* ent, uint32_t stage_ctr) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int l = ent[D_LAYER], r = ent[D_A];
@@ -1915,7 +1923,7 @@ __device__ __noinline__ uint32_t rn_task(const Params& p, const int32_t* ent, ui
 // route locally) and by the debug reads.  It also stands in for the signals
 // of the unused slots' tiles and zeroes the other step parity's accumulators
 // of the layer for the next step.
-__device__ __noinline__ void topk_task(const Params& p, int l) {
+__device__ __forceinline__ void topk_task(const Params& p, int l) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   const int B = p.B, E = p.E, S = p.S, NR = p.NR;
@@ -1955,7 +1963,7 @@ __device__ __noinline__ void topk_task(const Params& p, int l) {
 // HD: the head dimension.  Each launch runs the instantiation of its batch and
 // shape, so its consumer code holds one GEMV path and one attention routine.
 template <int NBK, int HD>
-__device__ __noinline__ void consumer_loop(const Params& p) {
+__device__ __forceinline__ void consumer_loop(const Params& p) {
   const Smem sm = smem_view(p);
   MK_CONSUMER_IDS;
   uint32_t stage_ctr = 0, ngemv = 0;
@@ -2088,7 +2096,7 @@ __device__ __noinline__ void consumer_loop(const Params& p) {
 // for the consumer warps' partials, reduces them, writes the outputs and
 // completes the task (partials buffer, B activation buffer, done); every
 // entry it passes is released to the producer together with the signaler.
-__device__ __noinline__ void epilogue_loop(const Params& p) {
+__device__ __forceinline__ void epilogue_loop(const Params& p) {
   const Smem sm = smem_view(p);
   const int lane = threadIdx.x & 31;
   const int PC = p.part_cols;
@@ -2179,15 +2187,21 @@ __global__ void __launch_bounds__(kThreads, 1) mk_interp(const __grid_constant__
     }
   }
   __syncthreads();
-  if (warp == kProducerWarp) {
-    producer_loop(p);
-  } else if (warp == kLoaderWarp) {
-    loader_loop(p);
-  } else if (warp == kSignalWarp) {
-    signal_loop(p);
-  } else if (warp == kEpilogueWarp) {
-    epilogue_loop(p);
+  if (warp < kFirstConsumerWarp) {
+    // warpgroup 0 releases registers first; each consumer warpgroup's
+    // increase waits until the CTA's pool holds them
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRoleRegs));
+    if (warp == kProducerWarp) {
+      producer_loop(p);
+    } else if (warp == kLoaderWarp) {
+      loader_loop(p);
+    } else if (warp == kSignalWarp) {
+      signal_loop(p);
+    } else {
+      epilogue_loop(p);
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
     consumer_loop<NBK, HD>(p);
   }
   __syncthreads();
@@ -2229,8 +2243,15 @@ cudaError_t launch_interp(const Params& p, int grid, cudaStream_t stream) {
   KernelSlot& k = kernel_for(p.B, p.hd);
   int* conf = configured_entry(k);
   if (!conf || *conf != p.smem_bytes) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+    // the register split needs the registers it hands out: a build whose
+    // launch holds fewer would leave the consumers' increase waiting forever,
+    // so it is refused here instead of launched
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, k.fn);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs * kThreads < 128 * kRoleRegs + 256 * kConsumerRegs)
+      return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
     if (e != cudaSuccess) return e;
     if (conf) *conf = p.smem_bytes;
   }
