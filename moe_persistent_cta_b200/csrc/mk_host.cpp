@@ -462,6 +462,7 @@ mk_status mk_build_schedule(mk_ctx* c, int batch, const int32_t* seq_lens,
   p.off_bars = sl.off_bars;
   p.off_fifo = sl.off_fifo;
   p.off_scratch = sl.off_scratch;
+  p.attn_in_actB = sl.attn_in_actB;
   p.off_actA = sl.off_actA;
   p.off_actB = sl.off_actB;
   p.actB_bytes = sl.actB_bytes;

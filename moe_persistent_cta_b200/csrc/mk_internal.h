@@ -51,7 +51,7 @@ constexpr int kMapRouter = 2;
 // Activation rows are padded by 8 floats so that the 8 columns a warp reads
 // at one k land in different shared-memory banks.
 constexpr int kActPad = 8;
-constexpr int kRnStage = 4096;       // floats of residual partials staged per round
+constexpr int kRnStage = 1536;       // floats of the norm tile's staging area (group sums, gamma x, part pointers)
 constexpr int kRouterRowsPerStage = 128;   // router weight rows (x 64 columns) per ring stage
 constexpr int kMaxAttnOut = 512;    // G x hd floats of one (token, KV head) output (G <= 4, hd <= 128)
 // Batch sizes up to which each producer computes a layer's routing table
@@ -242,6 +242,10 @@ struct Params {
   // shared-memory layout (byte offsets from the 1024-aligned base)
   int n_stages, nA, actA_stride;
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, actB_bytes, off_ring;
+  // 1: an attention chunk keeps its per-warp merge area and rotated query in
+  // its own B buffer, after the chunk's inputs (when the buffer has the room);
+  // 0: in the scratch area
+  int attn_in_actB;
   int off_epi;       // GEMV partials [2][kConsumerWarps][16][part_cols], then the
                      // per-level 1/rms ring [kRstdRing][kMaxBatch]
   int off_ptrs;      // per-layer pointer table, copied in at launch (see PtrTable)
@@ -309,6 +313,7 @@ struct SmemLayout {
   int actA_stride;    // bytes per A buffer
   int actB_bytes;     // bytes per small-activation buffer (two of them)
   int scratch_bytes;
+  int attn_in_actB;   // see Params
   int n_stages;       // ring stages of kStageBytes
   int off_bars, off_fifo, off_scratch, off_actA, off_actB, off_ring, off_epi, off_ptrs;
   int off_rcache;

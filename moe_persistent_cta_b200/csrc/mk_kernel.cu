@@ -1433,7 +1433,9 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   const float* k_raw = q_raw + G * HD;
   const float* v_raw = k_raw + HD;
   const float* csv = v_raw + HD;
-  float* mrg = reinterpret_cast<float*>(sm.scratch);       // [8][G][HD+4]
+  float* mrg = p.attn_in_actB                              // [8][G][HD+4]
+                   ? reinterpret_cast<float*>(const_cast<uint8_t*>(act) + (G + 3) * HD * 4)
+                   : reinterpret_cast<float*>(sm.scratch);
   float* qs = mrg + 8 * G * (HD + 4);                      // [G][HD]
   float* kn = qs + G * HD;                                 // [HD]
   float* vn = kn + HD;                                     // [HD]

@@ -95,7 +95,12 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   int b_need = std::max(4 * (G * s.hd + kActPad) * B,
                         std::max(4 * (s.F + kActPad) * B, (G + 3) * s.hd * 4));
   o->actB_bytes = round_up(b_need, 128);
-  int sc_attn = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4 + 256;
+  // attention's working area: the 8 warps' partial outputs, the rotated query
+  // and the new token's K and V; in the chunk's own B buffer, after its inputs
+  // (G + 3 rows of hd floats), where that buffer has the room (batch > 2)
+  const int attn_work = 8 * G * (s.hd + 4) * 4 + G * s.hd * 4 + 2 * s.hd * 4;
+  o->attn_in_actB = (G + 3) * s.hd * 4 + attn_work <= o->actB_bytes ? 1 : 0;
+  int sc_attn = o->attn_in_actB ? 0 : attn_work + 256;
   int sc_gemv = 8 * 512 + 1024 * 4 + 64;
   int sc_topk = (64 + 64 + kRouteMaskWords + 1) * 4;              // selections, weights, masks
   int sc_rn = (kMaxBatch * 64 + kRnStage) * 4 + 64;
@@ -108,10 +113,12 @@ int smem_layout(const Shape& s, int B, int max_chunks, SmemLayout* o) {
   o->part_cols = B <= 2 ? B : 8;
   const int epi = round_up(2 * kConsumerWarps * 16 * o->part_cols * 4 + kRstdRing * kMaxBatch * 4,
                            128);
-  const int budget = 232448 - 2048;   // max per block, less alignment slack and static smem
+  const int budget = 232448 - 1040;   // max per block, less the alignment pad and static smem
   const int ptrs = round_up(ptr_table_words(s.L) * 8, 128);
-  const int rcache =
-      round_up((route_words(B, s.k, std::min(s.E, B * s.k)) + kRouteTmpWords) * 4, 128);
+  // the routing table copy, plus the producer's own routing scratch when it
+  // computes the table itself (B <= kLocalRouteMaxB)
+  const int rcache = round_up((route_words(B, s.k, std::min(s.E, B * s.k)) +
+                               (B <= kLocalRouteMaxB ? kRouteTmpWords : 0)) * 4, 128);
   int rest1 = bars + fifo + epi + ptrs + rcache + o->scratch_bytes + o->actA_stride +
               2 * o->actB_bytes;
   int rest2 = rest1 + o->actA_stride;
