@@ -37,10 +37,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "e41829350a2ab10ca5e403fb79fb0b2f661f8ecd9f9086c94ac503178bb64534",
+    "kernel_sha256": "dd8497981e9fd0583536fb71491a47bb606f8ec1f62ea506cef957152422d195",
     "workload": "moe30b_b1",
-    "fixed_bytes": 623.12e6,
-    "per_layer_bytes": 114.26e6,
+    "fixed_bytes": 623.17e6,
+    "per_layer_bytes": 114.31e6,
 }
 
 
