@@ -292,7 +292,8 @@ size_t mk_debug_size(mk_ctx* ctx, int which);
  * run time every CTA takes the next task with an atomic add.
  *   meta (HOST int32[16]) receives {n_tasks, n_counters, n_slots, max_chunks,
  *   desc_words, n_phases, qkv_rows_per_tile, pages_per_chunk, dispenser
- *   counter, first phase dispenser counter, 0...}.
+ *   counter, first phase dispenser counter, ring stages per CTA, 1 if an
+ *   attention chunk works in its own activation buffer (else 0), 0...}.
  *   desc (HOST int32[n_tasks][desc_words] or NULL) receives the descriptors;
  *   pass NULL first to learn n_tasks from meta.
  *   targets (HOST int32[n_counters] or NULL) receives each counter's

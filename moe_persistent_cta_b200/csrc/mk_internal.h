@@ -290,6 +290,7 @@ struct Shape {
 
 struct Plan {
   int n_ctas = 0, B = 0, S = 0, max_chunks = 1, n_counters = 0, n_tasks = 0;
+  int n_stages = 0, attn_in_actB = 0;   // from the shared-memory layout
   int n_phases = 0;
   int r_qkv = 16;
   int grab = 0;                      // dispenser counter of the fused list

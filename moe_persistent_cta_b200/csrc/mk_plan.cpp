@@ -516,7 +516,8 @@ int plan_schedule(const Shape& s, int n_ctas, int B, const int32_t* seq_lens,
   }
   if (with_phases) group_by_phase(*out, out->phase_desc);
   std::memcpy(out->targets, targets.data(), sizeof(int32_t) * n_counters);
-  (void)sl;
+  out->n_stages = sl.n_stages;
+  out->attn_in_actB = sl.attn_in_actB;
   return MK_OK;
 }
 
@@ -562,6 +563,8 @@ extern "C" mk_status mk_plan_schedule(const mk_config* cfg, int n_ctas, int batc
   meta[7] = p.ppc[0];
   meta[8] = p.grab;
   meta[9] = p.grab_phase0;
+  meta[10] = p.n_stages;
+  meta[11] = p.attn_in_actB;
   if (desc) std::memcpy(desc, p.desc, sizeof(int32_t) * (size_t)p.n_tasks * mk::kDescWords);
   if (targets) std::memcpy(targets, p.targets, sizeof(int32_t) * p.n_counters);
   p.release();

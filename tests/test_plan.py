@@ -265,3 +265,16 @@ def test_unused_slot_tiles_can_be_skipped(lens):
         for r in (0, NR - 1):
             c = set(rows[rows[:, D_B] == r][:, D_S0].tolist())
             assert len(c) == 1 and targets[c.pop()] == S + shape["n_kv_heads"]
+
+
+def test_ring_depth_and_attention_work_area():
+    """Shared memory of the 30B shape: at batch 1 the ring holds 10 stages and
+    attention works in the scratch area; at batch 8 the 64 KB fp32
+    activation buffer leaves room for 5 stages only because an attention
+    chunk works in the rest of its own B buffer (sized for the down tiles'
+    8 x 768 floats)."""
+    m1, _, _ = engine.plan_schedule(configs.MOE30B, 148, [8192])
+    m8, _, _ = engine.plan_schedule(configs.MOE30B, 148,
+                                    [9291, 10503, 5128, 15912, 9509, 6887, 1439, 10393])
+    assert (m1[10], m1[11]) == (10, 0)
+    assert (m8[10], m8[11]) == (5, 1)
