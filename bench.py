@@ -367,6 +367,63 @@ def measure_steps(name, W, dev, steps, warmup, impl="mk", dist=None, rank=0, wor
     return out
 
 
+def measure_prefill(W, dev, steps, warmup, prefix=8192, chunk=8):
+    """Chunked prefill through the interpreter: each step feeds `chunk`
+    prompt tokens of one sequence as a prefill group (consecutive entries,
+    equal seq_lens = the cached prefix, positions prefix + 0 .. chunk - 1, one
+    page-table row), and the prefix grows by `chunk` per step.  The roofline
+    counts each byte once: the weights of the experts the step touched and the
+    prefix K/V once (the group's entries re-read the same pages)."""
+    import torch
+    from moe_persistent_cta_b200 import configs, engine, mk, synth
+    wl = configs.WORKLOADS["moe30b_b1"]
+    shape, B = dict(wl["shape"]), chunk
+    total = warmup + steps
+    row, n_pages = synth.make_page_tables([prefix], False, wl["page_seed"],
+                                          growth=chunk * total + 64)
+    table = row.repeat(B, 1)
+    k, v = synth.make_kv(shape, n_pages, wl["kv_seed"], str(dev))
+    dec = engine.Decoder(shape, W, k, v, max_batch=B, device=dev.index)
+    dec.build_schedule([prefix] * B, table.shape[1], plan_len=[prefix + chunk * total + 1] * B)
+    gen = torch.Generator(device="cpu").manual_seed(wl["token_seed"])
+    toks = torch.randint(0, shape["vocab"], (total, B), generator=gen, dtype=torch.int32)
+    lens = torch.tensor([[prefix + chunk * i] * B for i in range(total)], dtype=torch.int32)
+    pos = lens + torch.arange(B, dtype=torch.int32)
+    toks_d, lens_d, pos_d, table_d = toks.to(dev), lens.to(dev), pos.to(dev), table.to(dev)
+    logits = torch.empty((B, shape["vocab"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            dec.step(toks_d[i], pos_d[i], table_d, lens_d[i], logits, stream=stream)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(warmup, total):
+        dec.step(toks_d[i], pos_d[i], table_d, lens_d[i], logits, stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dec.check_ok()
+    ms = ev0.elapsed_time(ev1)
+    nslots = dec.debug(mk.MK_BUF_NSLOTS)
+    mid = prefix + chunk * (warmup + steps // 2)
+    res = {"metric": "prefill tok/s (prompt tokens through the fused step)",
+           "value": B * steps / (ms / 1e3), "unit": "tok/s", "ms_per_step": ms / steps,
+           "steps": steps, "warmup": warmup, "clocks": clk, "gpu_launches": steps,
+           "roofline": step_roofline(shape, [mid] + [0] * (B - 1), nslots, ms / steps),
+           "config": {"workload": f"30B-MoE shape, chunked prefill: {chunk} prompt tokens of "
+                                  f"one sequence per step after a {prefix}-token prefix "
+                                  "(shuffled pages, uniform routing)",
+                      "batch": B, "impl": "fused megakernel, one prefill group per step"}}
+    dec.close()
+    del k, v
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_greedy(name, W, dev, steps, warmup):
     """K greedy steps in one mk_decode_greedy call: the tokens, positions and
     lengths advance on the device with no host round trip between steps.
@@ -598,6 +655,8 @@ def main():
         per_config["greedy_moe30b_b1"] = measure_greedy("moe30b_b1", W, dev, args.steps,
                                                         args.warmup)
         per_config["continuous_moe30b_cb"] = measure_continuous(Wz, dev, args.cb_steps)
+        per_config["prefill_moe30b_chunk8"] = measure_prefill(W, dev, max(3, args.steps // 2),
+                                                              args.warmup)
 
     if rank == 0:
         out = {

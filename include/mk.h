@@ -133,14 +133,25 @@ mk_status mk_build_schedule(mk_ctx* ctx, int batch, const int32_t* seq_lens,
 
 /* Run one decode step on `stream` (a cudaStream_t; NULL = legacy stream).
  * Device inputs:
- *   tokens     int32[batch]    token fed to each sequence
- *   positions  int32[batch]    must equal seq_lens (checked on device)
+ *   tokens     int32[batch]    token fed to each entry
+ *   positions  int32[batch]    position of each entry's token: seq_lens[b],
+ *              or seq_lens[b] + g for the (g+1)-th token of a prefill group
  *   page_table int32[batch][max_pages_per_seq]  logical page -> physical page;
  *              the entry for page positions[b] / page_size must already be a
  *              valid page (the step writes the new K/V there)
  *   seq_lens   int32[batch]    cached tokens before the step
  * Device output:
  *   logits     float32[batch][vocab]
+ * Chunked prefill: up to `batch` consecutive prompt tokens of one sequence
+ * run as consecutive entries b0 .. b0 + M - 1 with equal seq_lens (the cached
+ * prefix, possibly 0), positions seq_lens + 0 .. M - 1 and the same
+ * page-table row.  Entry b0 + g attends to the prefix and to tokens b0 ..
+ * b0 + g (causal), so its logits are those of a decode step at its position
+ * after the tokens before it; all M tokens' K/V are appended.  Groups and
+ * single decode entries mix freely in one batch.  A position that breaks
+ * these rules (positions[b] - seq_lens[b] outside 0 .. b, or an entry whose
+ * predecessor is not the previous token of its group) stops the step with a
+ * device-side error before any attention reads out of the group.
  * Asynchronous: returns after the launch.  Returns MK_ERR_STATE before any
  * schedule was built.  Device-side errors surface through mk_check.         */
 mk_status mk_decode_step(mk_ctx* ctx, const int32_t* tokens, const int32_t* positions,
@@ -159,7 +170,8 @@ mk_status mk_decode_step(mk_ctx* ctx, const int32_t* tokens, const int32_t* posi
  * the LM head of the pages' serving loop (aimodeling.com, "Cohere megakernel
  * engine: one CUDA file, 1.58x vLLM on H100", "From demo to a full serving
  * system"), done on the device.
- *   tokens, positions, seq_lens  int32[batch], device, read and updated
+ *   tokens, positions, seq_lens  int32[batch], device, read and updated;
+ *               positions must equal seq_lens (no prefill groups)
  *   page_table  as for mk_decode_step; it must already map the page of every
  *               token the n_steps steps append
  *   logits      float32[batch][vocab], device: the last step's logits

@@ -163,6 +163,8 @@ enum ResolvedField : int {
   R_SEQLEN = 4,     // attention: cached tokens of the sequence
   R_PHYS_NEW = 5,   // attention: physical page receiving the new token
   R_TASK = 6,       // index of the task in the step's list (-1: no more tasks)
+  R_POS = 7,        // attention: position of the new token (seq_len + its index
+                    //   in a prefill group)
   R_TOK = 8,        // [8] slot token ids
   R_RANK = 16,      // [8] rank of the expert in each token's top-k
   R_W = 24          // [8] routing weight (float bits)

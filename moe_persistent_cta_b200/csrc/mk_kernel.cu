@@ -644,7 +644,7 @@ __device__ __forceinline__ void producer_loop(const Params& p) {
     }
     int32_t rw = 0;  // resolved word `lane`
     uint32_t pwait = 0;
-    int expert = -1, ntok = 0, p0 = 0, seqlen = 0, phys_new = -1;
+    int expert = -1, ntok = 0, p0 = 0, seqlen = 0, phys_new = -1, pos = 0;
     bool fail = false;
     if (op == OP_GATEUP || op == OP_DOWN) {
       const int ctr = __shfl_sync(FULL, dw, D_PW);
@@ -729,18 +729,23 @@ __device__ __forceinline__ void producer_loop(const Params& p) {
       const int nc = __shfl_sync(FULL, dw, D_D);
       const int ppc = __shfl_sync(FULL, dw, D_PPC);
       seqlen = __ldg(pp.seq_lens + b);
+      // a prefill group: entries b - grp .. b - 1 hold the tokens before this
+      // one, so the chunks read the cached prefix only
+      pos = __ldg(p.positions + b);
+      const int grp = pos - seqlen;
       const int pages_now = (seqlen + kPage - 1) / kPage;
       p0 = c * ppc;
       int np = min(ppc, pages_now - p0);
       if (np < 0) np = 0;
       const bool last = (c == nc - 1);
-      if (seqlen < 0 || (last && p0 + ppc < pages_now) || (seqlen / kPage) >= pp.max_pages) {
-        if (lane == 0) raise_error(p, MK_ERR_STATE, t, op, -1, seqlen, pages_now, b);
+      if (seqlen < 0 || grp < 0 || grp > b || (last && p0 + ppc < pages_now) ||
+          (pos / kPage) >= pp.max_pages) {
+        if (lane == 0) raise_error(p, MK_ERR_STATE, t, op, -1, seqlen, pos, b);
         set_abort();
         fail = true;
       }
       if (!fail && last) {
-        phys_new = __ldg(pp.page_table + (size_t)b * pp.max_pages + seqlen / kPage);
+        phys_new = __ldg(pp.page_table + (size_t)b * pp.max_pages + pos / kPage);
         if (phys_new < 0 || phys_new >= pp.n_pages) {
           if (lane == 0) raise_error(p, MK_ERR_DEVICE, t, op, -1, phys_new, pp.n_pages, 2);
           set_abort();
@@ -757,6 +762,7 @@ __device__ __forceinline__ void producer_loop(const Params& p) {
     if (lane == R_P0) rw = p0;
     if (lane == R_SEQLEN) rw = seqlen;
     if (lane == R_PHYS_NEW) rw = phys_new;
+    if (lane == R_POS) rw = pos;
     if (lane == R_TASK) rw = t;
     ent[lane] = dw;
     ent[32 + lane] = rw;
@@ -1425,7 +1431,7 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   const int layer = ent[D_LAYER], b = ent[D_A], g = ent[D_B], chunk = ent[D_C];
   const int flags = ent[D_FLAGS];
   const int np = ent[32 + R_NTOK], p0 = ent[32 + R_P0], seqlen = ent[32 + R_SEQLEN];
-  const int phys_new = ent[32 + R_PHYS_NEW];
+  const int phys_new = ent[32 + R_PHYS_NEW], pos = ent[32 + R_POS];
   const int G = p.G;
   const int g8 = lane >> 2, q = lane & 3;
   constexpr int HALF = HD / 2;
@@ -1459,7 +1465,7 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     kn[i] = __bfloat162float(kb);
     vn[i] = __bfloat162float(vb);
     if (flags & F_LAST_CHUNK) {
-      const size_t off = (((size_t)phys_new * p.Hkv + g) * kPage + (seqlen % kPage)) * HD + i;
+      const size_t off = (((size_t)phys_new * p.Hkv + g) * kPage + (pos % kPage)) * HD + i;
       reinterpret_cast<__nv_bfloat16*>(kpool_of(p, sm, layer))[off] = kb;
       reinterpret_cast<__nv_bfloat16*>(vpool_of(p, sm, layer))[off] = vb;
     }
@@ -1492,7 +1498,10 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   float acc[HD / 8][4];
 #pragma unroll
   for (int j = 0; j < HD / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  // the new token joins the softmax of the chunk that owns it (warp 0)
+  // The new token joins the softmax of the chunk that owns it (warp 0).  In
+  // a prefill group so do the group's earlier tokens, which are not in the
+  // pool yet: their K (rotated at their own positions) and V come from this
+  // step's QKV output, rounded to bf16 as the pool stores them.
   if ((flags & F_LAST_CHUNK) && cw == 0) {
     float sn[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i = lane; i < HD; i += 32)
@@ -1507,6 +1516,41 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
       for (int j = 0; j < HD / 8; ++j) {
         acc[j][0] = vn[8 * j + 2 * q];
         acc[j][1] = vn[8 * j + 2 * q + 1];
+      }
+    }
+    const int grp = pos - seqlen;
+#pragma unroll 1
+    for (int j = 0; j < grp; ++j) {
+      const int bj = b - grp + j;
+      const float* kr = p.qkv + ((size_t)layer * p.B + bj) * p.qkvR + (size_t)p.Hq * HD + g * HD;
+      const float* vr = kr + (size_t)p.Hkv * HD;
+      const float* cs = p.cs + (size_t)bj * HD;
+      float sj[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = lane; i < HD; i += 32) {
+        const int i1 = i % HALF;
+        const float co = __ldcg(cs + i1), si = __ldcg(cs + HALF + i1);
+        const float x = __ldcg(kr + i);
+        const float y = __ldcg(kr + (i < HALF ? i + HALF : i - HALF));
+        const float kv = bf16r(i < HALF ? (x * co - y * si) : (x * co + y * si));
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          if (h < G) sj[h] += qs[h * HD + i] * kv;
+      }
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        for (int o = 16; o > 0; o >>= 1) sj[h] += __shfl_xor_sync(FULL, sj[h], o);
+      if (g8 < G) {
+        const float sc = g8 == 0 ? sj[0] : g8 == 1 ? sj[1] : g8 == 2 ? sj[2] : sj[3];
+        const float m_new = fmaxf(m_run, sc);
+        const float alpha = ex2(m_run - m_new), e = ex2(sc - m_new);
+        l_run = l_run * alpha + e;
+        m_run = m_new;
+#pragma unroll
+        for (int jj = 0; jj < HD / 8; ++jj) {
+          const float2 t2 = __ldcg(reinterpret_cast<const float2*>(vr + 8 * jj + 2 * q));
+          acc[jj][0] = acc[jj][0] * alpha + e * bf16r(t2.x);
+          acc[jj][1] = acc[jj][1] * alpha + e * bf16r(t2.y);
+        }
       }
     }
   }
@@ -1739,7 +1783,17 @@ __device__ __forceinline__ void rope_table(const Params& p, int task) {
     const int bb = t / half, i = t % half;
     const int pos = __ldg(p.positions + bb);
     const int sl = __ldg(p.seq_lens + bb);
-    if (pos != sl && i == 0) raise_error(p, MK_ERR_DEVICE, task, OP_RN, -1, pos, sl, 5);
+    if (i == 0) {
+      // positions == seq_lens, except in a prefill group: entry bb's
+      // position may exceed its length by g when entries bb - g .. bb - 1
+      // carry the sequence's previous tokens (same length, consecutive
+      // positions); greedy steps advance every entry alone, so none there
+      const int g = pos - sl;
+      const bool ok = g == 0 || (g > 0 && g <= bb && p.g_pos == nullptr &&
+                                 __ldg(p.seq_lens + bb - 1) == sl &&
+                                 __ldg(p.positions + bb - 1) == pos - 1);
+      if (!ok) raise_error(p, MK_ERR_DEVICE, task, OP_RN, -1, pos, sl, 5);
+    }
     double sv, cv;
     sincos((double)pos * p.inv_freq[i], &sv, &cv);
     p.cs[(size_t)bb * p.hd + i] = (float)cv;
