@@ -37,10 +37,10 @@ FALLBACK_HBM_GBS = 6650.0
 # into a per-layer and a fixed part; valid only for the kernel source it was
 # taken on (the summary sits in profiles/).  Reported as null otherwise.
 NCU_TRAFFIC = {
-    "kernel_sha256": "dd8497981e9fd0583536fb71491a47bb606f8ec1f62ea506cef957152422d195",
+    "kernel_sha256": "afbb5418b481a3e3bda55f7a313d304636120886cbe38db8a3b9c0664292c8ab",
     "workload": "moe30b_b1",
-    "fixed_bytes": 623.17e6,
-    "per_layer_bytes": 114.31e6,
+    "fixed_bytes": 622.53e6,
+    "per_layer_bytes": 114.50e6,
 }
 
 

@@ -41,20 +41,27 @@ def model():
 
 
 class Run:
-    def __init__(self, W, lens, seed=0, growth=64):
+    """One GPU step; `positions` defaults to the lengths (decode).  A prefill
+    group (positions = lengths + 0 .. M - 1) shares the first entry's
+    page-table row."""
+
+    def __init__(self, W, lens, seed=0, growth=64, positions=None):
         self.W = W
         self.lens = list(lens)
         self.B = len(lens)
+        self.pos = list(positions) if positions is not None else list(lens)
         self.dev = torch.device("cuda:0")
         self.table, self.n_pages = synth.make_page_tables(self.lens, False, seed + 3,
                                                           growth=growth)
+        if positions is not None:
+            self.table[1:] = self.table[0]
         self.k, self.v = synth.make_kv(SHAPE, self.n_pages, seed + 1, "cuda:0")
         self.tokens = synth.make_tokens(self.B, SHAPE["vocab"], seed + 2)
         self.dec = engine.Decoder(SHAPE, W, self.k, self.v, max_batch=self.B)
         self.dec.build_schedule(self.lens, self.table.shape[1])
         i32 = dict(dtype=torch.int32, device=self.dev)
         self.logits = torch.empty((self.B, SHAPE["vocab"]), dtype=torch.float32, device=self.dev)
-        self.dec.step(torch.tensor(self.tokens, **i32), torch.tensor(self.lens, **i32),
+        self.dec.step(torch.tensor(self.tokens, **i32), torch.tensor(self.pos, **i32),
                       self.table.to(self.dev), torch.tensor(self.lens, **i32), self.logits)
         self.dec.check_ok()
         L, d, E, K = SHAPE["n_layers"], SHAPE["d_model"], SHAPE["n_experts"], SHAPE["top_k"]
@@ -78,15 +85,15 @@ class Run:
         record, forced?)."""
         rec = {}
         pt = self.table[b].numpy()
-        x_out, _, _ = oracle.parallel_layer(self.S, self.WA, self.KV, l, x_in, self.lens[b], pt,
-                                            self.lens[b], rec=rec)
+        x_out, _, _ = oracle.parallel_layer(self.S, self.WA, self.KV, l, x_in, self.pos[b], pt,
+                                            self.pos[b], rec=rec)
         gpu_sel = [int(e) for e in self.ids[l, b]]
         if gpu_sel != [int(e) for e in rec["topk_idx"]]:
             gap = router_gap(rec["router_logits"], SHAPE["top_k"])
             assert gap < ROUTER_TIE, f"layer {l} token {b}: selection differs, gap {gap:.2e}"
             rec = {}
-            x_out, _, _ = oracle.parallel_layer(self.S, self.WA, self.KV, l, x_in, self.lens[b],
-                                                pt, self.lens[b], forced=gpu_sel, rec=rec)
+            x_out, _, _ = oracle.parallel_layer(self.S, self.WA, self.KV, l, x_in, self.pos[b],
+                                                pt, self.pos[b], forced=gpu_sel, rec=rec)
             return x_out, rec, True
         return x_out, rec, False
 
@@ -171,5 +178,30 @@ def test_30b_b1_256k(model):
         err, rel = compare_logits(got, ref)
         print(f"30B b1 256K: LM head from the GPU residual max-abs {err:.3e} rel-L2 {rel:.3e}")
         assert err <= 1e-3 and rel <= 1e-4
+    finally:
+        r.close()
+
+
+def test_30b_prefill_chunk8(model):
+    """Eight prompt tokens after an 8192-token prefix in one step (a prefill
+    group, as bench.py times it).  The oracle reads the KV pool as the GPU
+    step left it, so token g at position 8192 + g attends to the prefix and
+    to the group's g earlier tokens, appended by the step: every token's
+    layers 0, 24 and 47 teacher-forced, and the oracle's whole 48-layer pass
+    for the first and the last token."""
+    prefix = 8192
+    r = Run(model, [prefix] * 8, positions=[prefix + g for g in range(8)])
+    try:
+        worst = r.teacher_forced([0, 24, 47], range(8))
+        print(f"30B prefill chunk 8: teacher-forced layer max-abs {worst:.3e}")
+        for b in (0, 7):
+            ref, forced = r.whole_step(b)
+            got = r.logits[b].cpu().double().numpy()
+            err, rel = compare_logits(got, ref)
+            print(f"30B prefill token {b}: logits max-abs {err:.3e} rel-L2 {rel:.3e}, "
+                  f"forced {forced}")
+            assert err <= MAX_ABS and rel <= REL_L2
+            assert err <= LOGIT_TIGHT
+            assert int(np.argmax(got)) == int(np.argmax(ref))
     finally:
         r.close()
