@@ -409,11 +409,37 @@ def measure_prefill(W, dev, steps, warmup, prefix=8192, chunk=8):
     dec.check_ok()
     ms = ev0.elapsed_time(ev1)
     nslots = dec.debug(mk.MK_BUF_NSLOTS)
+    # e2e: the same steps again (the pool slots are overwritten with the same
+    # values) through the public API with pinned host buffers: tokens,
+    # positions, lengths and the page table in, the logits out, every step
+    h_toks, h_pos, h_lens = toks.pin_memory(), pos.pin_memory(), lens.pin_memory()
+    h_table = table.pin_memory()
+    h_logits = torch.empty((B, shape["vocab"]), dtype=torch.float32).pin_memory()
+    d_tok = torch.empty(B, dtype=torch.int32, device=dev)
+    d_pos = torch.empty(B, dtype=torch.int32, device=dev)
+    d_len = torch.empty(B, dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(warmup, total):
+            d_tok.copy_(h_toks[i], non_blocking=True)
+            d_pos.copy_(h_pos[i], non_blocking=True)
+            d_len.copy_(h_lens[i], non_blocking=True)
+            table_d.copy_(h_table, non_blocking=True)
+            dec.step(d_tok, d_pos, table_d, d_len, logits, stream=stream)
+            h_logits.copy_(logits, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dec.check_ok()
+    e2e = {"value": B * steps / (e0.elapsed_time(e1) / 1e3), "unit": "tok/s",
+           "h2d_bytes_per_step": B * 4 * 3 + table.numel() * 4,
+           "d2h_bytes_per_step": B * shape["vocab"] * 4}
     mid = prefix + chunk * (warmup + steps // 2)
     res = {"metric": "prefill tok/s (prompt tokens through the fused step)",
            "value": B * steps / (ms / 1e3), "unit": "tok/s", "ms_per_step": ms / steps,
            "steps": steps, "warmup": warmup, "clocks": clk, "gpu_launches": steps,
            "roofline": step_roofline(shape, [mid] + [0] * (B - 1), nslots, ms / steps),
+           "e2e": e2e,
            "config": {"workload": f"30B-MoE shape, chunked prefill: {chunk} prompt tokens of "
                                   f"one sequence per step after a {prefix}-token prefix "
                                   "(shuffled pages, uniform routing)",
