@@ -1060,6 +1060,9 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void sts16(uint32_t addr, unsigned short v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
 __device__ __forceinline__ float2 lds64f(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
@@ -1445,6 +1448,16 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   float* qs = mrg + 8 * G * (HD + 4);                      // [G][HD]
   float* kn = qs + G * HD;                                 // [HD]
   float* vn = kn + HD;                                     // [HD]
+  // The rotated, scaled query as the A operand of the score MMAs: a bf16
+  // tile of 8 rows x HD, rows [0, G) the hi halves and rows [G, 2G) the lo
+  // halves (the rest zero), its 16-byte chunks swizzled by row so that the
+  // page loop's ldmatrix reads are conflict-free.  It sits in the merge
+  // area, which is idle until the page loop ends.
+  const uint32_t qt = saddr(mrg);
+  auto qt_off = [](int row, int i) {
+    const int c = i >> 3;
+    return (uint32_t)(row * HD * 2 + (((c & ~7) | ((c ^ row) & 7)) << 4) + (i & 7) * 2);
+  };
   const float qscale = 1.4426950408889634f / sqrtf((float)HD);
   for (int idx = ct; idx < G * HD; idx += 256) {
     const int h = idx / HD, i = idx % HD, i1 = i % HALF;
@@ -1452,8 +1465,15 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     const float x = q_raw[h * HD + i];
     const float y = (i < HALF) ? q_raw[h * HD + i + HALF] : q_raw[h * HD + i - HALF];
     const float r = (i < HALF) ? (x * co - y * si) : (x * co + y * si);
-    qs[idx] = r * qscale;
+    const float v = r * qscale;
+    qs[idx] = v;
+    const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lb = __float2bfloat16_rn(v - __bfloat162float(hb));
+    sts16(qt + qt_off(h, i), __bfloat16_as_ushort(hb));
+    sts16(qt + qt_off(G + h, i), __bfloat16_as_ushort(lb));
   }
+  for (int idx = 2 * G * HD + ct; idx < 8 * HD; idx += 256)
+    sts16(qt + qt_off(idx / HD, idx % HD), 0);
   for (int i = ct; i < HD; i += 256) {
     const int i1 = i % HALF;
     const float co = csv[i1], si = csv[HALF + i1];
@@ -1471,29 +1491,11 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     }
   }
   cbar();
-  // Q as the A operand: rows [0,G) hi halves, rows [G,2G) lo halves
-  uint32_t qa[HD / 16][2];
-  {
-    const int row = g8;
-    const int h = row < G ? row : (row < 2 * G ? row - G : -1);
+  // this lane's ldmatrix rows of the query tile: row lane % 8, chunk
+  // 4 k2 + lane / 8 for the k2-th 32 columns (two 16-wide k steps)
+  uint32_t qaddr[HD / 32];
 #pragma unroll
-    for (int ks = 0; ks < HD / 16; ++ks) {
-      if (h < 0) {
-        qa[ks][0] = qa[ks][1] = 0u;
-      } else {
-        const float* v = qs + h * HD + ks * 16 + 2 * q;
-        float v0 = v[0], v1 = v[1], v2 = v[8], v3 = v[9];
-        if (row >= G) {
-          v0 -= bf16r(v0);
-          v1 -= bf16r(v1);
-          v2 -= bf16r(v2);
-          v3 -= bf16r(v3);
-        }
-        qa[ks][0] = pack_bf16(v0, v1);
-        qa[ks][1] = pack_bf16(v2, v3);
-      }
-    }
-  }
+  for (int k2 = 0; k2 < HD / 32; ++k2) qaddr[k2] = qt + qt_off(lane & 7, 32 * k2 + 8 * (lane >> 3));
   float m_run = -1e30f, l_run = 0.f;
   float acc[HD / 8][4];
 #pragma unroll
@@ -1560,6 +1562,10 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
   ring.init(stage_ctr, sm.NS);
   for (int pi = 0; pi < np; ++pi) {
     // ---- K page: scores of this warp's 8 keys for the G heads
+    uint32_t qa[HD / 32][4];
+#pragma unroll
+    for (int k2 = 0; k2 < HD / 32; ++k2)
+      ldsm_x4(qaddr[k2], qa[k2][0], qa[k2][1], qa[k2][2], qa[k2][3]);
     wait_bar(p, sm.full(ring.slot), ring.phase, 401);
     __syncwarp();
     const uint32_t kb = saddr(sm.ring + (size_t)ring.slot * kStageBytes);
@@ -1579,8 +1585,8 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     ++stage_ctr;
 #pragma unroll
     for (int k2 = 0; k2 < HD / 32; ++k2) {
-      mma16816(sc, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, kr[k2][0], kr[k2][1]);
-      mma16816(sd, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, kr[k2][2], kr[k2][3]);
+      mma16816(sc, qa[k2][0], 0u, qa[k2][1], 0u, kr[k2][0], kr[k2][1]);
+      mma16816(sd, qa[k2][2], 0u, qa[k2][3], 0u, kr[k2][2], kr[k2][3]);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) sc[j] += sd[j];
@@ -1640,6 +1646,7 @@ __device__ __forceinline__ uint32_t attn_task(const Params& p, const int32_t* en
     ++stage_ctr;
   }
   if (ct == 0) stamp(p, ent[32 + R_TASK], T_C_MATH);
+  cbar();   // every warp is done with the query tile in the merge area
   // ---- per-warp state -> shared memory: O = hi rows + lo rows
   float* mw = mrg + cw * G * (HD + 4);
 #pragma unroll
