@@ -263,6 +263,74 @@ def test_tiny_step_matches_library_restatement(lens, shuffled):
     assert np.allclose(got, ref, rtol=1e-9, atol=1e-9)
 
 
+def torch_reference_prefill(shape, W, k, v, row, prefix, prompt):
+    """Causal prefill of `prompt` after `prefix` cached tokens, restated in
+    batched form with torch library routines: all prompt tokens projected at
+    once, RoPE at each token's own position, and one masked
+    scaled_dot_product_attention in which token i sees the prefix and prompt
+    tokens 0 .. i.  Returns float64 logits [M][V]."""
+    L, d, Hq, Hkv, hd = (shape[x] for x in ("n_layers", "d_model", "n_q_heads", "n_kv_heads",
+                                             "head_dim"))
+    K, eps, theta = shape["top_k"], shape["rms_eps"], shape["rope_theta"]
+    M = len(prompt)
+    x = W["embed"][torch.tensor(prompt)].double()                       # [M, d]
+    pos = torch.arange(prefix, prefix + M, dtype=torch.float64)
+    inv = theta ** (-torch.arange(0, hd, 2, dtype=torch.float64) / hd)
+    rot = torch.polar(torch.ones(M, hd // 2, dtype=torch.float64), pos[:, None] * inv[None])
+    t = torch.arange(prefix)
+    pages = row[t // 64].long()
+    allowed = torch.ones(M, prefix + M, dtype=torch.bool)
+    allowed[:, prefix:] = torch.tril(torch.ones(M, M, dtype=torch.bool))
+
+    def rope(z):                                                         # [M, H, hd]
+        c = torch.complex(z[..., : hd // 2], z[..., hd // 2:]) * rot[:, None, :]
+        return torch.cat([c.real, c.imag], dim=-1)
+
+    for l in range(L):
+        n = F.rms_norm(x, (d,), weight=W["attn_norm"][l].double(), eps=eps)
+        qkv = n @ W["w_qkv"][l].double().T
+        q = rope(qkv[:, : Hq * hd].view(M, Hq, hd))
+        kk = rope(qkv[:, Hq * hd:(Hq + Hkv) * hd].view(M, Hkv, hd))
+        vv = qkv[:, (Hq + Hkv) * hd:].view(M, Hkv, hd)
+        kk = kk.float().to(torch.bfloat16).double()
+        vv = vv.float().to(torch.bfloat16).double()
+        Ks = torch.cat([k[l][pages, :, t % 64, :].double(), kk], 0).permute(1, 0, 2)[None]
+        Vs = torch.cat([v[l][pages, :, t % 64, :].double(), vv], 0).permute(1, 0, 2)[None]
+        o = F.scaled_dot_product_attention(q.permute(1, 0, 2)[None], Ks, Vs,
+                                           attn_mask=allowed, enable_gqa=True)
+        attn = o[0].permute(1, 0, 2).reshape(M, Hq * hd) @ W["w_o"][l].double().T
+        r = n @ W["w_router"][l].double().T
+        if W.get("router_bias") is not None:
+            r = r + W["router_bias"][l].double()
+        top = torch.topk(r, K, dim=1)
+        wts = torch.softmax(top.values, 1)
+        moe = torch.zeros(M, d, dtype=torch.float64)
+        for i in range(M):
+            for j in range(K):
+                e = int(top.indices[i, j])
+                g = W["w_gate"][l][e].double() @ n[i]
+                u = W["w_up"][l][e].double() @ n[i]
+                moe[i] += wts[i, j] * (W["w_down"][l][e].double() @ (F.silu(g) * u))
+        x = x + attn + moe
+    xf = F.rms_norm(x, (d,), weight=W["final_norm"].double(), eps=eps)
+    return (xf @ W["lm_head"].double().T).numpy()
+
+
+@pytest.mark.parametrize("prefix,m", [(0, 4), (61, 5), (128, 3)])
+def test_sequential_decode_is_causal_prefill(prefix, m):
+    """The prefill definition the GPU's prefill groups are checked against:
+    M decode steps in a row, each appending its token's K/V, give the logits
+    of a causal prefill of the M tokens written in batched form."""
+    shape, W, k, v, table, toks, lens = _tiny_case(lens=(prefix,), shuffled=True)
+    prompt = [int(x) for x in synth.make_tokens(m, shape["vocab"], 21)]
+    S, AW, KV = oracle_shape(shape), array_weights(W), array_kv(k, v)
+    row = table[0].numpy()
+    got = np.stack([oracle.decode_step(S, AW, KV, [prompt[j]], [prefix + j], [row],
+                                       append=True)[0] for j in range(m)])
+    ref = torch_reference_prefill(shape, W, k, v, table[0], prefix, prompt)
+    assert np.allclose(got, ref, rtol=1e-9, atol=1e-9)
+
+
 def test_layer_is_sum_of_branches():
     shape, W, k, v, table, toks, lens = _tiny_case()
     S, AW, KV = oracle_shape(shape), array_weights(W), array_kv(k, v)
