@@ -253,6 +253,23 @@ def step_roofline(shape, lens_mid, nslots, ms_per_step, n_layers_traffic=None, w
             "experts_per_layer_mean": float(np.mean(nslots))}
 
 
+def max_over_ranks(x, dist, device):
+    """The largest of the ranks' values (the slowest replica's time); the
+    value itself on one GPU."""
+    if not dist:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tok_s(world, batch, steps, ms):
+    """Whole-job throughput: the tokens all replicas decoded over the
+    slowest replica's time."""
+    return world * batch * steps / (ms / 1e3)
+
+
 def plan_launches(dec, unfused):
     """Kernel launches of one step: one for the fused step; one per operation
     phase that holds tasks for the unfused path (counted from the schedule)."""
@@ -315,15 +332,11 @@ def measure_steps(name, W, dev, steps, warmup, impl="mk", dist=None, rank=0, wor
     clk = clocks.stop() if rank == 0 else None
     dec.check_ok()
     nslots = dec.debug(mk.MK_BUF_NSLOTS)
-    ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     ms_per_step = ms / steps
     out = {"name": name, "shape": shape, "batch": B, "lens": lens, "steps": steps,
            "warmup": warmup, "ms_per_step": ms_per_step,
-           "value": world * B * steps / (ms / 1e3), "clocks": clk,
+           "value": job_tok_s(world, B, steps, ms), "clocks": clk,
            "gpu_launches": steps * plan_launches(dec, unfused)}
     mid = [s + warmup + steps // 2 for s in lens]
     out["roofline"] = step_roofline(shape, mid, nslots, ms_per_step, workload=name,
@@ -348,12 +361,8 @@ def measure_steps(name, W, dev, steps, warmup, impl="mk", dist=None, rank=0, wor
             e1.record(stream)
         torch.cuda.synchronize()
         dec.check_ok()
-        e2e_ms = e0.elapsed_time(e1)
-        if dist:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        out["e2e"] = {"value": world * B * steps / (e2e_ms / 1e3), "unit": "tok/s",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        out["e2e"] = {"value": job_tok_s(world, B, steps, e2e_ms), "unit": "tok/s",
                       "h2d_bytes_per_step": B * 4 * 2 + table.numel() * 4,
                       "d2h_bytes_per_step": B * shape["vocab"] * 4}
     out["wl"] = wl
